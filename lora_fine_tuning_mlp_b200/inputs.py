@@ -1,0 +1,161 @@
+"""Seeded synthetic inputs for the fused LoRA + SwiGLU MLP.
+
+This module only draws random numbers and rounds them to the storage formats
+(bf16, and the int4 block format of the frozen weights).  It holds none of the
+arithmetic of the MLP itself, so both the CUDA path and the CPU oracle can take
+their inputs from here without sharing any of the method.
+
+Layout (nn.Linear / PEFT convention, row-major):
+  X  [N, d]        Wg, Wu [d_ff, d]   Wd [d, d_ff]
+  Ag, Au [r, d]    Bg, Bu [d_ff, r]   Ad [r, d_ff]   Bd [d, r]
+  dOut [N, d]      (upstream gradient of the MLP output)
+
+Recipe (one numpy PCG64 generator, seed = 1234 + config index, draws in this
+order, each drawn in float32 and rounded to bf16 with round-to-nearest-even):
+  X ~ N(0, 1); Wg, Wu ~ N(0, 1/d); Wd ~ N(0, 1/d_ff)  (second argument = variance)
+  A ~ U(-1/sqrt(fan_in), +1/sqrt(fan_in)), fan_in = d for Ag, Au and d_ff for Ad
+  B ~ N(0, 0.02^2)  (std 0.02, non-zero so that every adapter gradient is exercised)
+  dOut ~ N(0, 1)
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+NAMES = ("X", "Wg", "Wu", "Wd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd", "dOut")
+WEIGHT_NAMES = ("Wg", "Wu", "Wd")
+ADAPTER_NAMES = ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")
+INT4_BLOCK = 64
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    name: str
+    N: int
+    d: int
+    d_ff: int
+    r: int
+    alpha: float
+    int4: bool = False
+    index: int = 0
+
+    @property
+    def s(self) -> float:
+        return self.alpha / self.r
+
+    @property
+    def seed(self) -> int:
+        return 1234 + self.index
+
+    def flops_fwd(self) -> float:
+        """Algorithmic forward flops: three dense projections plus the rank-r paths."""
+        return 6.0 * self.N * self.d * self.d_ff + 6.0 * self.N * self.r * (self.d + self.d_ff)
+
+    def flops_bwd(self) -> float:
+        """Algorithmic backward flops (no gradient for the frozen dense weights)."""
+        return 6.0 * self.N * self.d * self.d_ff + 12.0 * self.N * self.r * (self.d + self.d_ff)
+
+    def flops(self) -> float:
+        return self.flops_fwd() + self.flops_bwd()
+
+
+# The five workloads: a tiny one for full parity, and model-shaped ones.
+CONFIGS = (
+    Config("tiny", 512, 256, 704, 8, 16.0, index=0),
+    Config("tinyllama_mlp", 32768, 2048, 5632, 32, 32.0, index=1),
+    Config("llama3_8b_mlp", 4096, 4096, 14336, 16, 16.0, index=2),
+    Config("qwen2_7b_mlp", 8192, 3584, 18944, 64, 128.0, index=3),
+    Config("llama3_8b_mlp_int4", 4096, 4096, 14336, 16, 16.0, int4=True, index=4),
+)
+BY_NAME = {c.name: c for c in CONFIGS}
+
+
+def custom(N, d, d_ff, r, alpha, int4=False, seed_index=100, name="custom") -> Config:
+    return Config(name, N, d, d_ff, r, float(alpha), int4=int4, index=seed_index)
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit pattern (uint16), round to nearest, ties to even."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def quantize_int4(w: np.ndarray):
+    """Block-quantise a float32 [rows, cols] weight to symmetric int4.
+
+    Blocks of 64 consecutive input-dimension elements share one fp16 scale
+    equal to the block's absolute maximum (rounded to fp16).  Codes are
+    q = clamp(rint(7 * w / scale), -7, 7); an all-zero block gets scale 0 and
+    codes 0.  Packing: element 2k in the low nibble of byte k (two's
+    complement), rows packed along the input dimension.
+    Returns (packed uint8 [rows, cols/2], scales float16 [rows, cols/64]).
+    """
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    assert cols % INT4_BLOCK == 0
+    blocks = w.reshape(rows, cols // INT4_BLOCK, INT4_BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    scale16 = amax.astype(np.float16)
+    scale32 = scale16.astype(np.float32)
+    safe = np.where(scale32 > 0, scale32, np.float32(1.0))
+    q = np.rint(np.float32(7.0) * blocks / safe[:, :, None])
+    q = np.where(scale32[:, :, None] > 0, q, 0.0)
+    q = np.clip(q, -7, 7).astype(np.int8).reshape(rows, cols)
+    nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    packed = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return packed, scale16
+
+
+def make_inputs(cfg: Config) -> dict:
+    """Draw all inputs of one workload.
+
+    Returns a dict of bf16 bit arrays (uint16) keyed by NAMES.  For int4
+    workloads it also holds '<W>_q' (packed uint8) and '<W>_scale' (float16)
+    for each frozen weight; the bf16 '<W>' entry is then absent, because the
+    frozen weight only exists in its quantised form.
+    """
+    rng = np.random.Generator(np.random.PCG64(cfg.seed))
+    N, d, d_ff, r = cfg.N, cfg.d, cfg.d_ff, cfg.r
+    out = {}
+
+    def normal(shape, std):
+        return rng.standard_normal(shape, dtype=np.float32) * np.float32(std)
+
+    def uniform(shape, bound):
+        return rng.uniform(-bound, bound, size=shape).astype(np.float32)
+
+    f32 = {}
+    f32["X"] = normal((N, d), 1.0)
+    f32["Wg"] = normal((d_ff, d), 1.0 / np.sqrt(d))
+    f32["Wu"] = normal((d_ff, d), 1.0 / np.sqrt(d))
+    f32["Wd"] = normal((d, d_ff), 1.0 / np.sqrt(d_ff))
+    f32["Ag"] = uniform((r, d), 1.0 / np.sqrt(d))
+    f32["Bg"] = normal((d_ff, r), 0.02)
+    f32["Au"] = uniform((r, d), 1.0 / np.sqrt(d))
+    f32["Bu"] = normal((d_ff, r), 0.02)
+    f32["Ad"] = uniform((r, d_ff), 1.0 / np.sqrt(d_ff))
+    f32["Bd"] = normal((d, r), 0.02)
+    f32["dOut"] = normal((N, d), 1.0)
+    for k in NAMES:
+        if cfg.int4 and k in WEIGHT_NAMES:
+            q, sc = quantize_int4(f32[k])
+            out[k + "_q"] = q
+            out[k + "_scale"] = sc
+        else:
+            out[k] = f32_to_bf16_bits(f32[k])
+        del f32[k]
+    return out
+
+
+def zero_B(inputs: dict) -> dict:
+    """Same inputs with every adapter B set to zero (the frozen-MLP special case)."""
+    o = dict(inputs)
+    for k in ("Bg", "Bu", "Bd"):
+        o[k] = np.zeros_like(inputs[k])
+    return o

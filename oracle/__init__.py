@@ -1,0 +1,17 @@
+"""CPU oracle (fp64) for the fused LoRA + SwiGLU MLP.
+
+TEST INFRASTRUCTURE ONLY: tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline / reference arm may import it; the product path never does.
+"""
+from .lora_mlp import (  # noqa: F401
+    backward,
+    bf16_to_f64,
+    dequant_int4,
+    f32_to_bf16_rne,
+    forward,
+    forward_backward,
+    sigmoid,
+    token_rows,
+    up_gate_feature_grads,
+    weights_f64,
+)
