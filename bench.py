@@ -1,0 +1,396 @@
+"""Benchmark of the fused LoRA + SwiGLU MLP forward + backward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload NAME]
+
+One step = forward + backward of the whole hot path over one batch of
+synthetic tokens (all kernels: rank-r projections, gate/up GEMM with SwiGLU
+epilogue, down GEMM, dH GEMM with SwiGLU-backward epilogue, dX GEMM, the
+adapter-gradient reductions).  Inputs are resident in HBM when the timed
+region starts; the frozen weights (352 MB on the default workload) are larger
+than the 126 MB L2, so no L2 flush is needed between steps.
+
+For N > 1 (torchrun) every rank runs an independent replica of the same
+workload (the MLP has no exchange step on this path), the barrier-bracketed
+device time is the max over ranks, and `value` is the total tokens of all
+ranks over that time ("weak" scaling).
+
+--impl reference times the fp64 CPU oracle on the host cores instead, on a
+bounded token sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from lora_fine_tuning_mlp_b200 import inputs as synth  # noqa: E402
+
+METRIC = "fused LoRA-SwiGLU MLP fwd+bwd tokens/s and TFLOP/s vs bf16 dense peak"
+DEFAULT_WORKLOAD = "llama3_8b_mlp"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"bf16_tflops": p.get("bf16_tflops", 1590.0),
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", 1400.0),
+                "hbm_gbs": p.get("hbm_gbs", 6650.0), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def gemm_flops(cfg) -> dict:
+    """Algorithmic flops of each tensor-core GEMM launch (2 per multiply-add)."""
+    N, d, f, r = cfg.N, cfg.d, cfg.d_ff, cfg.r
+    return {
+        "F1_gate_up_swiglu": 2.0 * N * f * (2 * d + 2 * r),
+        "F3_down": 2.0 * N * d * (f + r),
+        "B1_dh_swiglu_bwd": 2.0 * N * f * (d + r),
+        "B4_dX": 2.0 * N * d * (2 * f + 2 * r),
+        "F0_lowrank_in": 2.0 * N * d * 2 * r,
+        "F2_lowrank_mid": 2.0 * N * f * r,
+        "B0_lowrank_out": 2.0 * N * d * r,
+        "B0_dBd": 2.0 * N * d * r,
+        "B2_dAd": 2.0 * N * f * r,
+        "B3_lowrank_gu": 2.0 * 2 * N * f * r,
+        "B3_dBgu": 2.0 * 2 * N * f * r,
+        "B5_dA_in": 2.0 * N * d * 2 * r,
+    }
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+
+def time_oracle(cfg, budget_s: float, inp=None):
+    """Time the fp64 oracle forward+backward on a token sample of `cfg` sized
+    to take about budget_s.  Returns (tokens/s, sample tokens, seconds, threads)."""
+    import oracle
+
+    if inp is None:
+        inp = synth.make_inputs(synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4,
+                                             seed_index=cfg.index))
+    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut")})
+
+    def run(n):
+        p = dict(p_full)
+        p["X"] = oracle.bf16_to_f64(inp["X"][:n])
+        dOut = oracle.bf16_to_f64(inp["dOut"][:n])
+        t0 = time.perf_counter()
+        f = oracle.forward(p, cfg.alpha)
+        oracle.backward(p, cfg.alpha, dOut, f)
+        return time.perf_counter() - t0
+
+    t_probe = run(32)
+    n = int(32 * budget_s / max(t_probe, 1e-3))
+    n = max(32, min(n, inp["X"].shape[0]))
+    n = n // 32 * 32
+    dt = run(n)
+    return n / dt, n, dt
+
+
+def threads_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------- arms
+
+
+def reference_arm(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    import oracle
+
+    inp = synth.make_inputs(synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4,
+                                         seed_index=cfg.index))
+    _, n, _ = time_oracle(cfg, per_step, inp)
+    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut")})
+    times = []
+    for i in range(args.warmup + args.steps):
+        lo = (i * n) % inp["X"].shape[0]
+        idx = np.arange(lo, lo + n) % inp["X"].shape[0]
+        p = dict(p_full)
+        p["X"] = oracle.bf16_to_f64(inp["X"][idx])
+        dOut = oracle.bf16_to_f64(inp["dOut"][idx])
+        t0 = time.perf_counter()
+        f = oracle.forward(p, cfg.alpha)
+        oracle.backward(p, cfg.alpha, dOut, f)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total
+    cores = threads_used()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg),
+        "tflops": cfg.flops() * (n / cfg.N) * len(times) / total / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(cfg):
+    return {"workload": cfg.name, "N_tokens": cfg.N, "d": cfg.d, "d_ff": cfg.d_ff, "r": cfg.r, "alpha": cfg.alpha,
+            "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
+            "l2": "no flush: inputs larger than L2 (frozen weights %.0f MB > 126 MB)" % (
+                3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6),
+            "parallelism": "replicas" }
+
+
+def b200_arm(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    from lora_fine_tuning_mlp_b200 import _lib, api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _lib.lib()
+
+    inp = synth.make_inputs(cfg)
+    w = api.weights_from_host(inp, cfg.alpha, dev)
+    X = api.to_device_bf16(inp["X"], dev)
+    dOut = api.to_device_bf16(inp["dOut"], dev)
+    N, d, f = cfg.N, cfg.d, cfg.d_ff
+    out = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    wsf, wsb = api.Workspace(), api.Workspace()
+    stream = torch.cuda.current_stream()
+
+    def step(x=X, g_out=dOut):
+        o, saved = api.forward(x, w, out=out, workspace=wsf)
+        api.backward(x, w, saved, g_out, dX=dX, grads=grads, workspace=wsb)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    sampler = ClockSampler(dev.index)
+    _lib.timing_enable(True)
+    _lib.timing_collect()
+    launches0 = _lib.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    launches = _lib.launch_count() - launches0
+    recs = _lib.timing_collect()
+    _lib.timing_enable(False)
+    ms = t0.elapsed_time(t1)
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    # ---- end-to-end through the public API with host buffers
+    Xh = torch.from_numpy(inp["X"].view("int16")).view(torch.bfloat16).pin_memory()
+    dOh = torch.from_numpy(inp["dOut"].view("int16")).view(torch.bfloat16).pin_memory()
+    gh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in grads.items()}
+    Xd, dOd = torch.empty_like(X), torch.empty_like(dOut)
+    h2d = Xh.numel() * 2 + dOh.numel() * 2
+    d2h = sum(v.numel() * 2 for v in gh.values())
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        dOd.copy_(dOh, non_blocking=True)
+        step(Xd, dOd)
+        for k in gh:
+            gh[k].copy_(grads[k], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ems], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ems = float(tt.item())
+
+    # ---- per-kernel breakdown and the dominant kernel's roofline
+    per = {}
+    for name, kms in recs:
+        s = per.setdefault(name, [0.0, 0])
+        s[0] += kms
+        s[1] += 1
+    peaks = load_peaks()
+    fl = gemm_flops(cfg)
+    dom = max(per.items(), key=lambda kv: kv[1][0])[0] if per else None
+    roof = None
+    if dom is not None and dom in fl:
+        avg_ms = per[dom][0] / per[dom][1]
+        achieved = fl[dom] / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
+                "flops_per_launch": fl[dom], "avg_launch_ms": avg_ms}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        per_step_ms = ms_max / args.steps
+        value = world * N * args.steps / (ms_max * 1e-3)
+        tflops = world * cfg.flops() * args.steps / (ms_max * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg),
+            "tflops": tflops, "frac_of_peak": {
+                "measured_burst": tflops / world / peaks["bf16_tflops"],
+                "measured_sustained": tflops / world / peaks["bf16_tflops_sustained"],
+                "nominal_2250": tflops / world / 2250.0},
+            "roofline": roof,
+            "e2e": {"value": world * N * args.steps / (ems * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "H2D of X and dOut from pinned host, forward+backward, D2H of the six adapter grads"},
+            "gpu_launches": launches,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(per.items(), key=lambda kv: -kv[1][0])},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            tps, n, dt = time_oracle(cfg, args.cpu_budget)
+            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
+                                    "sample": f"{n} tokens of the {cfg.name} shapes, numpy fp64 oracle, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=("b200", "reference"))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = synth.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, cfg)
+    return b200_arm(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

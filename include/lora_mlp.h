@@ -1,0 +1,146 @@
+/*
+ * lora_mlp.h — C ABI of the fused LoRA + SwiGLU MLP for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  A SwiGLU MLP whose gate, up and down projections each carry
+ * a LoRA adapter, run forward and backward as one fused unit with
+ * hand-derived gradients, so that the intermediates autograd would keep are
+ * never stored ("Unsloth 深度分析报告", nightvoyager.top, section 核心价值提炼 /
+ * 创新之处, item "融合 LoRA MLP 反向传播 Kernel"; matmul and LoRA fused into
+ * single kernels: "Unsloth 还是 AirLLM？一个炼丹，一个硬跑", section 核心原理).
+ * With s = alpha / r and the nn.Linear layout (W [out, in], A [r, in], B [out, r]):
+ *
+ *   G   = X Wg^T + s (X Ag^T) Bg^T          U = X Wu^T + s (X Au^T) Bu^T
+ *   H   = silu(G) * U                        out = H Wd^T + s (H Ad^T) Bd^T
+ *
+ * and the backward gives dX and the six adapter gradients for an upstream dOut
+ * (the frozen W get no gradient).
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer is caller-owned memory; the library never allocates or
+ *    frees device memory, and never synchronises the stream (except
+ *    lora_mlp_device_status, which says so).  Work is enqueued on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream) on
+ *    the current CUDA device.
+ *  - Float tensors are bf16, row-major, densely packed (leading dimension =
+ *    the row length).  Device pointers must be 16-byte aligned.
+ *  - Sizes: N >= 1 tokens; d, d_ff multiples of 8 (of 64 for int4 weights);
+ *    r a multiple of 8 in [8, 128]; alpha finite.
+ *  - Results are written, never accumulated into.  Results are deterministic:
+ *    the same inputs give the same bits on every run.
+ *  - Return value: LORA_MLP_OK or a negative LORA_MLP_ERR_* code.  Argument
+ *    errors are detected on the host before anything is enqueued.
+ *  - Not thread-safe on one stream; independent streams may be used from
+ *    several threads.
+ */
+#ifndef LORA_MLP_H
+#define LORA_MLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LORA_MLP_OK 0
+#define LORA_MLP_ERR_INVALID_ARG (-1)         /* null pointer, non-positive size, non-finite alpha */
+#define LORA_MLP_ERR_UNSUPPORTED_SHAPE (-2)   /* divisibility or range rule above violated        */
+#define LORA_MLP_ERR_MISALIGNED (-3)          /* a device pointer is not 16-byte aligned          */
+#define LORA_MLP_ERR_WORKSPACE_TOO_SMALL (-4) /* workspace_bytes below lora_mlp_sizes()           */
+#define LORA_MLP_ERR_UNSUPPORTED_ARCH (-5)    /* current device is not compute capability 10.0    */
+#define LORA_MLP_ERR_CUDA (-6)                /* a CUDA runtime call or launch failed             */
+#define LORA_MLP_ERR_DEVICE_TIMEOUT (-7)      /* a kernel's bounded wait expired (see device_status) */
+
+/* Storage format of the frozen weights Wg, Wu, Wd. */
+#define LORA_MLP_WEIGHTS_BF16 0
+/* Symmetric int4 codes in [-7, 7], blocks of 64 consecutive input-dimension
+ * elements, one fp16 scale (the block's absolute maximum) per block:
+ * w = bf16_rne((fp32(q) * fp32(scale)) / 7.0f).  Packed as uint8
+ * [out, in/2] with element 2k in the low nibble of byte k (two's complement);
+ * scales fp16 [out, in/64] row-major.  ("native 4-bit QLoRA": blog.cn-res.vip
+ * page, 核心原理; the block layout itself is this library's choice.) */
+#define LORA_MLP_WEIGHTS_INT4_B64 1
+
+typedef struct lora_mlp_shape {
+    int64_t N;             /* tokens (rows of X)          */
+    int64_t d;             /* model width                 */
+    int64_t d_ff;          /* MLP hidden width            */
+    int64_t r;             /* LoRA rank                   */
+    float alpha;           /* LoRA scale numerator, s = alpha / r */
+    int32_t weight_format; /* LORA_MLP_WEIGHTS_*          */
+} lora_mlp_shape;
+
+/* Device pointers.  bf16 format: Wg, Wu [d_ff, d], Wd [d, d_ff] and Sg = Su =
+ * Sd = NULL.  int4 format: Wg, Wu uint8 [d_ff, d/2], Wd uint8 [d, d_ff/2]
+ * packed codes; Sg, Su fp16 [d_ff, d/64], Sd fp16 [d, d_ff/64].
+ * Adapters, always bf16: Ag, Au [r, d]; Bg, Bu [d_ff, r]; Ad [r, d_ff]; Bd [d, r]. */
+typedef struct lora_mlp_weights {
+    const void *Wg, *Wu, *Wd;
+    const void *Sg, *Su, *Sd;
+    const void *Ag, *Bg, *Au, *Bu, *Ad, *Bd;
+} lora_mlp_weights;
+
+/* Device pointers to the adapter gradients, bf16, same shapes as the adapters. */
+typedef struct lora_mlp_grads {
+    void *dAg, *dBg, *dAu, *dBu, *dAd, *dBd;
+} lora_mlp_grads;
+
+/* Byte sizes the caller must provide: the scratch workspace of forward and of
+ * backward (one buffer may serve both in turn), and the `saved` buffer that
+ * forward fills with the rank-r projections s·X·Ag^T, s·X·Au^T, s·H·Ad^T and
+ * backward reads back (an opaque layout; keep it alive from forward to
+ * backward together with g and u).  Pure host function, no CUDA call.
+ * Any output pointer may be NULL. */
+int lora_mlp_sizes(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes,
+                   size_t* bwd_workspace_bytes, size_t* saved_bytes);
+
+/* Forward.  X [N, d] in; out [N, d], g [N, d_ff] and u [N, d_ff] (the gate and
+ * up pre-activations, rounded to bf16, kept for backward) and `saved` out.
+ * H = silu(g) * u is formed from the bf16 g and u in the gate/up GEMM's
+ * epilogue and lives only in the workspace. */
+int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w,
+                     const void* X, void* out, void* g, void* u, void* saved,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward.  X, g, u, saved from the forward of the same X; dOut [N, d] in;
+ * dX [N, d] and the six adapter gradients out.  silu and sigmoid are
+ * recomputed from g and u in the epilogue of the dH GEMM. */
+int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w,
+                      const void* X, const void* g, const void* u, const void* saved,
+                      const void* dOut, void* dX, const lora_mlp_grads* grads,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Dequantise one block-int4 weight (format above) to bf16 [rows, cols];
+ * cols a multiple of 64.  The same device routine the int4 path uses, exposed
+ * so that its bits can be checked. */
+int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, int64_t cols,
+                          void* w_bf16, void* stream);
+
+/* Reads and clears the library's device status word for the current device:
+ * 0, or LORA_MLP_ERR_DEVICE_TIMEOUT if any kernel gave up a bounded wait since
+ * the last call.  Synchronises `stream`. */
+int lora_mlp_device_status(void* stream, int* status);
+
+/* Human-readable name of a return code (static string). */
+const char* lora_mlp_strerror(int code);
+
+/* Kernel-time recording for measurement.  While enabled, every kernel launch
+ * of the library is bracketed by a pair of CUDA events on its stream.
+ * lora_mlp_timing_collect synchronises those events, writes up to `max`
+ * (name, milliseconds) records in launch order, returns how many were
+ * recorded in *count, and clears the record.  Names are static strings. */
+typedef struct lora_mlp_kernel_time {
+    const char* name;
+    float ms;
+} lora_mlp_kernel_time;
+int lora_mlp_timing_enable(int enable);
+int lora_mlp_timing_collect(lora_mlp_kernel_time* out, int max, int* count);
+
+/* Number of kernels this library has launched in this process (all devices). */
+int64_t lora_mlp_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_MLP_H */

@@ -1,0 +1,160 @@
+"""ctypes binding of liblora_mlp.so (include/lora_mlp.h).
+
+Argument marshalling only: every step of the MLP runs in the library's CUDA
+kernels.  Loading fails loudly if the shared library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblora_mlp.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_SHAPE = -2
+ERR_MISALIGNED = -3
+ERR_WORKSPACE_TOO_SMALL = -4
+ERR_UNSUPPORTED_ARCH = -5
+ERR_CUDA = -6
+ERR_DEVICE_TIMEOUT = -7
+
+WEIGHTS_BF16 = 0
+WEIGHTS_INT4_B64 = 1
+
+WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Sg", "Su", "Sd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")
+GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
+
+# Every symbol include/lora_mlp.h declares.
+SYMBOLS = (
+    "lora_mlp_sizes",
+    "lora_mlp_forward",
+    "lora_mlp_backward",
+    "lora_mlp_dequant_int4",
+    "lora_mlp_device_status",
+    "lora_mlp_strerror",
+    "lora_mlp_timing_enable",
+    "lora_mlp_timing_collect",
+    "lora_mlp_launch_count",
+)
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d", ctypes.c_int64), ("d_ff", ctypes.c_int64),
+                ("r", ctypes.c_int64), ("alpha", ctypes.c_float), ("weight_format", ctypes.c_int32)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_FIELDS]
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("ms", ctypes.c_float)]
+
+
+class LoraMLPError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing: build it first (python -c 'import __graft_entry__ as g; g.build()')")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+            L.lora_mlp_sizes.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                         ctypes.POINTER(sz)]
+            L.lora_mlp_forward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp, vp,
+                                           vp, sz, vp]
+            L.lora_mlp_backward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp, vp,
+                                            vp, ctypes.POINTER(Grads), vp, sz, vp]
+            L.lora_mlp_dequant_int4.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.lora_mlp_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+            L.lora_mlp_strerror.argtypes = [ctypes.c_int]
+            L.lora_mlp_strerror.restype = ctypes.c_char_p
+            L.lora_mlp_timing_enable.argtypes = [ctypes.c_int]
+            L.lora_mlp_timing_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int,
+                                                  ctypes.POINTER(ctypes.c_int)]
+            L.lora_mlp_launch_count.argtypes = []
+            L.lora_mlp_launch_count.restype = ctypes.c_int64
+            for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_backward", "lora_mlp_dequant_int4",
+                         "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    try:
+        return lib().lora_mlp_strerror(code).decode()
+    except ImportError:
+        return "error"
+
+
+def check(code: int, what: str) -> None:
+    if code != OK:
+        raise LoraMLPError(code, what)
+
+
+def make_shape(N, d, d_ff, r, alpha, weight_format=WEIGHTS_BF16) -> Shape:
+    return Shape(int(N), int(d), int(d_ff), int(r), float(alpha), int(weight_format))
+
+
+def sizes(shape: Shape):
+    f, b, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().lora_mlp_sizes(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b), ctypes.byref(s)),
+          "lora_mlp_sizes")
+    return f.value, b.value, s.value
+
+
+def forward(shape: Shape, weights: Weights, X, out, g, u, saved, workspace, workspace_bytes, stream) -> int:
+    return lib().lora_mlp_forward(ctypes.byref(shape), ctypes.byref(weights), X, out, g, u, saved, workspace,
+                                  workspace_bytes, stream)
+
+
+def backward(shape: Shape, weights: Weights, X, g, u, saved, dOut, dX, grads: Grads, workspace,
+             workspace_bytes, stream) -> int:
+    return lib().lora_mlp_backward(ctypes.byref(shape), ctypes.byref(weights), X, g, u, saved, dOut, dX,
+                                   ctypes.byref(grads), workspace, workspace_bytes, stream)
+
+
+def dequant_int4(packed, scales, rows, cols, w_bf16, stream) -> int:
+    return lib().lora_mlp_dequant_int4(packed, scales, int(rows), int(cols), w_bf16, stream)
+
+
+def device_status(stream) -> int:
+    v = ctypes.c_int(0)
+    check(lib().lora_mlp_device_status(stream, ctypes.byref(v)), "lora_mlp_device_status")
+    return v.value
+
+
+def timing_enable(on: bool) -> None:
+    check(lib().lora_mlp_timing_enable(1 if on else 0), "lora_mlp_timing_enable")
+
+
+def timing_collect(max_records: int = 4096):
+    buf = (KernelTime * max_records)()
+    n = ctypes.c_int(0)
+    check(lib().lora_mlp_timing_collect(buf, max_records, ctypes.byref(n)), "lora_mlp_timing_collect")
+    return [(buf[i].name.decode(), float(buf[i].ms)) for i in range(min(n.value, max_records))]
+
+
+def launch_count() -> int:
+    return int(lib().lora_mlp_launch_count())

@@ -1,0 +1,224 @@
+"""PyTorch-facing wrappers of the C ABI.
+
+PyTorch provides device memory and the current stream; every step of the
+LoRA SwiGLU MLP runs in the library's sm_100a kernels.  There is no fallback:
+if the CUDA library is missing or the device is not a B200 the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+BF16 = torch.bfloat16
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+@dataclass
+class MLPWeights:
+    """Frozen SwiGLU weights and the three LoRA adapters (nn.Linear layout).
+
+    bf16 weights: Wg, Wu [d_ff, d], Wd [d, d_ff].  int4 weights: Wg, Wu uint8
+    [d_ff, d/2], Wd uint8 [d, d_ff/2] and fp16 scales Sg, Su [d_ff, d/64],
+    Sd [d, d_ff/64].  Adapters (bf16): Ag, Au [r, d]; Bg, Bu [d_ff, r];
+    Ad [r, d_ff]; Bd [d, r].
+    """
+    Wg: torch.Tensor
+    Wu: torch.Tensor
+    Wd: torch.Tensor
+    Ag: torch.Tensor
+    Bg: torch.Tensor
+    Au: torch.Tensor
+    Bu: torch.Tensor
+    Ad: torch.Tensor
+    Bd: torch.Tensor
+    alpha: float
+    Sg: torch.Tensor | None = None
+    Su: torch.Tensor | None = None
+    Sd: torch.Tensor | None = None
+
+    @property
+    def int4(self) -> bool:
+        return self.Wg.dtype == torch.uint8
+
+    @property
+    def r(self) -> int:
+        return int(self.Ag.shape[0])
+
+    @property
+    def d(self) -> int:
+        return int(self.Ag.shape[1])
+
+    @property
+    def d_ff(self) -> int:
+        return int(self.Bg.shape[0])
+
+    def shape(self, N: int) -> _lib.Shape:
+        fmt = _lib.WEIGHTS_INT4_B64 if self.int4 else _lib.WEIGHTS_BF16
+        return _lib.make_shape(N, self.d, self.d_ff, self.r, self.alpha, fmt)
+
+    def validate(self):
+        d, d_ff, r = self.d, self.d_ff, self.r
+        if self.int4:
+            _need(self.Wg, "Wg", torch.uint8, (d_ff, d // 2))
+            _need(self.Wu, "Wu", torch.uint8, (d_ff, d // 2))
+            _need(self.Wd, "Wd", torch.uint8, (d, d_ff // 2))
+            _need(self.Sg, "Sg", torch.float16, (d_ff, d // 64))
+            _need(self.Su, "Su", torch.float16, (d_ff, d // 64))
+            _need(self.Sd, "Sd", torch.float16, (d, d_ff // 64))
+        else:
+            _need(self.Wg, "Wg", BF16, (d_ff, d))
+            _need(self.Wu, "Wu", BF16, (d_ff, d))
+            _need(self.Wd, "Wd", BF16, (d, d_ff))
+        _need(self.Ag, "Ag", BF16, (r, d))
+        _need(self.Au, "Au", BF16, (r, d))
+        _need(self.Bg, "Bg", BF16, (d_ff, r))
+        _need(self.Bu, "Bu", BF16, (d_ff, r))
+        _need(self.Ad, "Ad", BF16, (r, d_ff))
+        _need(self.Bd, "Bd", BF16, (d, r))
+
+    def c_struct(self) -> _lib.Weights:
+        return _lib.Weights(*[None if getattr(self, n) is None else getattr(self, n).data_ptr()
+                              for n in _lib.WEIGHT_FIELDS])
+
+
+@dataclass
+class Saved:
+    """What forward keeps for backward: the bf16 pre-activations g, u and the
+    library's opaque rank-r buffer."""
+    g: torch.Tensor
+    u: torch.Tensor
+    lowrank: torch.Tensor
+
+
+class Workspace:
+    """A reusable device scratch buffer (grown on demand)."""
+
+    def __init__(self):
+        self.buf = None
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+def sizes(w: MLPWeights, N: int):
+    """(forward workspace, backward workspace, saved) byte counts."""
+    return _lib.sizes(w.shape(N))
+
+
+def forward(X: torch.Tensor, w: MLPWeights, *, out=None, workspace: Workspace | None = None, stream=None):
+    """out = MLP(X).  Returns (out, Saved)."""
+    N, d = X.shape
+    _need(X, "X", BF16, (N, w.d))
+    w.validate()
+    shape = w.shape(N)
+    fws, _, svs = _lib.sizes(shape)
+    dev = X.device
+    out = torch.empty((N, d), dtype=BF16, device=dev) if out is None else _need(out, "out", BF16, (N, d))
+    g = torch.empty((N, w.d_ff), dtype=BF16, device=dev)
+    u = torch.empty((N, w.d_ff), dtype=BF16, device=dev)
+    lowrank = torch.empty(max(svs, 256), dtype=torch.uint8, device=dev)
+    ws = (workspace or Workspace()).get(fws, dev)
+    _lib.check(_lib.forward(shape, w.c_struct(), _p(X), _p(out), _p(g), _p(u), _p(lowrank), _p(ws),
+                            ws.numel(), _stream(stream)), "lora_mlp_forward")
+    return out, Saved(g, u, lowrank)
+
+
+def backward(X: torch.Tensor, w: MLPWeights, saved: Saved, dOut: torch.Tensor, *, dX=None, grads=None,
+             workspace: Workspace | None = None, stream=None):
+    """Returns (dX, {dAg, dBg, dAu, dBu, dAd, dBd})."""
+    N, d = X.shape
+    _need(X, "X", BF16, (N, w.d))
+    _need(dOut, "dOut", BF16, (N, d))
+    w.validate()
+    shape = w.shape(N)
+    _, bws, _ = _lib.sizes(shape)
+    dev = X.device
+    dX = torch.empty((N, d), dtype=BF16, device=dev) if dX is None else _need(dX, "dX", BF16, (N, d))
+    if grads is None:
+        grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    gs = _lib.Grads(*[grads[k].data_ptr() for k in _lib.GRAD_FIELDS])
+    ws = (workspace or Workspace()).get(bws, dev)
+    _lib.check(_lib.backward(shape, w.c_struct(), _p(X), _p(saved.g), _p(saved.u), _p(saved.lowrank), _p(dOut),
+                             _p(dX), gs, _p(ws), ws.numel(), _stream(stream)), "lora_mlp_backward")
+    return dX, grads
+
+
+def dequant_int4(packed: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+    rows, half = packed.shape
+    _need(packed, "packed", torch.uint8)
+    _need(scales, "scales", torch.float16, (rows, 2 * half // 64))
+    w = torch.empty((rows, 2 * half), dtype=BF16, device=packed.device)
+    _lib.check(_lib.dequant_int4(_p(packed), _p(scales), rows, 2 * half, _p(w), _stream(stream)),
+               "lora_mlp_dequant_int4")
+    return w
+
+
+class LoRAMLPFunction(torch.autograd.Function):
+    """autograd wrapper: out = LoRA-SwiGLU-MLP(X); backward fills X.grad and the
+    adapter grads.  Usage: LoRAMLPFunction.apply(X, w, Ag, Bg, Au, Bu, Ad, Bd)
+    where w is an MLPWeights whose adapter tensors are the same objects."""
+
+    @staticmethod
+    def forward(ctx, X, w: MLPWeights, Ag, Bg, Au, Bu, Ad, Bd):
+        out, saved = forward(X.contiguous(), w)
+        ctx.w = w
+        ctx.saved_lr = saved
+        ctx.save_for_backward(X)
+        return out
+
+    @staticmethod
+    def backward(ctx, dOut):
+        (X,) = ctx.saved_tensors
+        dX, g = backward(X, ctx.w, ctx.saved_lr, dOut.contiguous())
+        return dX, None, g["dAg"], g["dBg"], g["dAu"], g["dBu"], g["dAd"], g["dBd"]
+
+
+def weights_from_host(inp: dict, alpha: float, device="cuda") -> MLPWeights:
+    """Upload a host input dict (bf16 bits as uint16 numpy arrays, int4 as
+    packed uint8 + fp16 scales) to the device."""
+    def bf(a):
+        return torch.from_numpy(a.view("int16")).view(BF16).to(device)
+
+    kw = {}
+    for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd"):
+        kw[k] = bf(inp[k])
+    if "Wg_q" in inp:
+        for k, s in (("Wg", "Sg"), ("Wu", "Su"), ("Wd", "Sd")):
+            kw[k] = torch.from_numpy(inp[k + "_q"]).to(device)
+            kw[s] = torch.from_numpy(inp[k + "_scale"]).to(device)
+    else:
+        for k in ("Wg", "Wu", "Wd"):
+            kw[k] = bf(inp[k])
+    return MLPWeights(alpha=float(alpha), **kw)
+
+
+def to_device_bf16(a, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(a.view("int16")).view(BF16).to(device)

@@ -1,0 +1,49 @@
+"""Build liblora_mlp.so in-tree with nvcc for sm_100a.
+
+No --use_fast_math: the int4 dequantisation relies on IEEE fp32 multiply and
+divide.  Run:  python -m lora_fine_tuning_mlp_b200.build
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+SOURCES = [os.path.join(CSRC, "lora_mlp.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma_gemm.cuh", "aux_kernels.cuh")] + [
+    os.path.join(ROOT, "include", "lora_mlp.h")]
+OUT = os.path.join(HERE, "liblora_mlp.so")
+
+
+def nvcc_cmd(out=OUT, extra=()):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    return [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+            "-shared", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-o", out, *SOURCES, *extra]
+
+
+def up_to_date(out=OUT) -> bool:
+    if not os.path.exists(out):
+        return False
+    t = os.path.getmtime(out)
+    return all(os.path.getmtime(p) <= t for p in DEPS)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return OUT
+    cmd = nvcc_cmd(extra=("-Xptxas", "-v") if verbose else ())
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building liblora_mlp.so")
+    if verbose:
+        sys.stderr.write(res.stderr)
+    return OUT
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

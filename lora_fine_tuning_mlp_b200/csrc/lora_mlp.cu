@@ -1,0 +1,800 @@
+// C ABI of the fused LoRA + SwiGLU MLP (include/lora_mlp.h): argument
+// validation, workspace layout, tensor-map encoding and the stream-ordered
+// launch sequence of forward and backward.
+//
+// Forward  (s = alpha / r; S_x denotes an s-scaled rank-r projection):
+//   F0  [S_g | S_u] = s X [Ag; Au]^T          tcgen05, two accumulators, split-K
+//   F1  G = X Wg^T + S_g Bg^T, U likewise;   tcgen05, two accumulators,
+//       epilogue writes g, u and h = silu(g) u (bf16)
+//   F2  S_d = s h Ad^T                        tcgen05, split-K
+//   F3  out = h Wd^T + S_d Bd^T               tcgen05
+// Backward:
+//   B0  T_d = s dOut Bd;  dBd = dOut^T S_d    tcgen05 (token-reduction for dBd)
+//   B1  dH = dOut Wd + T_d Ad; epilogue recomputes sigmoid/silu from g, u and
+//       writes dg, du (and h for B2)          tcgen05, MN-major weights
+//   B2  dAd = T_d^T h                          tcgen05 token-reduction
+//   B3  T_g = s dg Bg, T_u = s du Bu;  dBg = dg^T S_g, dBu = du^T S_u
+//   B4  dX = dg Wg + du Wu + T_g Ag + T_u Au   tcgen05, K = 2 d_ff + 2r
+//   B5  dAg = T_g^T X, dAu = T_u^T X           tcgen05 token-reduction
+// (The chain rule of the LoRA SwiGLU MLP; "Unsloth 深度分析报告", 创新之处:
+// hand-derived fused LoRA MLP backward that stores no autograd intermediates.)
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lora_mlp.h"
+#include "aux_kernels.cuh"
+#include "ptx.cuh"
+#include "umma_gemm.cuh"
+
+using namespace lmlp;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a layout constant
+constexpr int kMaxSplits = 32;
+constexpr size_t kAlign = 256;
+constexpr uint32_t kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
+
+std::atomic<int64_t> g_launches{0};
+
+// ----------------------------------------------------------------------------- device info
+struct DevInfo {
+    int checked;
+    int ok;
+    int sms;
+    void* status_addr;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int device_info(DevInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_MLP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo& di = g_dev[dev];
+    if (!di.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return LORA_MLP_ERR_CUDA;
+        di.ok = (major == 10 && minor == 0);
+        di.sms = sms;
+        void* addr = nullptr;
+        if (di.ok && cudaGetSymbolAddress(&addr, g_lmlp_status) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+        di.status_addr = addr;
+        di.checked = 1;
+    }
+    *out = di;
+    return di.ok ? LORA_MLP_OK : LORA_MLP_ERR_UNSUPPORTED_ARCH;
+}
+
+// ----------------------------------------------------------------------------- timing
+struct TimingRec {
+    const char* name;
+    cudaEvent_t beg, end;
+};
+std::mutex g_time_mu;
+std::atomic<int> g_timing{0};
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+struct LaunchScope {
+    const char* name;
+    cudaStream_t st;
+    cudaEvent_t beg = nullptr, end = nullptr;
+    LaunchScope(const char* n, cudaStream_t s) : name(n), st(s) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (g_timing.load(std::memory_order_relaxed)) {
+            std::lock_guard<std::mutex> lk(g_time_mu);
+            beg = pool_event();
+            end = pool_event();
+            cudaEventRecord(beg, st);
+        }
+    }
+    ~LaunchScope() {
+        if (beg != nullptr) {
+            cudaEventRecord(end, st);
+            std::lock_guard<std::mutex> lk(g_time_mu);
+            g_recs.push_back({name, beg, end});
+        }
+    }
+};
+
+int last_launch_error() { return cudaGetLastError() == cudaSuccess ? LORA_MLP_OK : LORA_MLP_ERR_CUDA; }
+
+// ----------------------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// Builds the argument block of one GEMM launch.
+struct GemmBuilder {
+    GemmArgs a;
+    int nmaps = 0;
+    bool ok = true;
+    int units = 0;
+
+    explicit GemmBuilder(int bn) {
+        std::memset(&a, 0, sizeof(a));
+        a.bn = bn;
+        a.group_m = 16;
+    }
+    // bf16 matrix [outer, inner] with row stride ld elements; box inner x outer.
+    int map(const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t box_inner, uint32_t box_outer) {
+        if (nmaps >= kMaxMaps) {
+            ok = false;
+            return 0;
+        }
+        EncodeTiledFn fn = encode_fn();
+        if (fn == nullptr) {
+            ok = false;
+            return 0;
+        }
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+        cuuint32_t box[2] = {box_inner, box_outer};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = fn(&a.maps[nmaps], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) ok = false;
+        return nmaps++;
+    }
+    // A operand, K-major: matrix [rows, K] (K contiguous).
+    int a_k(const void* p, int64_t rows, int64_t K, int64_t ld) { return map(p, K, rows, ld, kBK, kBM); }
+    // A operand, MN-major: matrix [K, M] (M contiguous), read as A[m, k].
+    int a_mn(const void* p, int64_t K, int64_t M, int64_t ld) { return map(p, M, K, ld, 64, kBK); }
+    // B operand, K-major: matrix [Nn, K].
+    int b_k(const void* p, int64_t Nn, int64_t K, int64_t ld) {
+        return map(p, K, Nn, ld, kBK, static_cast<uint32_t>(a.bn));
+    }
+    // B operand, MN-major: matrix [K, Nn] (Nn contiguous), read as B[n, k].
+    int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
+
+    Prob* prob(int64_t M, int64_t N, int splits) {
+        if (a.nprobs >= kMaxProbs) {
+            ok = false;
+            return &a.prob[0];
+        }
+        Prob& p = a.prob[a.nprobs++];
+        p.M = static_cast<int>(M);
+        p.N = static_cast<int>(N);
+        p.tiles_m = ceil_div(M, kBM);
+        p.tiles_n = ceil_div(N, a.bn);
+        p.splits = splits;
+        return &p;
+    }
+    void seg(Prob* p, int amap, int b0, int b1, int64_t k_len) {
+        if (p->nsegs >= kMaxSegs) {
+            ok = false;
+            return;
+        }
+        Seg& s = p->seg[p->nsegs++];
+        s.a_map = amap;
+        s.b_map[0] = b0;
+        s.b_map[1] = b1;
+        s.k_len = static_cast<int>(k_len);
+        s.kblocks = ceil_div(k_len, kBK);
+        p->nkb += s.kblocks;
+    }
+    void finish() {
+        int u = 0;
+        for (int i = 0; i < a.nprobs; ++i) {
+            Prob& p = a.prob[i];
+            if (p.splits > p.nkb) p.splits = p.nkb;
+            if (p.splits < 1) p.splits = 1;
+            p.unit0 = u;
+            u += p.tiles_m * p.tiles_n * p.splits;
+        }
+        a.total_units = u;
+        units = u;
+    }
+};
+
+template <int NACC, bool A_MN, bool B_MN, int EPI>
+int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name) {
+    if (!b.ok) return LORA_MLP_ERR_CUDA;
+    b.finish();
+    GemmArgs& a = b.a;
+    a.b_bytes = static_cast<uint32_t>(B_MN ? (a.bn / 64) * 8192 : a.bn * 128);
+    const uint32_t stage_bytes = kATileBytes + NACC * a.b_bytes;
+    const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
+    int stages = static_cast<int>(budget / stage_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    a.stages = stages;
+    const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + gemm_ctl_bytes();
+    auto kern = umma_gemm_kernel<NACC, A_MN, B_MN, EPI>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+            return LORA_MLP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int grid = b.units < sms ? b.units : sms;
+    {
+        LaunchScope scope(name, st);
+        kern<<<grid, kGemmThreads, smem, st>>>(a);
+    }
+    return last_launch_error();
+}
+
+int launch_reduce(const float* P, int splits, long long split_stride, int M, int ldp, int col0, int ncols,
+                  float scale, void* rm, long long ld_rm, void* tr, long long ld_tr, cudaStream_t st,
+                  const char* name) {
+    if (ncols > kRedMaxCols) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    {
+        LaunchScope scope(name, st);
+        reduce_partials_kernel<<<ceil_div(M, kRedRows), 256, 0, st>>>(
+            P, splits, split_stride, M, ldp, col0, ncols, scale, static_cast<__nv_bfloat16*>(rm), ld_rm,
+            static_cast<__nv_bfloat16*>(tr), ld_tr);
+    }
+    return last_launch_error();
+}
+
+int launch_transpose(const void* in, int64_t R, int64_t C, void* out, cudaStream_t st) {
+    {
+        LaunchScope scope("transpose_B", st);
+        transpose_bf16_kernel<<<ceil_div(R, kRedRows), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
+                                                                       static_cast<int>(R), static_cast<int>(C),
+                                                                       static_cast<__nv_bfloat16*>(out));
+    }
+    return last_launch_error();
+}
+
+int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
+                   cudaStream_t st) {
+    const long long words = rows * cols / 8;
+    long long blocks = (words + 255) / 256;
+    const long long cap = static_cast<long long>(sms) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    {
+        LaunchScope scope("dequant_int4", st);
+        dequant_int4_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
+            static_cast<const uint32_t*>(packed), static_cast<const __half*>(scales), rows, cols,
+            static_cast<__nv_bfloat16*>(w));
+    }
+    return last_launch_error();
+}
+
+// ----------------------------------------------------------------------------- layout
+int splits_for(int64_t tiles, int64_t nkb) {
+    int64_t s = kTargetCtas / (tiles > 0 ? tiles : 1);
+    if (s < 1) s = 1;
+    if (s > nkb) s = nkb;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return static_cast<int>(s < 1 ? 1 : s);
+}
+
+struct Plan {
+    int64_t N, d, d_ff, r, ldN;
+    float s;
+    bool int4;
+    int bn_r, bn_2r;
+    int sp_f0, sp_f2, sp_b0a, sp_b0b, sp_b2, sp_b3a, sp_b3b, sp_b5;
+    // forward workspace
+    size_t f_h, f_sgu, f_sd, f_part, f_w[3], f_total;
+    // backward workspace
+    size_t b_dg, b_du, b_h, b_bdT, b_bgT, b_buT, b_td, b_tdT, b_tgu, b_tguT, b_part, b_w[3], b_total;
+    // saved
+    size_t s_sgT, s_suT, s_sdT, s_total;
+};
+
+struct Carver {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off += (bytes + kAlign - 1) / kAlign * kAlign;
+        return o;
+    }
+};
+
+Plan make_plan(const lora_mlp_shape& sh) {
+    Plan p{};
+    p.N = sh.N;
+    p.d = sh.d;
+    p.d_ff = sh.d_ff;
+    p.r = sh.r;
+    p.ldN = round_up(sh.N, 8);
+    p.s = static_cast<float>(static_cast<double>(sh.alpha) / static_cast<double>(sh.r));
+    p.int4 = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64;
+    p.bn_r = static_cast<int>(round_up(sh.r, 32));
+    p.bn_2r = static_cast<int>(round_up(2 * sh.r, 32));
+    const int64_t tm_N = ceil_div(p.N, kBM);
+    p.sp_f0 = splits_for(tm_N, ceil_div(p.d, kBK));
+    p.sp_f2 = splits_for(tm_N, ceil_div(p.d_ff, kBK));
+    p.sp_b0a = splits_for(tm_N, ceil_div(p.d, kBK));
+    p.sp_b0b = splits_for(ceil_div(p.d, kBM), ceil_div(p.N, kBK));
+    p.sp_b2 = splits_for(ceil_div(p.d_ff, kBM), ceil_div(p.N, kBK));
+    p.sp_b3a = splits_for(2 * tm_N, ceil_div(p.d_ff, kBK));
+    p.sp_b3b = splits_for(2 * ceil_div(p.d_ff, kBM), ceil_div(p.N, kBK));
+    p.sp_b5 = splits_for(ceil_div(p.d, kBM), ceil_div(p.N, kBK));
+    const size_t bf = 2, f32 = 4;
+    const size_t N = p.N, d = p.d, dff = p.d_ff, r = p.r, ldN = p.ldN;
+    const size_t wsz[3] = {dff * d * bf, dff * d * bf, d * dff * bf};
+
+    Carver f;
+    p.f_h = f.take(N * dff * bf);
+    p.f_sgu = f.take(N * 2 * r * bf);
+    p.f_sd = f.take(N * r * bf);
+    size_t part = p.sp_f0 * N * 2 * r;
+    part = std::max(part, p.sp_f2 * N * r);
+    p.f_part = f.take(part * f32);
+    for (int i = 0; i < 3; ++i) p.f_w[i] = p.int4 ? f.take(wsz[i]) : 0;
+    p.f_total = f.off;
+
+    Carver b;
+    p.b_dg = b.take(N * dff * bf);
+    p.b_du = b.take(N * dff * bf);
+    p.b_h = b.take(N * dff * bf);
+    p.b_bdT = b.take(r * d * bf);
+    p.b_bgT = b.take(r * dff * bf);
+    p.b_buT = b.take(r * dff * bf);
+    p.b_td = b.take(N * r * bf);
+    p.b_tdT = b.take(r * ldN * bf);
+    p.b_tgu = b.take(N * 2 * r * bf);
+    p.b_tguT = b.take(2 * r * ldN * bf);
+    size_t bpart = p.sp_b0a * N * r;
+    bpart = std::max(bpart, p.sp_b0b * d * r);
+    bpart = std::max(bpart, p.sp_b2 * dff * r);
+    bpart = std::max(bpart, p.sp_b3a * N * 2 * r);
+    bpart = std::max(bpart, p.sp_b3b * dff * 2 * r);
+    bpart = std::max(bpart, p.sp_b5 * d * 2 * r);
+    p.b_part = b.take(bpart * f32);
+    for (int i = 0; i < 3; ++i) p.b_w[i] = p.int4 ? b.take(wsz[i]) : 0;
+    p.b_total = b.off;
+
+    Carver s;
+    p.s_sgT = s.take(r * ldN * bf);
+    p.s_suT = p.s_sgT + r * ldN * bf;  // contiguous with S_g^T: [S_g^T; S_u^T] is one [2r, ldN] matrix
+    s.take(r * ldN * bf);
+    p.s_sdT = s.take(r * ldN * bf);
+    p.s_total = s.off;
+    return p;
+}
+
+// ----------------------------------------------------------------------------- validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_shape(const lora_mlp_shape* sh) {
+    if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->N < 1 || sh->d < 1 || sh->d_ff < 1 || sh->r < 1) return LORA_MLP_ERR_INVALID_ARG;
+    if (!std::isfinite(sh->alpha)) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->d % 8 || sh->d_ff % 8 || sh->r % 8) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    if (sh->r > 128) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64 && (sh->d % 64 || sh->d_ff % 64))
+        return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    const int64_t lim = (int64_t{1} << 31) - 1;
+    if (sh->N > lim || sh->d > lim || sh->d_ff > lim) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    return LORA_MLP_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+    for (const void* p : ps) {
+        if (p == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    }
+    for (const void* p : ps) {
+        if (!aligned16(p)) return LORA_MLP_ERR_MISALIGNED;
+    }
+    return LORA_MLP_OK;
+}
+
+int check_weights(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
+    if (w == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    int rc = check_ptrs({w->Wg, w->Wu, w->Wd, w->Ag, w->Bg, w->Au, w->Bu, w->Ad, w->Bd});
+    if (rc) return rc;
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_ptrs({w->Sg, w->Su, w->Sd});
+    return LORA_MLP_OK;
+}
+
+#define LMLP_TRY(expr)              \
+    do {                            \
+        const int rc_ = (expr);     \
+        if (rc_ != LORA_MLP_OK) return rc_; \
+    } while (0)
+
+// Resolve the frozen weights to bf16 pointers (dequantising int4 into the workspace).
+int frozen_weights(const Plan& pl, const lora_mlp_weights* w, uint8_t* ws, const size_t off[3], int sms,
+                   cudaStream_t st, const void* out[3]) {
+    if (!pl.int4) {
+        out[0] = w->Wg;
+        out[1] = w->Wu;
+        out[2] = w->Wd;
+        return LORA_MLP_OK;
+    }
+    const void* q[3] = {w->Wg, w->Wu, w->Wd};
+    const void* sc[3] = {w->Sg, w->Su, w->Sd};
+    const int64_t rows[3] = {pl.d_ff, pl.d_ff, pl.d};
+    const int64_t cols[3] = {pl.d, pl.d, pl.d_ff};
+    for (int i = 0; i < 3; ++i) {
+        LMLP_TRY(launch_dequant(q[i], sc[i], rows[i], cols[i], ws + off[i], sms, st));
+        out[i] = ws + off[i];
+    }
+    return LORA_MLP_OK;
+}
+
+}  // namespace
+
+// ============================================================================= C ABI
+
+extern "C" {
+
+int lora_mlp_sizes(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes, size_t* bwd_workspace_bytes,
+                   size_t* saved_bytes) {
+    LMLP_TRY(validate_shape(shape));
+    const Plan pl = make_plan(*shape);
+    if (fwd_workspace_bytes) *fwd_workspace_bytes = pl.f_total;
+    if (bwd_workspace_bytes) *bwd_workspace_bytes = pl.b_total;
+    if (saved_bytes) *saved_bytes = pl.s_total;
+    return LORA_MLP_OK;
+}
+
+int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out, void* g,
+                     void* u, void* saved, void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    LMLP_TRY(check_weights(shape, w));
+    LMLP_TRY(check_ptrs({X, out, g, u, saved, workspace}));
+    const Plan pl = make_plan(*shape);
+    if (workspace_bytes < pl.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* sv = static_cast<uint8_t*>(saved);
+    const int64_t N = pl.N, d = pl.d, dff = pl.d_ff, r = pl.r;
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_h);
+    __nv_bfloat16* Sgu = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_sgu);
+    __nv_bfloat16* Sd = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_sd);
+    float* part = reinterpret_cast<float*>(ws + pl.f_part);
+    const void* W[3];
+    LMLP_TRY(frozen_weights(pl, w, ws, pl.f_w, di.sms, st, W));
+
+    {  // F0: [S_g | S_u] = s X [Ag; Au]^T
+        GemmBuilder b(pl.bn_r);
+        const int ax = b.a_k(X, N, d, d);
+        const int bg = b.b_k(w->Ag, r, d, d);
+        const int bu = b.b_k(w->Au, r, d, d);
+        Prob* p = b.prob(N, r, pl.sp_f0);
+        b.seg(p, ax, bg, bu, d);
+        p->out0 = part;
+        p->out1 = part + r;
+        p->ld = 2 * r;
+        p->split_stride = N * 2 * r;
+        LMLP_TRY((launch_gemm<2, false, false, EPI_F32>(b, di.sms, st, "F0_lowrank_in")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * 2 * r, static_cast<int>(N), static_cast<int>(2 * r), 0,
+                               static_cast<int>(2 * r), pl.s, Sgu, 2 * r, sv + pl.s_sgT, pl.ldN, st, "F0_reduce"));
+    }
+    {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h
+        GemmBuilder b(128);
+        const int ax = b.a_k(X, N, d, d);
+        const int asg = b.a_k(Sgu, N, r, 2 * r);
+        const int asu = b.a_k(Sgu + r, N, r, 2 * r);
+        const int bwg = b.b_k(W[0], dff, d, d);
+        const int bwu = b.b_k(W[1], dff, d, d);
+        const int bbg = b.b_k(w->Bg, dff, r, r);
+        const int bbu = b.b_k(w->Bu, dff, r, r);
+        Prob* p = b.prob(N, dff, 1);
+        b.seg(p, ax, bwg, bwu, d);
+        b.seg(p, asg, bbg, -1, r);
+        b.seg(p, asu, -1, bbu, r);
+        p->out0 = g;
+        p->out1 = u;
+        p->out2 = h;
+        p->ld = dff;
+        LMLP_TRY((launch_gemm<2, false, false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu")));
+    }
+    {  // F2: S_d = s h Ad^T
+        GemmBuilder b(pl.bn_r);
+        const int ah = b.a_k(h, N, dff, dff);
+        const int bad = b.b_k(w->Ad, r, dff, dff);
+        Prob* p = b.prob(N, r, pl.sp_f2);
+        b.seg(p, ah, bad, -1, dff);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = N * r;
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "F2_lowrank_mid")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * r, static_cast<int>(N), static_cast<int>(r), 0,
+                               static_cast<int>(r), pl.s, Sd, r, sv + pl.s_sdT, pl.ldN, st, "F2_reduce"));
+    }
+    {  // F3: out = h Wd^T + S_d Bd^T
+        GemmBuilder b(256);
+        const int ah = b.a_k(h, N, dff, dff);
+        const int asd = b.a_k(Sd, N, r, r);
+        const int bwd = b.b_k(W[2], d, dff, dff);
+        const int bbd = b.b_k(w->Bd, d, r, r);
+        Prob* p = b.prob(N, d, 1);
+        b.seg(p, ah, bwd, -1, dff);
+        b.seg(p, asd, bbd, -1, r);
+        p->out0 = out;
+        p->ld = d;
+        LMLP_TRY((launch_gemm<1, false, false, EPI_BF16>(b, di.sms, st, "F3_down")));
+    }
+    return LORA_MLP_OK;
+}
+
+int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, const void* g,
+                      const void* u, const void* saved, const void* dOut, void* dX, const lora_mlp_grads* grads,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    LMLP_TRY(check_weights(shape, w));
+    if (grads == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_ptrs({X, g, u, saved, dOut, dX, workspace, grads->dAg, grads->dBg, grads->dAu, grads->dBu,
+                         grads->dAd, grads->dBd}));
+    const Plan pl = make_plan(*shape);
+    if (workspace_bytes < pl.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    const int64_t N = pl.N, d = pl.d, dff = pl.d_ff, r = pl.r, ldN = pl.ldN;
+    __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_dg);
+    __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_du);
+    __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_h);
+    __nv_bfloat16* BdT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_bdT);
+    __nv_bfloat16* BgT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_bgT);
+    __nv_bfloat16* BuT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_buT);
+    __nv_bfloat16* Td = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_td);
+    __nv_bfloat16* TdT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tdT);
+    __nv_bfloat16* Tgu = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tgu);
+    __nv_bfloat16* TguT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tguT);
+    float* part = reinterpret_cast<float*>(ws + pl.b_part);
+    const void* SgT = sv + pl.s_sgT;
+    const void* SuT = sv + pl.s_suT;
+    const void* SdT = sv + pl.s_sdT;
+    const void* W[3];
+    LMLP_TRY(frozen_weights(pl, w, ws, pl.b_w, di.sms, st, W));
+
+    // adapter B matrices as K-major operands of the rank-r projections
+    LMLP_TRY(launch_transpose(w->Bd, d, r, BdT, st));
+    LMLP_TRY(launch_transpose(w->Bg, dff, r, BgT, st));
+    LMLP_TRY(launch_transpose(w->Bu, dff, r, BuT, st));
+
+    {  // B0a: T_d = s dOut Bd
+        GemmBuilder b(pl.bn_r);
+        const int a = b.a_k(dOut, N, d, d);
+        const int bb = b.b_k(BdT, r, d, d);
+        Prob* p = b.prob(N, r, pl.sp_b0a);
+        b.seg(p, a, bb, -1, d);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = N * r;
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B0_lowrank_out")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * r, static_cast<int>(N), static_cast<int>(r), 0,
+                               static_cast<int>(r), pl.s, Td, r, TdT, ldN, st, "B0_reduce"));
+    }
+    {  // B0b: dBd = dOut^T S_d
+        GemmBuilder b(pl.bn_r);
+        const int a = b.a_mn(dOut, N, d, d);
+        const int bb = b.b_k(SdT, r, N, ldN);
+        Prob* p = b.prob(d, r, pl.sp_b0b);
+        b.seg(p, a, bb, -1, N);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = d * r;
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B0_dBd")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, d * r, static_cast<int>(d), static_cast<int>(r), 0,
+                               static_cast<int>(r), 1.0f, grads->dBd, r, nullptr, 0, st, "B0_dBd_reduce"));
+    }
+    {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
+        GemmBuilder b(256);
+        const int a = b.a_k(dOut, N, d, d);
+        const int atd = b.a_k(Td, N, r, r);
+        const int bwd = b.b_mn(W[2], d, dff, dff);
+        const int bad = b.b_mn(w->Ad, r, dff, dff);
+        Prob* p = b.prob(N, dff, 1);
+        b.seg(p, a, bwd, -1, d);
+        b.seg(p, atd, bad, -1, r);
+        p->in0 = g;
+        p->in1 = u;
+        p->out0 = dg;
+        p->out1 = du;
+        p->out2 = hb;
+        p->ld = dff;
+        LMLP_TRY((launch_gemm<1, false, true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd")));
+    }
+    {  // B2: dAd = T_d^T h
+        GemmBuilder b(pl.bn_r);
+        const int a = b.a_mn(hb, N, dff, dff);
+        const int bb = b.b_k(TdT, r, N, ldN);
+        Prob* p = b.prob(dff, r, pl.sp_b2);
+        b.seg(p, a, bb, -1, N);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = dff * r;
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B2_dAd")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, dff * r, static_cast<int>(dff), static_cast<int>(r), 0,
+                               static_cast<int>(r), 1.0f, nullptr, 0, grads->dAd, dff, st, "B2_reduce"));
+    }
+    {  // B3a: T_g = s dg Bg, T_u = s du Bu
+        GemmBuilder b(pl.bn_r);
+        const int ag = b.a_k(dg, N, dff, dff);
+        const int au = b.a_k(du, N, dff, dff);
+        const int bg = b.b_k(BgT, r, dff, dff);
+        const int bu = b.b_k(BuT, r, dff, dff);
+        Prob* p0 = b.prob(N, r, pl.sp_b3a);
+        b.seg(p0, ag, bg, -1, dff);
+        p0->out0 = part;
+        p0->ld = 2 * r;
+        p0->split_stride = N * 2 * r;
+        Prob* p1 = b.prob(N, r, pl.sp_b3a);
+        b.seg(p1, au, bu, -1, dff);
+        p1->out0 = part + r;
+        p1->ld = 2 * r;
+        p1->split_stride = N * 2 * r;
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B3_lowrank_gu")));
+        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * 2 * r, static_cast<int>(N), static_cast<int>(2 * r), 0,
+                               static_cast<int>(2 * r), pl.s, Tgu, 2 * r, TguT, ldN, st, "B3_reduce"));
+    }
+    {  // B3b: dBg = dg^T S_g, dBu = du^T S_u
+        GemmBuilder b(pl.bn_r);
+        const int ag = b.a_mn(dg, N, dff, dff);
+        const int au = b.a_mn(du, N, dff, dff);
+        const int bg = b.b_k(SgT, r, N, ldN);
+        const int bu = b.b_k(SuT, r, N, ldN);
+        Prob* p0 = b.prob(dff, r, pl.sp_b3b);
+        b.seg(p0, ag, bg, -1, N);
+        p0->out0 = part;
+        p0->ld = 2 * r;
+        p0->split_stride = dff * 2 * r;
+        Prob* p1 = b.prob(dff, r, pl.sp_b3b);
+        b.seg(p1, au, bu, -1, N);
+        p1->out0 = part + r;
+        p1->ld = 2 * r;
+        p1->split_stride = dff * 2 * r;
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B3_dBgu")));
+        const int sp = b.a.prob[0].splits;
+        LMLP_TRY(launch_reduce(part, sp, dff * 2 * r, static_cast<int>(dff), static_cast<int>(2 * r), 0,
+                               static_cast<int>(r), 1.0f, grads->dBg, r, nullptr, 0, st, "B3_dBg_reduce"));
+        LMLP_TRY(launch_reduce(part, sp, dff * 2 * r, static_cast<int>(dff), static_cast<int>(2 * r),
+                               static_cast<int>(r), static_cast<int>(r), 1.0f, grads->dBu, r, nullptr, 0, st,
+                               "B3_dBu_reduce"));
+    }
+    {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
+        GemmBuilder b(256);
+        const int adg = b.a_k(dg, N, dff, dff);
+        const int adu = b.a_k(du, N, dff, dff);
+        const int atg = b.a_k(Tgu, N, r, 2 * r);
+        const int atu = b.a_k(Tgu + r, N, r, 2 * r);
+        const int bwg = b.b_mn(W[0], dff, d, d);
+        const int bwu = b.b_mn(W[1], dff, d, d);
+        const int bag = b.b_mn(w->Ag, r, d, d);
+        const int bau = b.b_mn(w->Au, r, d, d);
+        Prob* p = b.prob(N, d, 1);
+        b.seg(p, adg, bwg, -1, dff);
+        b.seg(p, adu, bwu, -1, dff);
+        b.seg(p, atg, bag, -1, r);
+        b.seg(p, atu, bau, -1, r);
+        p->out0 = dX;
+        p->ld = d;
+        LMLP_TRY((launch_gemm<1, false, true, EPI_BF16>(b, di.sms, st, "B4_dX")));
+    }
+    {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]
+        GemmBuilder b(pl.bn_2r);
+        const int a = b.a_mn(X, N, d, d);
+        const int bb = b.b_k(TguT, 2 * r, N, ldN);
+        Prob* p = b.prob(d, 2 * r, pl.sp_b5);
+        b.seg(p, a, bb, -1, N);
+        p->out0 = part;
+        p->ld = 2 * r;
+        p->split_stride = d * 2 * r;
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B5_dA_in")));
+        const int sp = b.a.prob[0].splits;
+        LMLP_TRY(launch_reduce(part, sp, d * 2 * r, static_cast<int>(d), static_cast<int>(2 * r), 0,
+                               static_cast<int>(r), 1.0f, nullptr, 0, grads->dAg, d, st, "B5_dAg_reduce"));
+        LMLP_TRY(launch_reduce(part, sp, d * 2 * r, static_cast<int>(d), static_cast<int>(2 * r),
+                               static_cast<int>(r), static_cast<int>(r), 1.0f, nullptr, 0, grads->dAu, d, st,
+                               "B5_dAu_reduce"));
+    }
+    return LORA_MLP_OK;
+}
+
+int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w_bf16,
+                          void* stream) {
+    if (rows < 1 || cols < 1) return LORA_MLP_ERR_INVALID_ARG;
+    if (cols % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    LMLP_TRY(check_ptrs({packed, scales, w_bf16}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return launch_dequant(packed, scales, rows, cols, w_bf16, di.sms, static_cast<cudaStream_t>(stream));
+}
+
+int lora_mlp_device_status(void* stream, int* status) {
+    if (status == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyAsync(&v, di.status_addr, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(di.status_addr, &zero, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return LORA_MLP_ERR_CUDA;
+    *status = v;
+    return LORA_MLP_OK;
+}
+
+const char* lora_mlp_strerror(int code) {
+    switch (code) {
+        case LORA_MLP_OK: return "ok";
+        case LORA_MLP_ERR_INVALID_ARG: return "invalid argument";
+        case LORA_MLP_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case LORA_MLP_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case LORA_MLP_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case LORA_MLP_ERR_UNSUPPORTED_ARCH: return "device is not compute capability 10.0 (B200)";
+        case LORA_MLP_ERR_CUDA: return "CUDA error";
+        case LORA_MLP_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+        default: return "unknown error";
+    }
+}
+
+int lora_mlp_timing_enable(int enable) {
+    g_timing.store(enable ? 1 : 0);
+    return LORA_MLP_OK;
+}
+
+int lora_mlp_timing_collect(lora_mlp_kernel_time* out, int max, int* count) {
+    std::lock_guard<std::mutex> lk(g_time_mu);
+    int n = 0;
+    int rc = LORA_MLP_OK;
+    for (const TimingRec& rec : g_recs) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(rec.end) != cudaSuccess || cudaEventElapsedTime(&ms, rec.beg, rec.end) != cudaSuccess)
+            rc = LORA_MLP_ERR_CUDA;
+        if (out != nullptr && n < max) {
+            out[n].name = rec.name;
+            out[n].ms = ms;
+        }
+        ++n;
+        g_event_pool.push_back(rec.beg);
+        g_event_pool.push_back(rec.end);
+    }
+    g_recs.clear();
+    if (count) *count = n;
+    return rc;
+}
+
+int64_t lora_mlp_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,492 @@
+// Persistent, warp-specialised tcgen05 GEMM for sm_100a.
+//
+//   C[m, n] = sum_k A[m, k] * B[n, k]      (bf16 in, fp32 accumulate in TMEM)
+//
+// One CTA per SM walks a list of output tiles ("units").  Warp 0 is the TMA
+// producer, warp 1 allocates TMEM and issues tcgen05.mma from one thread,
+// warps 2-5 are the epilogue (TMEM -> registers -> global).  Shared-memory
+// stages hand operands from TMA to the tensor core through full/empty
+// mbarriers; two TMEM accumulator buffers let the epilogue of one tile run
+// under the mainloop of the next.
+//
+// The K dimension of a tile is a list of "segments", each with its own A and
+// B tensor maps: this is how the rank-r LoRA path joins a dense projection —
+// [X | s·X·A^T] times [W | B]^T is one accumulation, the low-rank segment being
+// a K = r extension of the dense one.  With two accumulators (NACC = 2) the
+// gate and up projections share the A tiles (X) and each segment says which
+// accumulator(s) it feeds.
+//
+// Tiles are 128 x BN, K blocks are 64 bf16 = 128 B wide, every smem operand
+// tile uses the 128-byte swizzle written by TMA.  A is K-major, or MN-major
+// (activations [tokens, features] read as the transposed operand of a
+// token-reduction); B likewise.  Out-of-range rows/columns of a box are
+// zero-filled by TMA, so ragged M, N and K need no special case in the
+// mainloop; the epilogue predicates its stores.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace lmlp {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kMaxMaps = 12;
+constexpr int kMaxSegs = 4;
+constexpr int kMaxProbs = 2;
+constexpr int kMaxStages = 8;
+constexpr int kGemmThreads = 192;
+
+enum EpiKind : int {
+    EPI_BF16 = 0,        // out0[m, n] = bf16(C)
+    EPI_F32 = 1,         // fp32 partial tile (split-K), acc a -> out_a + split * split_stride
+    EPI_SWIGLU_FWD = 2,  // NACC = 2: g = bf16(C0), u = bf16(C1), h = bf16(silu(g) * u)
+    EPI_SWIGLU_BWD = 3,  // C = dH; reads g, u; writes dg, du and h (recomputed)
+};
+
+struct Seg {
+    int a_map;
+    int b_map[2];  // per accumulator; -1 = this segment does not feed it
+    int kblocks;
+    int k_len;
+};
+
+struct Prob {
+    int M, N;
+    int tiles_m, tiles_n, splits, nkb, nsegs, unit0;
+    Seg seg[kMaxSegs];
+    void* out0;
+    void* out1;
+    void* out2;
+    const void* in0;
+    const void* in1;
+    long long ld;            // row stride (elements) of out*/in*
+    long long split_stride;  // elements between split-K partials (EPI_F32)
+};
+
+struct alignas(64) GemmArgs {
+    CUtensorMap maps[kMaxMaps];
+    Prob prob[kMaxProbs];
+    int nprobs;
+    int total_units;
+    int bn;            // tile N (= UMMA N), multiple of 32, <= 256
+    int stages;
+    int group_m;       // raster: consecutive tiles walk down groups of this many M tiles
+    uint32_t b_bytes;  // one B tile: bn rows (or bn/64 MN chunks) x 128 B
+};
+
+struct Unit {
+    int p, mb, nb, ks, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+    Unit r;
+    r.p = (a.nprobs > 1 && u >= a.prob[1].unit0) ? 1 : 0;
+    const Prob& P = a.prob[r.p];
+    const int lu = u - P.unit0;
+    const int tile = lu / P.splits;
+    r.ks = lu - tile * P.splits;
+    const int per_group = a.group_m * P.tiles_n;
+    const int grp = tile / per_group;
+    const int first_m = grp * a.group_m;
+    const int gsz = min(a.group_m, P.tiles_m - first_m);
+    const int local = tile - grp * per_group;
+    r.mb = first_m + local % gsz;
+    r.nb = local / gsz;
+    r.kb0 = static_cast<int>((static_cast<long long>(r.ks) * P.nkb) / P.splits);
+    r.kb1 = static_cast<int>((static_cast<long long>(r.ks + 1) * P.nkb) / P.splits);
+    return r;
+}
+
+__device__ int g_lmlp_status;  // LORA_MLP_ERR_DEVICE_TIMEOUT once any bounded wait expired
+
+struct SmemCtl {
+    uint32_t full, empty, accf, acce, drain;  // barrier array bases (shared addresses)
+    uint32_t tmem_slot;
+    volatile int* abort_flag;
+};
+
+// Bounded wait that also gives up as soon as another role of this CTA gave up.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_lmlp_status, -7 /* LORA_MLP_ERR_DEVICE_TIMEOUT */);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x * __frcp_rn(1.0f + __expf(-x)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------------------
+// roles
+
+template <int NACC, bool A_MN, bool B_MN>
+__device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
+                                              const SmemCtl& c) {
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
+        const Unit t = decode_unit(a, u);
+        const Prob& P = a.prob[t.p];
+        int seg = 0, seg_kb0 = 0;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                seg_kb0 += P.seg[seg].kblocks;
+                ++seg;
+            }
+            const Seg& S = P.seg[seg];
+            const int k0 = (kb - seg_kb0) * kBK;
+            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c.abort_flag)) return;
+            uint32_t bytes = kATileBytes;
+#pragma unroll
+            for (int acc = 0; acc < NACC; ++acc)
+                if (S.b_map[acc] >= 0) bytes += a.b_bytes;
+            const uint32_t fb = c.full + 8u * stage;
+            mbar_arrive_expect_tx(fb, bytes);
+            const uint32_t sA = smem_base + stage * stage_bytes;
+            const CUtensorMap* am = &a.maps[S.a_map];
+            if (A_MN) {
+                tma_load_2d(sA, am, fb, t.mb * kBM, k0);
+                tma_load_2d(sA + 8192u, am, fb, t.mb * kBM + 64, k0);
+            } else {
+                tma_load_2d(sA, am, fb, k0, t.mb * kBM);
+            }
+#pragma unroll
+            for (int acc = 0; acc < NACC; ++acc) {
+                if (S.b_map[acc] < 0) continue;
+                const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
+                const CUtensorMap* bm = &a.maps[S.b_map[acc]];
+                if (B_MN) {
+                    for (int j = 0; j < a.bn / 64; ++j) tma_load_2d(sB + 8192u * j, bm, fb, t.nb * a.bn + 64 * j, k0);
+                } else {
+                    tma_load_2d(sB, bm, fb, k0, t.nb * a.bn);
+                }
+            }
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+}
+
+template <int NACC, bool A_MN, bool B_MN>
+__device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
+                                         uint32_t tmem_base, const SmemCtl& c) {
+    int stage = 0;
+    uint32_t phase = 0;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    const uint32_t idesc = idesc_bf16(static_cast<uint32_t>(a.bn), A_MN, B_MN);
+    // Two accumulators fed by the same segment sit side by side in TMEM and
+    // their B tiles side by side in smem, so one UMMA of N = 2*bn does both
+    // (A is read from smem once instead of twice).
+    const bool pair_ok = NACC == 2 && !B_MN && 2 * a.bn <= 256;
+    const uint32_t idesc_pair = idesc_bf16(static_cast<uint32_t>(2 * a.bn), A_MN, B_MN);
+    const uint32_t acc_cols = NACC * a.bn;
+    for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
+        const Unit t = decode_unit(a, u);
+        const Prob& P = a.prob[t.p];
+        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
+        tc_fence_after();
+        uint32_t started = 0;
+        int seg = 0, seg_kb0 = 0;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                seg_kb0 += P.seg[seg].kblocks;
+                ++seg;
+            }
+            const Seg& S = P.seg[seg];
+            const int k0 = (kb - seg_kb0) * kBK;
+            const int kvalid = min(kBK, S.k_len - k0);
+            const int nk = (kvalid + 15) >> 4;
+            if (!wait_or_abort(c.full + 8u * stage, phase, c.abort_flag)) return;
+            tc_fence_after();
+            const uint32_t sA = smem_base + stage * stage_bytes;
+            if (pair_ok && S.b_map[0] >= 0 && S.b_map[1] >= 0 && (started == 0u || started == 3u)) {
+                const uint32_t sB = sA + kATileBytes;
+                const uint32_t d = tmem_base + abuf * acc_cols;
+                for (int k = 0; k < nk; ++k) {
+                    const uint64_t ad = A_MN ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
+                                             : sw128_desc(sA + 32u * k, 16u, 1024u);
+                    const uint64_t bd = sw128_desc(sB + 32u * k, 16u, 1024u);
+                    umma_bf16(d, ad, bd, idesc_pair, (started & 1u) | (k > 0 ? 1u : 0u));
+                }
+                started = 3u;
+                umma_commit(c.empty + 8u * stage);
+                if (++stage == a.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                continue;
+            }
+#pragma unroll
+            for (int acc = 0; acc < NACC; ++acc) {
+                if (S.b_map[acc] < 0) continue;
+                const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
+                const uint32_t d = tmem_base + abuf * acc_cols + acc * a.bn;
+                for (int k = 0; k < nk; ++k) {
+                    const uint64_t ad = A_MN ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
+                                             : sw128_desc(sA + 32u * k, 16u, 1024u);
+                    const uint64_t bd = B_MN ? sw128_desc(sB + 2048u * k, 8192u, 1024u)
+                                             : sw128_desc(sB + 32u * k, 16u, 1024u);
+                    umma_bf16(d, ad, bd, idesc, ((started >> acc) & 1u) | (k > 0 ? 1u : 0u));
+                }
+                started |= 1u << acc;
+            }
+            umma_commit(c.empty + 8u * stage);
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        umma_commit(c.accf + 8u * abuf);
+        if (++abuf == 2) {
+            abuf = 0;
+            aphase ^= 1u;
+        }
+    }
+}
+
+template <int NACC, int EPI>
+__device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_base, const SmemCtl& c) {
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: [32*quarter, 32*quarter+32)
+    int abuf = 0;
+    uint32_t aphase = 0;
+    const uint32_t acc_cols = NACC * a.bn;
+    for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
+        const Unit t = decode_unit(a, u);
+        const Prob& P = a.prob[t.p];
+        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
+        tc_fence_after();
+        const int row = t.mb * kBM + quarter * 32 + lane;
+        const bool row_ok = row < P.M;
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * acc_cols;
+        const int nchunks = a.bn >> 5;
+        for (int ch = 0; ch < nchunks; ++ch) {
+            const int col0 = t.nb * a.bn + ch * 32;
+            if (col0 >= P.N) break;  // warp-uniform
+            if constexpr (EPI == EPI_BF16) {
+                uint32_t v[32];
+                tmem_ld32(tacc + ch * 32, v);
+                tmem_ld_wait();
+                if (row_ok) {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(P.out0) + row * P.ld + col0;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (col0 + 8 * q < P.N) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                            w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                            w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                            w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                            *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+                        }
+                    }
+                }
+            } else if constexpr (EPI == EPI_F32) {
+#pragma unroll
+                for (int acc = 0; acc < NACC; ++acc) {
+                    uint32_t v[32];
+                    tmem_ld32(tacc + acc * a.bn + ch * 32, v);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float* dst = static_cast<float*>(acc == 0 ? P.out0 : P.out1) + t.ks * P.split_stride +
+                                     row * P.ld + col0;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (col0 + 4 * q < P.N) {
+                                uint4 w = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                                *reinterpret_cast<uint4*>(dst + 4 * q) = w;
+                            }
+                        }
+                    }
+                }
+            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+                uint32_t vg[32], vu[32];
+                tmem_ld32(tacc + ch * 32, vg);
+                tmem_ld32(tacc + a.bn + ch * 32, vu);
+                tmem_ld_wait();
+                if (row_ok) {
+                    const long long off = row * P.ld + col0;
+                    __nv_bfloat16* gd = static_cast<__nv_bfloat16*>(P.out0) + off;
+                    __nv_bfloat16* ud = static_cast<__nv_bfloat16*>(P.out1) + off;
+                    __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(P.out2) + off;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (col0 + 8 * q < P.N) {
+                            uint32_t gw[4], uw[4], hw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                gw[e] = pack_bf16(__uint_as_float(vg[8 * q + 2 * e]), __uint_as_float(vg[8 * q + 2 * e + 1]));
+                                uw[e] = pack_bf16(__uint_as_float(vu[8 * q + 2 * e]), __uint_as_float(vu[8 * q + 2 * e + 1]));
+                                const float h0 = silu_f(bf16_lo(gw[e])) * bf16_lo(uw[e]);
+                                const float h1 = silu_f(bf16_hi(gw[e])) * bf16_hi(uw[e]);
+                                hw[e] = pack_bf16(h0, h1);
+                            }
+                            *reinterpret_cast<uint4*>(gd + 8 * q) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+                            *reinterpret_cast<uint4*>(ud + 8 * q) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+                            *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        }
+                    }
+                }
+            } else {  // EPI_SWIGLU_BWD
+                uint4 gv[4], uv[4];
+                const long long off = row * P.ld + col0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (row_ok && col0 + 8 * q < P.N) {
+                        gv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.in0) + off + 8 * q);
+                        uv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.in1) + off + 8 * q);
+                    } else {
+                        gv[q] = make_uint4(0, 0, 0, 0);
+                        uv[q] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                uint32_t v[32];
+                tmem_ld32(tacc + ch * 32, v);
+                tmem_ld_wait();
+                if (row_ok) {
+                    __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(P.out0) + off;
+                    __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(P.out1) + off;
+                    __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(P.out2) + off;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (col0 + 8 * q < P.N) {
+                            const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+                            const uint32_t uw[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+                            uint32_t dgw[4], duw[4], hw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float dg2[2], du2[2], h2[2];
+#pragma unroll
+                                for (int hsel = 0; hsel < 2; ++hsel) {
+                                    const float gx = hsel ? bf16_hi(gw[e]) : bf16_lo(gw[e]);
+                                    const float ux = hsel ? bf16_hi(uw[e]) : bf16_lo(uw[e]);
+                                    const float dh = __uint_as_float(v[8 * q + 2 * e + hsel]);
+                                    const float sg = __frcp_rn(1.0f + __expf(-gx));
+                                    const float sl = gx * sg;
+                                    du2[hsel] = dh * sl;
+                                    dg2[hsel] = dh * ux * sg * (1.0f + gx * (1.0f - sg));
+                                    h2[hsel] = sl * ux;
+                                }
+                                dgw[e] = pack_bf16(dg2[0], dg2[1]);
+                                duw[e] = pack_bf16(du2[0], du2[1]);
+                                hw[e] = pack_bf16(h2[0], h2[1]);
+                            }
+                            *reinterpret_cast<uint4*>(dgd + 8 * q) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                            *reinterpret_cast<uint4*>(dud + 8 * q) = make_uint4(duw[0], duw[1], duw[2], duw[3]);
+                            *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c.acce + 8u * abuf);
+        if (++abuf == 2) {
+            abuf = 0;
+            aphase ^= 1u;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// kernel
+
+__host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 5) + 16u; }
+
+__host__ __device__ inline uint32_t gemm_tmem_cols(int nacc, int bn) {
+    uint32_t need = 2u * nacc * bn, cols = 32;
+    while (cols < need) cols <<= 1;
+    return cols;
+}
+
+template <int NACC, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t stage_bytes = kATileBytes + NACC * args.b_bytes;
+    const uint32_t ctl = base + args.stages * stage_bytes;
+    uint8_t* ctl_ptr = smem_raw + (ctl - raw);
+
+    SmemCtl c;
+    c.full = ctl;
+    c.empty = ctl + 8u * kMaxStages;
+    c.accf = ctl + 8u * (2 * kMaxStages);
+    c.acce = c.accf + 16u;
+    c.drain = c.acce + 16u;
+    c.tmem_slot = c.drain + 8u;
+    c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t tmem_cols = gemm_tmem_cols(NACC, args.bn);
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < args.stages; ++s) {
+            mbar_init(c.full + 8u * s, 1);
+            mbar_init(c.empty + 8u * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(c.accf + 8u * b, 1);
+            mbar_init(c.acce + 8u * b, 4);
+        }
+        mbar_init(c.drain, 1);
+        *c.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(c.tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(ctl_ptr + (c.tmem_slot - ctl));
+
+    if (warp == 0) {
+        if (lane == 0) producer_loop<NACC, A_MN, B_MN>(args, base, stage_bytes, c);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            mma_loop<NACC, A_MN, B_MN>(args, base, stage_bytes, tmem_base, c);
+            // Drain: wait until every MMA issued by this thread has finished
+            // before TMEM is released (matters only after an abort).
+            umma_commit(c.drain);
+            const long long t0 = clock64();
+            while (!mbar_try_wait(c.drain, 0)) {
+                if (clock64() - t0 > kWaitLimitCycles) break;
+            }
+        }
+        __syncwarp();
+    } else {
+        epilogue_loop<NACC, EPI>(args, tmem_base, c);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+}  // namespace lmlp

@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every symbol the header declares, sizes its buffers, and rejects bad
+arguments with the documented codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lora_fine_tuning_mlp_b200 import _lib
+from lora_fine_tuning_mlp_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_mlp.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.lib()
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lora_mlp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert header_symbols() == sorted(_lib.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_symbols():
+        assert hasattr(L, name), name
+
+
+def test_strerror_codes(L):
+    for code in range(0, -8, -1):
+        assert _lib.strerror(code) not in ("", "unknown error")
+    assert _lib.strerror(-99) == "unknown error"
+
+
+def shape(N=512, d=256, d_ff=704, r=8, alpha=16.0, fmt=0):
+    return _lib.make_shape(N, d, d_ff, r, alpha, fmt)
+
+
+def test_sizes_are_positive_and_grow_with_N(L):
+    f1, b1, s1 = _lib.sizes(shape(N=512))
+    f2, b2, s2 = _lib.sizes(shape(N=4096))
+    assert 0 < f1 < f2 and 0 < b1 < b2 and 0 < s1 < s2
+    # the saved rank-r buffer holds three bf16 [r, N] tiles (N padded to 8)
+    assert s1 >= 3 * 8 * 512 * 2
+    # backward keeps dg, du and h in its workspace
+    assert b1 >= 3 * 512 * 704 * 2
+
+
+def test_int4_workspace_holds_dequantised_weights(L):
+    with pytest.raises(_lib.LoraMLPError) as e:
+        _lib.sizes(shape(d=256, d_ff=712, fmt=1))   # 712 is not a multiple of 64
+    assert e.value.code == _lib.ERR_UNSUPPORTED_SHAPE
+    f1, b1, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=1))
+    f0b, b0b, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=0))
+    assert f1 - f0b >= 3 * 256 * 768 * 2 and b1 - b0b >= 3 * 256 * 768 * 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), _lib.ERR_INVALID_ARG),
+    (dict(d=-8), _lib.ERR_INVALID_ARG),
+    (dict(alpha=float("nan")), _lib.ERR_INVALID_ARG),
+    (dict(alpha=float("inf")), _lib.ERR_INVALID_ARG),
+    (dict(fmt=7), _lib.ERR_INVALID_ARG),
+    (dict(d=260), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(d_ff=700), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(r=12), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(r=136), _lib.ERR_UNSUPPORTED_SHAPE),
+])
+def test_shape_validation(L, kw, code):
+    sh = shape(**kw)
+    f = ctypes.c_size_t()
+    assert L.lora_mlp_sizes(ctypes.byref(sh), ctypes.byref(f), None, None) == code
+
+
+FAKE = 0x10000  # a 16-byte-aligned non-null address: never dereferenced, validation fails first
+
+
+def weights(**over):
+    vals = {n: FAKE for n in _lib.WEIGHT_FIELDS}
+    vals.update({"Sg": None, "Su": None, "Sd": None})
+    vals.update(over)
+    return _lib.Weights(*[vals[n] for n in _lib.WEIGHT_FIELDS])
+
+
+def fwd(L, sh, w, X=FAKE, ws_bytes=1 << 40, saved=FAKE):
+    return _lib.forward(sh, w, X, FAKE, FAKE, FAKE, saved, FAKE, ws_bytes, None)
+
+
+def test_forward_argument_errors(L):
+    sh = shape()
+    assert fwd(L, sh, weights(Wg=None)) == _lib.ERR_INVALID_ARG
+    assert fwd(L, sh, weights(Bd=FAKE + 2)) == _lib.ERR_MISALIGNED
+    assert fwd(L, sh, weights(), X=None) == _lib.ERR_INVALID_ARG
+    assert fwd(L, sh, weights(), X=FAKE + 8) == _lib.ERR_MISALIGNED
+    assert fwd(L, sh, weights(), saved=None) == _lib.ERR_INVALID_ARG
+    fws, _, _ = _lib.sizes(sh)
+    assert fwd(L, sh, weights(), ws_bytes=fws - 1) == _lib.ERR_WORKSPACE_TOO_SMALL
+    # int4 needs the scale pointers
+    sh4 = shape(d_ff=768, fmt=1)
+    assert fwd(L, sh4, weights()) == _lib.ERR_INVALID_ARG
+    assert L.lora_mlp_forward(None, ctypes.byref(weights()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, None) \
+        == _lib.ERR_INVALID_ARG
+
+
+def test_backward_argument_errors(L):
+    sh = shape()
+    _, bws, _ = _lib.sizes(sh)
+    g = _lib.Grads(*([FAKE] * 6))
+    w = weights()
+
+    def bwd(dOut=FAKE, grads=g, ws=bws):
+        return _lib.backward(sh, w, FAKE, FAKE, FAKE, FAKE, dOut, FAKE, grads, FAKE, ws, None)
+
+    assert bwd(dOut=None) == _lib.ERR_INVALID_ARG
+    assert bwd(dOut=FAKE + 4) == _lib.ERR_MISALIGNED
+    assert bwd(grads=_lib.Grads(FAKE, FAKE, None, FAKE, FAKE, FAKE)) == _lib.ERR_INVALID_ARG
+    assert bwd(ws=bws - 1) == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert L.lora_mlp_backward(ctypes.byref(sh), ctypes.byref(w), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                               bws, None) == _lib.ERR_INVALID_ARG
+
+
+def test_dequant_argument_errors(L):
+    assert _lib.dequant_int4(FAKE, FAKE, 4, 100, FAKE, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _lib.dequant_int4(FAKE, FAKE, 0, 64, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.dequant_int4(None, FAKE, 4, 64, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.dequant_int4(FAKE, FAKE + 1, 4, 64, FAKE, None) == _lib.ERR_MISALIGNED
+
+
+def test_timing_toggle_without_gpu(L):
+    _lib.timing_enable(True)
+    _lib.timing_enable(False)
+    assert _lib.timing_collect() == []
+    assert _lib.launch_count() == 0
