@@ -32,6 +32,7 @@
 #include "aux_kernels.cuh"
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
+#include "umma2_gemm.cuh"
 
 using namespace lmlp;
 
@@ -140,6 +141,22 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// Tiled, 128-byte-swizzled TMA descriptor of a bf16 matrix [outer, inner]
+// (row stride ld elements) with a box_inner x box_outer box.  Out-of-range
+// elements of a box read as zero.
+bool encode_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t box_inner,
+                uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
@@ -161,19 +178,7 @@ struct GemmBuilder {
             ok = false;
             return 0;
         }
-        EncodeTiledFn fn = encode_fn();
-        if (fn == nullptr) {
-            ok = false;
-            return 0;
-        }
-        cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
-        cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-        cuuint32_t box[2] = {box_inner, box_outer};
-        cuuint32_t es[2] = {1, 1};
-        CUresult r = fn(&a.maps[nmaps], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) ok = false;
+        if (!encode_map(&a.maps[nmaps], ptr, inner, outer, ld, box_inner, box_outer)) ok = false;
         return nmaps++;
     }
     // A operand, K-major: matrix [rows, K] (K contiguous).
@@ -184,9 +189,6 @@ struct GemmBuilder {
     int b_k(const void* p, int64_t Nn, int64_t K, int64_t ld) {
         return map(p, K, Nn, ld, kBK, static_cast<uint32_t>(a.bn));
     }
-    // B operand, MN-major: matrix [K, Nn] (Nn contiguous), read as B[n, k].
-    int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
-
     Prob* prob(int64_t M, int64_t N, int splits) {
         if (a.nprobs >= kMaxProbs) {
             ok = false;
@@ -254,6 +256,96 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name) {
         LaunchScope scope(name, st);
         kern<<<grid, kGemmThreads, smem, st>>>(a);
     }
+    return last_launch_error();
+}
+
+// Builds the argument block of one CTA-pair GEMM launch (256-row tiles).
+struct PairBuilder {
+    PairArgs a;
+    int nmaps = 0;
+    bool ok = true;
+
+    PairBuilder(int64_t M, int64_t N, int tile_n) {
+        std::memset(&a, 0, sizeof(a));
+        a.group_m = 8;
+        a.prob.M = static_cast<int>(M);
+        a.prob.N = static_cast<int>(N);
+        a.prob.tile_n = tile_n;
+        a.prob.tiles_m = ceil_div(M, kPairBM);
+        a.prob.tiles_n = ceil_div(N, tile_n);
+    }
+    int map(const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t bi, uint32_t bo) {
+        if (nmaps >= kMaxMaps) {
+            ok = false;
+            return 0;
+        }
+        if (!encode_map(&a.maps[nmaps], ptr, inner, outer, ld, bi, bo)) ok = false;
+        return nmaps++;
+    }
+    int a_k(const void* p, int64_t rows, int64_t K, int64_t ld) { return map(p, K, rows, ld, kBK, kBM); }
+    int b_k(const void* p, int64_t Nn, int64_t K, int64_t ld) { return map(p, K, Nn, ld, kBK, kPairHalfN); }
+    int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
+    void seg(int amap, int b0, int b1, int row0, int row1, int k0, int k1, int64_t k_len) {
+        PairProb& p = a.prob;
+        if (p.nsegs >= kMaxSegs) {
+            ok = false;
+            return;
+        }
+        PairSeg& s = p.seg[p.nsegs++];
+        s.a_map = amap;
+        s.b_map[0] = b0;
+        s.b_map[1] = b1;
+        s.b_row[0] = row0;
+        s.b_row[1] = row1;
+        s.b_k[0] = k0;
+        s.b_k[1] = k1;
+        s.k_len = static_cast<int>(k_len);
+        s.kblocks = ceil_div(k_len, kBK);
+        p.nkb += s.kblocks;
+    }
+};
+
+template <bool B_MN, int EPI>
+int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name) {
+    if (!b.ok) return LORA_MLP_ERR_CUDA;
+    PairArgs& a = b.a;
+    a.total_units = a.prob.tiles_m * a.prob.tiles_n;
+    const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
+    int stages = static_cast<int>(budget / kPairStageBytes);
+    if (stages > kPairMaxStages) stages = kPairMaxStages;
+    a.stages = stages;
+    const size_t smem = 1024 + static_cast<size_t>(stages) * kPairStageBytes + gemm_ctl_bytes();
+    auto kern = umma2_gemm_kernel<B_MN, EPI>;
+    static int max_clusters[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters[dev] == 0) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+            return LORA_MLP_ERR_CUDA;
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = sms / 2;
+        max_clusters[dev] = n;
+    }
+    int clusters = a.total_units < max_clusters[dev] ? a.total_units : max_clusters[dev];
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cudaError_t err;
+    {
+        LaunchScope scope(name, st);
+        err = cudaLaunchKernelEx(&cfg, kern, a);
+    }
+    if (err != cudaSuccess) return LORA_MLP_ERR_CUDA;
     return last_launch_error();
 }
 
@@ -505,24 +597,21 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * 2 * r, static_cast<int>(N), static_cast<int>(2 * r), 0,
                                static_cast<int>(2 * r), pl.s, Sgu, 2 * r, sv + pl.s_sgT, pl.ldN, st, "F0_reduce"));
     }
-    {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h
-        GemmBuilder b(128);
+    {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
+        PairBuilder b(N, dff, 128);
         const int ax = b.a_k(X, N, d, d);
-        const int asg = b.a_k(Sgu, N, r, 2 * r);
-        const int asu = b.a_k(Sgu + r, N, r, 2 * r);
+        const int asgu = b.a_k(Sgu, N, 2 * r, 2 * r);
         const int bwg = b.b_k(W[0], dff, d, d);
         const int bwu = b.b_k(W[1], dff, d, d);
         const int bbg = b.b_k(w->Bg, dff, r, r);
         const int bbu = b.b_k(w->Bu, dff, r, r);
-        Prob* p = b.prob(N, dff, 1);
-        b.seg(p, ax, bwg, bwu, d);
-        b.seg(p, asg, bbg, -1, r);
-        b.seg(p, asu, -1, bbu, r);
-        p->out0 = g;
-        p->out1 = u;
-        p->out2 = h;
-        p->ld = dff;
-        LMLP_TRY((launch_gemm<2, false, false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu")));
+        b.seg(ax, bwg, bwu, 0, 0, 0, 0, d);
+        b.seg(asgu, bbg, bbu, 0, 0, 0, static_cast<int>(-r), 2 * r);
+        b.a.prob.out0 = g;
+        b.a.prob.out1 = u;
+        b.a.prob.out2 = h;
+        b.a.prob.ld = dff;
+        LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu")));
     }
     {  // F2: S_d = s h Ad^T
         GemmBuilder b(pl.bn_r);
@@ -538,17 +627,16 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
                                static_cast<int>(r), pl.s, Sd, r, sv + pl.s_sdT, pl.ldN, st, "F2_reduce"));
     }
     {  // F3: out = h Wd^T + S_d Bd^T
-        GemmBuilder b(256);
+        PairBuilder b(N, d, 256);
         const int ah = b.a_k(h, N, dff, dff);
         const int asd = b.a_k(Sd, N, r, r);
         const int bwd = b.b_k(W[2], d, dff, dff);
         const int bbd = b.b_k(w->Bd, d, r, r);
-        Prob* p = b.prob(N, d, 1);
-        b.seg(p, ah, bwd, -1, dff);
-        b.seg(p, asd, bbd, -1, r);
-        p->out0 = out;
-        p->ld = d;
-        LMLP_TRY((launch_gemm<1, false, false, EPI_BF16>(b, di.sms, st, "F3_down")));
+        b.seg(ah, bwd, bwd, 0, kPairHalfN, 0, 0, dff);
+        b.seg(asd, bbd, bbd, 0, kPairHalfN, 0, 0, r);
+        b.a.prob.out0 = out;
+        b.a.prob.ld = d;
+        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down")));
     }
     return LORA_MLP_OK;
 }
@@ -618,21 +706,21 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
                                static_cast<int>(r), 1.0f, grads->dBd, r, nullptr, 0, st, "B0_dBd_reduce"));
     }
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
-        GemmBuilder b(256);
+        PairBuilder b(N, dff, 256);
         const int a = b.a_k(dOut, N, d, d);
         const int atd = b.a_k(Td, N, r, r);
         const int bwd = b.b_mn(W[2], d, dff, dff);
         const int bad = b.b_mn(w->Ad, r, dff, dff);
-        Prob* p = b.prob(N, dff, 1);
-        b.seg(p, a, bwd, -1, d);
-        b.seg(p, atd, bad, -1, r);
-        p->in0 = g;
-        p->in1 = u;
-        p->out0 = dg;
-        p->out1 = du;
-        p->out2 = hb;
-        p->ld = dff;
-        LMLP_TRY((launch_gemm<1, false, true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd")));
+        b.seg(a, bwd, bwd, 0, kPairHalfN, 0, 0, d);
+        b.seg(atd, bad, bad, 0, kPairHalfN, 0, 0, r);
+        PairProb& p = b.a.prob;
+        p.in0 = g;
+        p.in1 = u;
+        p.out0 = dg;
+        p.out1 = du;
+        p.out2 = hb;
+        p.ld = dff;
+        LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd")));
     }
     {  // B2: dAd = T_d^T h
         GemmBuilder b(pl.bn_r);
@@ -692,7 +780,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
                                "B3_dBu_reduce"));
     }
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
-        GemmBuilder b(256);
+        PairBuilder b(N, d, 256);
         const int adg = b.a_k(dg, N, dff, dff);
         const int adu = b.a_k(du, N, dff, dff);
         const int atg = b.a_k(Tgu, N, r, 2 * r);
@@ -701,14 +789,13 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         const int bwu = b.b_mn(W[1], dff, d, d);
         const int bag = b.b_mn(w->Ag, r, d, d);
         const int bau = b.b_mn(w->Au, r, d, d);
-        Prob* p = b.prob(N, d, 1);
-        b.seg(p, adg, bwg, -1, dff);
-        b.seg(p, adu, bwu, -1, dff);
-        b.seg(p, atg, bag, -1, r);
-        b.seg(p, atu, bau, -1, r);
-        p->out0 = dX;
-        p->ld = d;
-        LMLP_TRY((launch_gemm<1, false, true, EPI_BF16>(b, di.sms, st, "B4_dX")));
+        b.seg(adg, bwg, bwg, 0, kPairHalfN, 0, 0, dff);
+        b.seg(adu, bwu, bwu, 0, kPairHalfN, 0, 0, dff);
+        b.seg(atg, bag, bag, 0, kPairHalfN, 0, 0, r);
+        b.seg(atu, bau, bau, 0, kPairHalfN, 0, 0, r);
+        b.a.prob.out0 = dX;
+        b.a.prob.ld = d;
+        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX")));
     }
     {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]
         GemmBuilder b(pl.bn_2r);

@@ -1,0 +1,280 @@
+// Persistent tcgen05 GEMM on CTA pairs (cta_group::2) for the four large
+// projections of the MLP.
+//
+// A 2-CTA cluster computes a 256 x 256 accumulator: each CTA TMA-loads its
+// own 128 rows of A and its own 128-row half of B into its shared memory
+// (plain loads, no multicast), the leader CTA issues M = 256 UMMAs that read
+// both CTAs' operands, and each CTA's TMEM receives its 128 rows.  Per SM this
+// moves half the B bytes of a 1-CTA 128 x 256 tile for the same work, which
+// is what lets the TMA keep up with the tensor core.
+//
+// Synchronisation: both CTAs' loads count on the leader's "full" barrier
+// (TMA with .cta_group::2); the leader's tcgen05.commit multicasts to the
+// "empty" and "acc-full" barriers of both CTAs; both CTAs' epilogue warps
+// arrive on the leader's "acc-empty" barrier.  Every wait is bounded.
+//
+// The B halves are addressed per segment (map, row offset, K offset), so the
+// same kernel serves
+//   * single outputs (tile = 256 output columns, halves = rows n0 and n0+128), and
+//   * the gate/up pair (tile = 128 output columns; half 0 = Wg rows, half 1 =
+//     Wu rows, accumulator columns [0,128) = G and [128,256) = U).  Their
+//     rank-r extension is one K = 2r segment: A = [S_g | S_u], half 0 reads
+//     Bg at K offset 0 and half 1 reads Bu at K offset -r, the zero fill of
+//     out-of-range columns supplying the two zero blocks.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "epilogue.cuh"
+#include "ptx.cuh"
+#include "umma_gemm.cuh"
+
+namespace lmlp {
+
+constexpr int kPairBM = 256;
+constexpr int kPairHalfN = 128;
+constexpr uint32_t kPairBBytes = kPairHalfN * kBK * 2;                  // 16 KB per CTA
+constexpr uint32_t kPairStageBytes = kATileBytes + kPairBBytes;         // 32 KB per CTA
+constexpr int kPairMaxStages = 8;
+constexpr uint32_t kPairTmemCols = 512;                                 // 2 buffers x 256 columns
+
+struct PairSeg {
+    int a_map;
+    int b_map[2];  // B half 0 / half 1
+    int b_row[2];  // N-row offset of each half from the tile's first B row
+    int b_k[2];    // K-coordinate offset of each half
+    int kblocks;
+    int k_len;
+};
+
+struct PairProb {
+    int M, N;    // output rows / columns
+    int tile_n;  // output columns per tile (256, or 128 for the gate/up pair)
+    int tiles_m, tiles_n, nkb, nsegs;
+    PairSeg seg[kMaxSegs];
+    void* out0;
+    void* out1;
+    void* out2;
+    const void* in0;
+    const void* in1;
+    long long ld;
+};
+
+struct alignas(64) PairArgs {
+    CUtensorMap maps[kMaxMaps];
+    PairProb prob;
+    int total_units;
+    int stages;
+    int group_m;
+};
+
+__device__ __forceinline__ void pair_decode(const PairArgs& a, int u, int& mb, int& nb) {
+    const PairProb& P = a.prob;
+    const int per_group = a.group_m * P.tiles_n;
+    const int grp = u / per_group;
+    const int first_m = grp * a.group_m;
+    const int gsz = min(a.group_m, P.tiles_m - first_m);
+    const int local = u - grp * per_group;
+    mb = first_m + local % gsz;
+    nb = local / gsz;
+}
+
+template <bool B_MN>
+__device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, uint32_t rank, bool leader,
+                                              const SmemCtl& c) {
+    const PairProb& P = a.prob;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int u = cid; u < a.total_units; u += ncl) {
+        int mb, nb;
+        pair_decode(a, u, mb, nb);
+        int seg = 0, seg_kb0 = 0;
+        for (int kb = 0; kb < P.nkb; ++kb) {
+            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                seg_kb0 += P.seg[seg].kblocks;
+                ++seg;
+            }
+            const PairSeg& S = P.seg[seg];
+            const int k0 = (kb - seg_kb0) * kBK;
+            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c.abort_flag)) return;
+            const uint32_t fb_local = c.full + 8u * stage;
+            if (leader) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
+            const uint32_t fb = mapa_shared(fb_local, 0);
+            const uint32_t sA = base + stage * kPairStageBytes;
+            const uint32_t sB = sA + kATileBytes;
+            tma_load_2d_pair(sA, &a.maps[S.a_map], fb, k0, mb * kPairBM + static_cast<int>(rank) * kBM);
+            const CUtensorMap* bm = &a.maps[S.b_map[rank]];
+            const int brow = nb * P.tile_n + S.b_row[rank];
+            const int bk = k0 + S.b_k[rank];
+            if (B_MN) {
+                tma_load_2d_pair(sB, bm, fb, brow, bk);
+                tma_load_2d_pair(sB + 8192u, bm, fb, brow + 64, bk);
+            } else {
+                tma_load_2d_pair(sB, bm, fb, bk, brow);
+            }
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+}
+
+template <bool B_MN>
+__device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint32_t tmem_base, const SmemCtl& c) {
+    const PairProb& P = a.prob;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    const uint32_t idesc = idesc_bf16(256u, false, B_MN, 256u);
+    int stage = 0;
+    uint32_t phase = 0;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    for (int u = cid; u < a.total_units; u += ncl) {
+        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
+        tc_fence_after();
+        const uint32_t d = tmem_base + abuf * 256u;
+        bool started = false;
+        int seg = 0, seg_kb0 = 0;
+        for (int kb = 0; kb < P.nkb; ++kb) {
+            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                seg_kb0 += P.seg[seg].kblocks;
+                ++seg;
+            }
+            const PairSeg& S = P.seg[seg];
+            const int k0 = (kb - seg_kb0) * kBK;
+            const int nk = (min(kBK, S.k_len - k0) + 15) >> 4;
+            if (!wait_or_abort(c.full + 8u * stage, phase, c.abort_flag)) return;
+            tc_fence_after();
+            const uint32_t sA = base + stage * kPairStageBytes;
+            const uint32_t sB = sA + kATileBytes;
+            for (int k = 0; k < nk; ++k) {
+                const uint64_t ad = sw128_desc(sA + 32u * k, 16u, 1024u);
+                const uint64_t bd = B_MN ? sw128_desc(sB + 2048u * k, 8192u, 1024u) : sw128_desc(sB + 32u * k, 16u, 1024u);
+                umma_bf16_pair(d, ad, bd, idesc, (started || k > 0) ? 1u : 0u);
+            }
+            started = true;
+            umma_commit_pair(c.empty + 8u * stage, 3);
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        umma_commit_pair(c.accf + 8u * abuf, 3);
+        if (++abuf == 2) {
+            abuf = 0;
+            aphase ^= 1u;
+        }
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_base, uint32_t rank,
+                                              const SmemCtl& c) {
+    constexpr int NACC = EPI == EPI_SWIGLU_FWD ? 2 : 1;
+    const PairProb& P = a.prob;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int quarter = warp & 3;
+    EpiOut o;
+    o.out0 = P.out0;
+    o.out1 = P.out1;
+    o.out2 = P.out2;
+    o.in0 = P.in0;
+    o.in1 = P.in1;
+    o.ld = P.ld;
+    o.split_off = 0;
+    o.M = P.M;
+    o.N = P.N;
+    const int bn = 256 / NACC;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    for (int u = cid; u < a.total_units; u += ncl) {
+        int mb, nb;
+        pair_decode(a, u, mb, nb);
+        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
+        tc_fence_after();
+        const int row = mb * kPairBM + static_cast<int>(rank) * kBM + quarter * 32 + lane;
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * 256u;
+        epilogue_tile<NACC, EPI>(o, row, nb * P.tile_n, bn, tacc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(c.acce + 8u * abuf, 0));
+        if (++abuf == 2) {
+            abuf = 0;
+            aphase ^= 1u;
+        }
+    }
+}
+
+template <bool B_MN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t ctl = base + args.stages * kPairStageBytes;
+    uint8_t* ctl_ptr = smem_raw + (ctl - raw);
+
+    SmemCtl c;
+    c.full = ctl;
+    c.empty = ctl + 8u * kMaxStages;
+    c.accf = ctl + 8u * (2 * kMaxStages);
+    c.acce = c.accf + 16u;
+    c.drain = c.acce + 16u;
+    c.tmem_slot = c.drain + 8u;
+    c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < args.stages; ++s) {
+            mbar_init(c.full + 8u * s, 1);
+            mbar_init(c.empty + 8u * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(c.accf + 8u * b, 1);
+            mbar_init(c.acce + 8u * b, 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(c.drain, 1);
+        *c.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(c.tmem_slot, kPairTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(ctl_ptr + (c.tmem_slot - ctl));
+
+    if (warp == 0) {
+        if (lane == 0) pair_producer<B_MN>(args, base, rank, leader, c);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            pair_mma<B_MN>(args, base, tmem_base, c);
+            umma_commit_pair(c.drain, 1);
+            const long long t0 = clock64();
+            while (!mbar_try_wait(c.drain, 0)) {
+                if (clock64() - t0 > kWaitLimitCycles) break;
+            }
+        }
+        __syncwarp();
+    } else {
+        pair_epilogue<EPI>(args, tmem_base, rank, c);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kPairTmemCols);
+}
+
+}  // namespace lmlp

@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace lmlp {
@@ -38,13 +39,6 @@ constexpr int kMaxSegs = 4;
 constexpr int kMaxProbs = 2;
 constexpr int kMaxStages = 8;
 constexpr int kGemmThreads = 192;
-
-enum EpiKind : int {
-    EPI_BF16 = 0,        // out0[m, n] = bf16(C)
-    EPI_F32 = 1,         // fp32 partial tile (split-K), acc a -> out_a + split * split_stride
-    EPI_SWIGLU_FWD = 2,  // NACC = 2: g = bf16(C0), u = bf16(C1), h = bf16(silu(g) * u)
-    EPI_SWIGLU_BWD = 3,  // C = dH; reads g, u; writes dg, du and h (recomputed)
-};
 
 struct Seg {
     int a_map;
@@ -123,14 +117,6 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     return true;
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x * __frcp_rn(1.0f + __expf(-x)); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------------------
 // roles
@@ -276,129 +262,19 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
         const Prob& P = a.prob[t.p];
         if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
         tc_fence_after();
+        EpiOut o;
+        o.out0 = P.out0;
+        o.out1 = P.out1;
+        o.out2 = P.out2;
+        o.in0 = P.in0;
+        o.in1 = P.in1;
+        o.ld = P.ld;
+        o.split_off = t.ks * P.split_stride;
+        o.M = P.M;
+        o.N = P.N;
         const int row = t.mb * kBM + quarter * 32 + lane;
-        const bool row_ok = row < P.M;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * acc_cols;
-        const int nchunks = a.bn >> 5;
-        for (int ch = 0; ch < nchunks; ++ch) {
-            const int col0 = t.nb * a.bn + ch * 32;
-            if (col0 >= P.N) break;  // warp-uniform
-            if constexpr (EPI == EPI_BF16) {
-                uint32_t v[32];
-                tmem_ld32(tacc + ch * 32, v);
-                tmem_ld_wait();
-                if (row_ok) {
-                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(P.out0) + row * P.ld + col0;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (col0 + 8 * q < P.N) {
-                            uint4 w;
-                            w.x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                            w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                            w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                            w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            *reinterpret_cast<uint4*>(dst + 8 * q) = w;
-                        }
-                    }
-                }
-            } else if constexpr (EPI == EPI_F32) {
-#pragma unroll
-                for (int acc = 0; acc < NACC; ++acc) {
-                    uint32_t v[32];
-                    tmem_ld32(tacc + acc * a.bn + ch * 32, v);
-                    tmem_ld_wait();
-                    if (row_ok) {
-                        float* dst = static_cast<float*>(acc == 0 ? P.out0 : P.out1) + t.ks * P.split_stride +
-                                     row * P.ld + col0;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (col0 + 4 * q < P.N) {
-                                uint4 w = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                                *reinterpret_cast<uint4*>(dst + 4 * q) = w;
-                            }
-                        }
-                    }
-                }
-            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-                uint32_t vg[32], vu[32];
-                tmem_ld32(tacc + ch * 32, vg);
-                tmem_ld32(tacc + a.bn + ch * 32, vu);
-                tmem_ld_wait();
-                if (row_ok) {
-                    const long long off = row * P.ld + col0;
-                    __nv_bfloat16* gd = static_cast<__nv_bfloat16*>(P.out0) + off;
-                    __nv_bfloat16* ud = static_cast<__nv_bfloat16*>(P.out1) + off;
-                    __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(P.out2) + off;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (col0 + 8 * q < P.N) {
-                            uint32_t gw[4], uw[4], hw[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                gw[e] = pack_bf16(__uint_as_float(vg[8 * q + 2 * e]), __uint_as_float(vg[8 * q + 2 * e + 1]));
-                                uw[e] = pack_bf16(__uint_as_float(vu[8 * q + 2 * e]), __uint_as_float(vu[8 * q + 2 * e + 1]));
-                                const float h0 = silu_f(bf16_lo(gw[e])) * bf16_lo(uw[e]);
-                                const float h1 = silu_f(bf16_hi(gw[e])) * bf16_hi(uw[e]);
-                                hw[e] = pack_bf16(h0, h1);
-                            }
-                            *reinterpret_cast<uint4*>(gd + 8 * q) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
-                            *reinterpret_cast<uint4*>(ud + 8 * q) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
-                            *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                        }
-                    }
-                }
-            } else {  // EPI_SWIGLU_BWD
-                uint4 gv[4], uv[4];
-                const long long off = row * P.ld + col0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (row_ok && col0 + 8 * q < P.N) {
-                        gv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.in0) + off + 8 * q);
-                        uv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(P.in1) + off + 8 * q);
-                    } else {
-                        gv[q] = make_uint4(0, 0, 0, 0);
-                        uv[q] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-                uint32_t v[32];
-                tmem_ld32(tacc + ch * 32, v);
-                tmem_ld_wait();
-                if (row_ok) {
-                    __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(P.out0) + off;
-                    __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(P.out1) + off;
-                    __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(P.out2) + off;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (col0 + 8 * q < P.N) {
-                            const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-                            const uint32_t uw[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
-                            uint32_t dgw[4], duw[4], hw[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float dg2[2], du2[2], h2[2];
-#pragma unroll
-                                for (int hsel = 0; hsel < 2; ++hsel) {
-                                    const float gx = hsel ? bf16_hi(gw[e]) : bf16_lo(gw[e]);
-                                    const float ux = hsel ? bf16_hi(uw[e]) : bf16_lo(uw[e]);
-                                    const float dh = __uint_as_float(v[8 * q + 2 * e + hsel]);
-                                    const float sg = __frcp_rn(1.0f + __expf(-gx));
-                                    const float sl = gx * sg;
-                                    du2[hsel] = dh * sl;
-                                    dg2[hsel] = dh * ux * sg * (1.0f + gx * (1.0f - sg));
-                                    h2[hsel] = sl * ux;
-                                }
-                                dgw[e] = pack_bf16(dg2[0], dg2[1]);
-                                duw[e] = pack_bf16(du2[0], du2[1]);
-                                hw[e] = pack_bf16(h2[0], h2[1]);
-                            }
-                            *reinterpret_cast<uint4*>(dgd + 8 * q) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                            *reinterpret_cast<uint4*>(dud + 8 * q) = make_uint4(duw[0], duw[1], duw[2], duw[3]);
-                            *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                        }
-                    }
-                }
-            }
-        }
+        epilogue_tile<NACC, EPI>(o, row, t.nb * a.bn, a.bn, tacc);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(c.acce + 8u * abuf);
