@@ -1,6 +1,6 @@
-// Small bandwidth-bound kernels around the GEMMs: the deterministic split-K
-// reduction that finishes every rank-r product, the transpose of the adapter
-// B matrices into K-major operands, and the block-int4 dequantisation.
+// Small bandwidth-bound kernels around the GEMMs: the transpose of the
+// adapter B matrices into K-major operands, and the block-int4
+// dequantisation.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -11,41 +11,27 @@ namespace lmlp {
 constexpr int kRedRows = 32;
 constexpr int kRedMaxCols = 256;
 
-// Sum `splits` fp32 partial tiles P[s][m][col0 + j] in split order, scale, and
-// write bf16 to up to two places: row-major rm[m][j] and transposed tr[j][m].
-// One block handles 32 rows and all `ncols` (<= 256) columns.
-__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ P, int splits,
-                                                              long long split_stride, int M, int ldp, int col0,
-                                                              int ncols, float scale, __nv_bfloat16* rm,
-                                                              long long ld_rm, __nv_bfloat16* tr, long long ld_tr) {
-    __shared__ float tile[kRedRows][kRedMaxCols + 1];
-    const int m0 = blockIdx.x * kRedRows;
-    for (int i = threadIdx.x; i < kRedRows * ncols; i += blockDim.x) {
-        const int rr = i / ncols, j = i - rr * ncols;
-        const int m = m0 + rr;
-        float acc = 0.0f;
-        if (m < M) {
-            const float* p = P + static_cast<long long>(m) * ldp + col0 + j;
-            for (int s = 0; s < splits; ++s) acc += p[s * split_stride];
-        }
-        acc *= scale;
-        tile[rr][j] = acc;
-        if (rm != nullptr && m < M) rm[static_cast<long long>(m) * ld_rm + j] = __float2bfloat16_rn(acc);
-    }
-    if (tr == nullptr) return;
-    __syncthreads();
-    for (int i = threadIdx.x; i < kRedRows * ncols; i += blockDim.x) {
-        const int j = i / kRedRows, rr = i - j * kRedRows;
-        const int m = m0 + rr;
-        if (m < M) tr[static_cast<long long>(j) * ld_tr + m] = __float2bfloat16_rn(tile[rr][j]);
-    }
-}
+// Up to three transposes out_i[c][r] = in_i[r][c] of bf16 [R_i, C] matrices
+// (the adapter B matrices, C = rank <= 256), 32 rows per block.
+struct TransposeJobs {
+    const __nv_bfloat16* in[3];
+    __nv_bfloat16* out[3];
+    int R[3];
+    int C;
+    int n;
+};
 
-// out[c][r] = in[r][c] for a bf16 [R, C] matrix with C <= 256 (an adapter B).
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, int R, int C,
-                                                             __nv_bfloat16* __restrict__ out) {
+__global__ void __launch_bounds__(256) transpose3_bf16_kernel(const TransposeJobs jobs) {
     __shared__ __nv_bfloat16 tile[kRedRows][kRedMaxCols + 2];
-    const int r0 = blockIdx.x * kRedRows;
+    int blk = blockIdx.x, job = 0;
+    while (job < jobs.n - 1 && blk >= (jobs.R[job] + kRedRows - 1) / kRedRows) {
+        blk -= (jobs.R[job] + kRedRows - 1) / kRedRows;
+        ++job;
+    }
+    const __nv_bfloat16* in = jobs.in[job];
+    __nv_bfloat16* out = jobs.out[job];
+    const int R = jobs.R[job], C = jobs.C;
+    const int r0 = blk * kRedRows;
     for (int i = threadIdx.x; i < kRedRows * C; i += blockDim.x) {
         const int rr = i / C, c = i - rr * C;
         if (r0 + rr < R) tile[rr][c] = in[static_cast<long long>(r0 + rr) * C + c];

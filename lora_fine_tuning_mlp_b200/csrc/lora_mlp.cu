@@ -215,14 +215,32 @@ struct GemmBuilder {
         s.kblocks = ceil_div(k_len, kBK);
         p->nkb += s.kblocks;
     }
-    void finish() {
-        int u = 0;
+    // Finalise problem p in-kernel (see Prob): scale, bf16 row-major and/or transposed outputs.
+    void fin(Prob* p, float scale, int fin_cols, void* rm, long long ld_rm, void* tr0, void* tr1, long long ld_tr,
+             int tr_split) {
+        p->scale = scale;
+        p->fin_cols = fin_cols;
+        p->rm = rm;
+        p->ld_rm = ld_rm;
+        p->tr0 = tr0;
+        p->tr1 = tr1;
+        p->ld_tr = ld_tr;
+        p->tr_split = tr_split;
+        p->counters = reinterpret_cast<int*>(1);  // placeholder: assigned in finish()
+    }
+    void finish(int* counters) {
+        int u = 0, c = 0;
         for (int i = 0; i < a.nprobs; ++i) {
             Prob& p = a.prob[i];
             if (p.splits > p.nkb) p.splits = p.nkb;
             if (p.splits < 1) p.splits = 1;
             p.unit0 = u;
             u += p.tiles_m * p.tiles_n * p.splits;
+            if (p.counters != nullptr) {
+                if (counters == nullptr || p.tiles_n != 1) ok = false;
+                p.counters = counters + c;
+                c += p.tiles_m * p.tiles_n;
+            }
         }
         a.total_units = u;
         units = u;
@@ -230,9 +248,9 @@ struct GemmBuilder {
 };
 
 template <int NACC, bool A_MN, bool B_MN, int EPI>
-int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name) {
+int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int* counters = nullptr) {
+    b.finish(counters);
     if (!b.ok) return LORA_MLP_ERR_CUDA;
-    b.finish();
     GemmArgs& a = b.a;
     a.b_bytes = static_cast<uint32_t>(B_MN ? (a.bn / 64) * 8192 : a.bn * 128);
     const uint32_t stage_bytes = kATileBytes + NACC * a.b_bytes;
@@ -349,25 +367,13 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name) {
     return last_launch_error();
 }
 
-int launch_reduce(const float* P, int splits, long long split_stride, int M, int ldp, int col0, int ncols,
-                  float scale, void* rm, long long ld_rm, void* tr, long long ld_tr, cudaStream_t st,
-                  const char* name) {
-    if (ncols > kRedMaxCols) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
-    {
-        LaunchScope scope(name, st);
-        reduce_partials_kernel<<<ceil_div(M, kRedRows), 256, 0, st>>>(
-            P, splits, split_stride, M, ldp, col0, ncols, scale, static_cast<__nv_bfloat16*>(rm), ld_rm,
-            static_cast<__nv_bfloat16*>(tr), ld_tr);
-    }
-    return last_launch_error();
-}
-
-int launch_transpose(const void* in, int64_t R, int64_t C, void* out, cudaStream_t st) {
+// Transpose up to three adapter B matrices [R_i, C] -> [C, R_i] in one launch.
+int launch_transpose3(const TransposeJobs& jobs, cudaStream_t st) {
+    int blocks = 0;
+    for (int i = 0; i < jobs.n; ++i) blocks += ceil_div(jobs.R[i], kRedRows);
     {
         LaunchScope scope("transpose_B", st);
-        transpose_bf16_kernel<<<ceil_div(R, kRedRows), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
-                                                                       static_cast<int>(R), static_cast<int>(C),
-                                                                       static_cast<__nv_bfloat16*>(out));
+        transpose3_bf16_kernel<<<blocks, 256, 0, st>>>(jobs);
     }
     return last_launch_error();
 }
@@ -389,12 +395,25 @@ int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t
 }
 
 // ----------------------------------------------------------------------------- layout
+// Split-K factor for a skinny product with `tiles` output tiles and `nkb`
+// K blocks: minimise the estimated makespan of the persistent grid, i.e. the
+// number of unit rounds per SM times the K blocks of one unit, plus a small
+// per-unit cost.  Depends only on the shape (a fixed 148-CTA grid), so the
+// workspace size does not depend on the device.
 int splits_for(int64_t tiles, int64_t nkb) {
-    int64_t s = kTargetCtas / (tiles > 0 ? tiles : 1);
-    if (s < 1) s = 1;
-    if (s > nkb) s = nkb;
-    if (s > kMaxSplits) s = kMaxSplits;
-    return static_cast<int>(s < 1 ? 1 : s);
+    if (tiles < 1) tiles = 1;
+    int best = 1;
+    double best_cost = 1e30;
+    const int64_t smax = std::min<int64_t>(kMaxSplits, std::max<int64_t>(nkb, 1));
+    for (int64_t sp = 1; sp <= smax; ++sp) {
+        const int64_t rounds = (tiles * sp + kTargetCtas - 1) / kTargetCtas;
+        const double cost = static_cast<double>(rounds) * (static_cast<double>(nkb) / sp + 2.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = static_cast<int>(sp);
+        }
+    }
+    return best;
 }
 
 struct Plan {
@@ -404,9 +423,10 @@ struct Plan {
     int bn_r, bn_2r;
     int sp_f0, sp_f2, sp_b0a, sp_b0b, sp_b2, sp_b3a, sp_b3b, sp_b5;
     // forward workspace
-    size_t f_h, f_sgu, f_sd, f_part, f_w[3], f_total;
+    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_w[3], f_total;
     // backward workspace
-    size_t b_dg, b_du, b_h, b_bdT, b_bgT, b_buT, b_td, b_tdT, b_tgu, b_tguT, b_part, b_w[3], b_total;
+    size_t b_dg, b_du, b_h, b_bdT, b_bgT, b_buT, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_w[3], b_total;
+    size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
     // saved
     size_t s_sgT, s_suT, s_sdT, s_total;
 };
@@ -451,6 +471,11 @@ Plan make_plan(const lora_mlp_shape& sh) {
     size_t part = p.sp_f0 * N * 2 * r;
     part = std::max(part, p.sp_f2 * N * r);
     p.f_part = f.take(part * f32);
+    const size_t ctr_slots = 2 * static_cast<size_t>(std::max<int64_t>(
+                                     std::max<int64_t>(ceil_div(p.N, kBM), ceil_div(p.d_ff, kBM)), ceil_div(p.d, kBM))) +
+                             8;
+    p.ctr_bytes = ctr_slots * sizeof(int);
+    p.f_ctr = f.take(p.ctr_bytes);
     for (int i = 0; i < 3; ++i) p.f_w[i] = p.int4 ? f.take(wsz[i]) : 0;
     p.f_total = f.off;
 
@@ -472,6 +497,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     bpart = std::max(bpart, p.sp_b3b * dff * 2 * r);
     bpart = std::max(bpart, p.sp_b5 * d * 2 * r);
     p.b_part = b.take(bpart * f32);
+    p.b_ctr = b.take(p.ctr_bytes);
     for (int i = 0; i < 3; ++i) p.b_w[i] = p.int4 ? b.take(wsz[i]) : 0;
     p.b_total = b.off;
 
@@ -579,10 +605,12 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     __nv_bfloat16* Sgu = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_sgu);
     __nv_bfloat16* Sd = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_sd);
     float* part = reinterpret_cast<float*>(ws + pl.f_part);
+    int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
+    if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
     const void* W[3];
     LMLP_TRY(frozen_weights(pl, w, ws, pl.f_w, di.sms, st, W));
 
-    {  // F0: [S_g | S_u] = s X [Ag; Au]^T
+    {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ax = b.a_k(X, N, d, d);
         const int bg = b.b_k(w->Ag, r, d, d);
@@ -593,9 +621,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         p->out1 = part + r;
         p->ld = 2 * r;
         p->split_stride = N * 2 * r;
-        LMLP_TRY((launch_gemm<2, false, false, EPI_F32>(b, di.sms, st, "F0_lowrank_in")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * 2 * r, static_cast<int>(N), static_cast<int>(2 * r), 0,
-                               static_cast<int>(2 * r), pl.s, Sgu, 2 * r, sv + pl.s_sgT, pl.ldN, st, "F0_reduce"));
+        b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
+        LMLP_TRY((launch_gemm<2, false, false, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
         PairBuilder b(N, dff, 128);
@@ -613,7 +640,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.ld = dff;
         LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu")));
     }
-    {  // F2: S_d = s h Ad^T
+    {  // F2: S_d = s h Ad^T  -> Sd [N, r] and saved S_d^T [r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ah = b.a_k(h, N, dff, dff);
         const int bad = b.b_k(w->Ad, r, dff, dff);
@@ -622,9 +649,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         p->out0 = part;
         p->ld = r;
         p->split_stride = N * r;
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "F2_lowrank_mid")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * r, static_cast<int>(N), static_cast<int>(r), 0,
-                               static_cast<int>(r), pl.s, Sd, r, sv + pl.s_sdT, pl.ldN, st, "F2_reduce"));
+        b.fin(p, pl.s, static_cast<int>(r), Sd, r, sv + pl.s_sdT, nullptr, pl.ldN, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
     }
     {  // F3: out = h Wd^T + S_d Bd^T
         PairBuilder b(N, d, 256);
@@ -668,6 +694,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     __nv_bfloat16* Tgu = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tgu);
     __nv_bfloat16* TguT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tguT);
     float* part = reinterpret_cast<float*>(ws + pl.b_part);
+    int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
+    if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
@@ -675,11 +703,22 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     LMLP_TRY(frozen_weights(pl, w, ws, pl.b_w, di.sms, st, W));
 
     // adapter B matrices as K-major operands of the rank-r projections
-    LMLP_TRY(launch_transpose(w->Bd, d, r, BdT, st));
-    LMLP_TRY(launch_transpose(w->Bg, dff, r, BgT, st));
-    LMLP_TRY(launch_transpose(w->Bu, dff, r, BuT, st));
+    {
+        TransposeJobs jobs{};
+        jobs.n = 3;
+        jobs.C = static_cast<int>(r);
+        const void* ins[3] = {w->Bd, w->Bg, w->Bu};
+        void* outs[3] = {BdT, BgT, BuT};
+        const int64_t rows[3] = {d, dff, dff};
+        for (int i = 0; i < 3; ++i) {
+            jobs.in[i] = static_cast<const __nv_bfloat16*>(ins[i]);
+            jobs.out[i] = static_cast<__nv_bfloat16*>(outs[i]);
+            jobs.R[i] = static_cast<int>(rows[i]);
+        }
+        LMLP_TRY(launch_transpose3(jobs, st));
+    }
 
-    {  // B0a: T_d = s dOut Bd
+    {  // B0a: T_d = s dOut Bd  -> Td [N, r] and Td^T [r, ldN]
         GemmBuilder b(pl.bn_r);
         const int a = b.a_k(dOut, N, d, d);
         const int bb = b.b_k(BdT, r, d, d);
@@ -688,9 +727,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p->out0 = part;
         p->ld = r;
         p->split_stride = N * r;
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B0_lowrank_out")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * r, static_cast<int>(N), static_cast<int>(r), 0,
-                               static_cast<int>(r), pl.s, Td, r, TdT, ldN, st, "B0_reduce"));
+        b.fin(p, pl.s, static_cast<int>(r), Td, r, TdT, nullptr, ldN, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B0_lowrank_out", ctr)));
     }
     {  // B0b: dBd = dOut^T S_d
         GemmBuilder b(pl.bn_r);
@@ -701,9 +739,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p->out0 = part;
         p->ld = r;
         p->split_stride = d * r;
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B0_dBd")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, d * r, static_cast<int>(d), static_cast<int>(r), 0,
-                               static_cast<int>(r), 1.0f, grads->dBd, r, nullptr, 0, st, "B0_dBd_reduce"));
+        b.fin(p, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B0_dBd", ctr)));
     }
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
         PairBuilder b(N, dff, 256);
@@ -722,7 +759,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p.ld = dff;
         LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd")));
     }
-    {  // B2: dAd = T_d^T h
+    {  // B2: dAd = T_d^T h  (written transposed: dAd [r, d_ff])
         GemmBuilder b(pl.bn_r);
         const int a = b.a_mn(hb, N, dff, dff);
         const int bb = b.b_k(TdT, r, N, ldN);
@@ -731,11 +768,10 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p->out0 = part;
         p->ld = r;
         p->split_stride = dff * r;
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B2_dAd")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, dff * r, static_cast<int>(dff), static_cast<int>(r), 0,
-                               static_cast<int>(r), 1.0f, nullptr, 0, grads->dAd, dff, st, "B2_reduce"));
+        b.fin(p, 1.0f, static_cast<int>(r), nullptr, 0, grads->dAd, nullptr, dff, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B2_dAd", ctr)));
     }
-    {  // B3a: T_g = s dg Bg, T_u = s du Bu
+    {  // B3a: T_g = s dg Bg, T_u = s du Bu  -> Tgu [N, 2r] and Tgu^T [2r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ag = b.a_k(dg, N, dff, dff);
         const int au = b.a_k(du, N, dff, dff);
@@ -746,14 +782,14 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p0->out0 = part;
         p0->ld = 2 * r;
         p0->split_stride = N * 2 * r;
+        b.fin(p0, pl.s, static_cast<int>(r), Tgu, 2 * r, TguT, nullptr, ldN, static_cast<int>(r));
         Prob* p1 = b.prob(N, r, pl.sp_b3a);
         b.seg(p1, au, bu, -1, dff);
         p1->out0 = part + r;
         p1->ld = 2 * r;
         p1->split_stride = N * 2 * r;
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B3_lowrank_gu")));
-        LMLP_TRY(launch_reduce(part, b.a.prob[0].splits, N * 2 * r, static_cast<int>(N), static_cast<int>(2 * r), 0,
-                               static_cast<int>(2 * r), pl.s, Tgu, 2 * r, TguT, ldN, st, "B3_reduce"));
+        b.fin(p1, pl.s, static_cast<int>(r), Tgu + r, 2 * r, TguT + r * ldN, nullptr, ldN, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B3_lowrank_gu", ctr)));
     }
     {  // B3b: dBg = dg^T S_g, dBu = du^T S_u
         GemmBuilder b(pl.bn_r);
@@ -766,18 +802,14 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p0->out0 = part;
         p0->ld = 2 * r;
         p0->split_stride = dff * 2 * r;
+        b.fin(p0, 1.0f, static_cast<int>(r), grads->dBg, r, nullptr, nullptr, 0, static_cast<int>(r));
         Prob* p1 = b.prob(dff, r, pl.sp_b3b);
         b.seg(p1, au, bu, -1, N);
         p1->out0 = part + r;
         p1->ld = 2 * r;
         p1->split_stride = dff * 2 * r;
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B3_dBgu")));
-        const int sp = b.a.prob[0].splits;
-        LMLP_TRY(launch_reduce(part, sp, dff * 2 * r, static_cast<int>(dff), static_cast<int>(2 * r), 0,
-                               static_cast<int>(r), 1.0f, grads->dBg, r, nullptr, 0, st, "B3_dBg_reduce"));
-        LMLP_TRY(launch_reduce(part, sp, dff * 2 * r, static_cast<int>(dff), static_cast<int>(2 * r),
-                               static_cast<int>(r), static_cast<int>(r), 1.0f, grads->dBu, r, nullptr, 0, st,
-                               "B3_dBu_reduce"));
+        b.fin(p1, 1.0f, static_cast<int>(r), grads->dBu, r, nullptr, nullptr, 0, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B3_dBgu", ctr)));
     }
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
         PairBuilder b(N, d, 256);
@@ -797,7 +829,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.a.prob.ld = d;
         LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX")));
     }
-    {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]
+    {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]  (written transposed: dAg, dAu [r, d])
         GemmBuilder b(pl.bn_2r);
         const int a = b.a_mn(X, N, d, d);
         const int bb = b.b_k(TguT, 2 * r, N, ldN);
@@ -806,13 +838,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p->out0 = part;
         p->ld = 2 * r;
         p->split_stride = d * 2 * r;
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B5_dA_in")));
-        const int sp = b.a.prob[0].splits;
-        LMLP_TRY(launch_reduce(part, sp, d * 2 * r, static_cast<int>(d), static_cast<int>(2 * r), 0,
-                               static_cast<int>(r), 1.0f, nullptr, 0, grads->dAg, d, st, "B5_dAg_reduce"));
-        LMLP_TRY(launch_reduce(part, sp, d * 2 * r, static_cast<int>(d), static_cast<int>(2 * r),
-                               static_cast<int>(r), static_cast<int>(r), 1.0f, nullptr, 0, grads->dAu, d, st,
-                               "B5_dAu_reduce"));
+        b.fin(p, 1.0f, static_cast<int>(2 * r), nullptr, 0, grads->dAg, grads->dAu, d, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B5_dA_in", ctr)));
     }
     return LORA_MLP_OK;
 }

@@ -216,14 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
     const uint32_t ctl = base + args.stages * kPairStageBytes;
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
-    SmemCtl c;
-    c.full = ctl;
-    c.empty = ctl + 8u * kMaxStages;
-    c.accf = ctl + 8u * (2 * kMaxStages);
-    c.acce = c.accf + 16u;
-    c.drain = c.acce + 16u;
-    c.tmem_slot = c.drain + 8u;
-    c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
+    const SmemCtl c = make_ctl(ctl, ctl_ptr);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;

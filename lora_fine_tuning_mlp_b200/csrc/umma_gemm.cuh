@@ -37,7 +37,7 @@ constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxMaps = 12;
 constexpr int kMaxSegs = 4;
 constexpr int kMaxProbs = 2;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kGemmThreads = 192;
 
 struct Seg {
@@ -58,6 +58,20 @@ struct Prob {
     const void* in1;
     long long ld;            // row stride (elements) of out*/in*
     long long split_stride;  // elements between split-K partials (EPI_F32)
+    // Split-K finalisation (EPI_F32 with counters != nullptr): the last CTA to
+    // finish a tile sums the splits' fp32 partials in split order (so results
+    // do not depend on timing), scales, and writes bf16 row-major to rm
+    // [M, fin_cols] and/or transposed: column j < tr_split to tr0[j][m], the
+    // rest to tr1[j - tr_split][m].  A tile covers all columns (tiles_n = 1).
+    int* counters;  // one per tile, zero before the launch; reset by the last CTA
+    float scale;
+    int fin_cols;
+    int tr_split;
+    void* rm;
+    long long ld_rm;
+    void* tr0;
+    void* tr1;
+    long long ld_tr;
 };
 
 struct alignas(64) GemmArgs {
@@ -100,6 +114,7 @@ struct SmemCtl {
     uint32_t full, empty, accf, acce, drain;  // barrier array bases (shared addresses)
     uint32_t tmem_slot;
     volatile int* abort_flag;
+    volatile int* fin_flag;
 };
 
 // Bounded wait that also gives up as soon as another role of this CTA gave up.
@@ -249,6 +264,54 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
     }
 }
 
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Called by all four epilogue warps after their rows of a split's partial
+// tile are stored.  The CTA that completes a tile last reduces it.
+__device__ __forceinline__ void splitk_finalize(const Prob& P, const Unit& t, int row, volatile int* fin_flag) {
+    __threadfence();
+    epi_bar();
+    if (threadIdx.x == 64) {
+        int* ctr = P.counters + t.mb * P.tiles_n + t.nb;
+        const int old = atomicAdd(ctr, 1);
+        const int last = old == P.splits - 1;
+        if (last) *ctr = 0;
+        *fin_flag = last;
+    }
+    epi_bar();
+    if (!*fin_flag) return;
+    __threadfence();
+    if (row >= P.M) return;
+    const float* src = static_cast<const float*>(P.out0) + row * P.ld;
+    __nv_bfloat16* rm = static_cast<__nv_bfloat16*>(P.rm);
+    __nv_bfloat16* tr0 = static_cast<__nv_bfloat16*>(P.tr0);
+    __nv_bfloat16* tr1 = static_cast<__nv_bfloat16*>(P.tr1);
+    for (int j = 0; j < P.fin_cols; j += 8) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        for (int sp = 0; sp < P.splits; ++sp) {
+            const float4* q = reinterpret_cast<const float4*>(src + sp * P.split_stride + j);
+            const float4 a0 = __ldcg(q), a1 = __ldcg(q + 1);
+            acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
+            acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = pack_bf16(acc[2 * e] * P.scale, acc[2 * e + 1] * P.scale);
+        if (rm != nullptr) *reinterpret_cast<uint4*>(rm + row * P.ld_rm + j) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (tr0 != nullptr) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int jj = j + e;
+                const __nv_bfloat16 v = __ushort_as_bfloat16(static_cast<unsigned short>(e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu));
+                if (jj < P.tr_split) tr0[jj * P.ld_tr + row] = v;
+                else tr1[(jj - P.tr_split) * P.ld_tr + row] = v;
+            }
+        }
+    }
+}
+
 template <int NACC, int EPI>
 __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_base, const SmemCtl& c) {
     const int warp = threadIdx.x >> 5;
@@ -282,6 +345,9 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
             abuf = 0;
             aphase ^= 1u;
         }
+        if constexpr (EPI == EPI_F32) {
+            if (P.counters != nullptr) splitk_finalize(P, t, row, c.fin_flag);
+        }
     }
 }
 
@@ -289,6 +355,20 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
 // kernel
 
 __host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 5) + 16u; }
+
+// Barrier/flag block that follows the operand stages in shared memory.
+__device__ __forceinline__ SmemCtl make_ctl(uint32_t ctl, uint8_t* ctl_ptr) {
+    SmemCtl c;
+    c.full = ctl;
+    c.empty = ctl + 8u * kMaxStages;
+    c.accf = ctl + 8u * (2 * kMaxStages);
+    c.acce = c.accf + 16u;
+    c.drain = c.acce + 16u;
+    c.tmem_slot = c.drain + 8u;
+    c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
+    c.fin_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 8u - ctl));
+    return c;
+}
 
 __host__ __device__ inline uint32_t gemm_tmem_cols(int nacc, int bn) {
     uint32_t need = 2u * nacc * bn, cols = 32;
@@ -305,14 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
     const uint32_t ctl = base + args.stages * stage_bytes;
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
-    SmemCtl c;
-    c.full = ctl;
-    c.empty = ctl + 8u * kMaxStages;
-    c.accf = ctl + 8u * (2 * kMaxStages);
-    c.acce = c.accf + 16u;
-    c.drain = c.acce + 16u;
-    c.tmem_slot = c.drain + 8u;
-    c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
+    const SmemCtl c = make_ctl(ctl, ctl_ptr);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;

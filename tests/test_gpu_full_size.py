@@ -1,0 +1,86 @@
+"""Parity at the workloads' full sizes, through the same calls bench.py times.
+
+Outputs the oracle can compute one by one are compared on samples: rows of
+out, g, u and dX for sampled tokens (every token is independent), and rows of
+dBg, dBu for sampled hidden features (column f of G, U and dH needs only
+column f of the projections).  The Llama-3-8B-shaped workloads (bf16 and
+int4 weights) are also compared on every output against the full fp64
+oracle.  Tolerance as everywhere: max|gpu - oracle| / max|oracle| <= 2e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lora_fine_tuning_mlp_b200 import _lib, api
+from lora_fine_tuning_mlp_b200 import build as libbuild
+from lora_fine_tuning_mlp_b200 import inputs as synth
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+TOL = 2e-2
+GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
+_cache = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    libbuild.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(0)
+
+
+def relerr(a, b):
+    den = float(np.max(np.abs(b)))
+    return float(np.max(np.abs(a - b))) / (den if den > 0 else 1.0)
+
+
+def gpu_run(cfg):
+    if cfg.name in _cache:
+        return _cache[cfg.name]
+    _cache.clear()
+    torch.cuda.empty_cache()
+    inp = synth.make_inputs(cfg)
+    dev = torch.device("cuda:0")
+    w = api.weights_from_host(inp, cfg.alpha, dev)
+    X = api.to_device_bf16(inp["X"], dev)
+    dOut = api.to_device_bf16(inp["dOut"], dev)
+    out, saved = api.forward(X, w)
+    dX, grads = api.backward(X, w, saved, dOut)
+    torch.cuda.synchronize()
+    assert _lib.device_status(None) == 0
+    res = {"out": out, "g": saved.g, "u": saved.u, "dX": dX}
+    res.update(grads)
+    res = {k: v.float().cpu().numpy().astype(np.float64) for k, v in res.items()}
+    del out, saved, dX, grads, w, X, dOut
+    torch.cuda.empty_cache()
+    _cache[cfg.name] = (inp, res)
+    return inp, res
+
+
+FULL = [c for c in synth.CONFIGS if c.name != "tiny"]
+
+
+@pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
+def test_sampled_rows_and_features(cfg):
+    inp, got = gpu_run(cfg)
+    rng = np.random.default_rng(cfg.seed)
+    rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.choice(cfg.N, 30, replace=False)]))
+    ref = oracle.token_rows(inp, cfg.alpha, rows)
+    errs = {k: relerr(got[g][rows], ref[k]) for g, k in (("out", "out"), ("g", "G"), ("u", "U"), ("dX", "dX"))}
+    feats = np.unique(np.concatenate([[0, cfg.d_ff - 1], rng.choice(cfg.d_ff, 14, replace=False)]))
+    fr = oracle.up_gate_feature_grads(inp, cfg.alpha, feats)
+    errs["dBg"] = relerr(got["dBg"][feats], fr["dBg"])
+    errs["dBu"] = relerr(got["dBu"][feats], fr["dBu"])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, f"{cfg.name}: {bad} (all {errs})"
+
+
+@pytest.mark.parametrize("cfg", [synth.BY_NAME["llama3_8b_mlp"], synth.BY_NAME["llama3_8b_mlp_int4"]],
+                         ids=lambda c: c.name)
+def test_every_output_against_full_oracle(cfg):
+    inp, got = gpu_run(cfg)
+    ref = oracle.forward_backward(inp, cfg.alpha)
+    errs = {k: relerr(got[k], ref[k]) for k in ("out", "dX") + GRADS}
+    errs["g"] = relerr(got["g"], ref["G"])
+    errs["u"] = relerr(got["u"], ref["U"])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, f"{cfg.name}: {bad} (all {errs})"
