@@ -139,6 +139,34 @@ int lora_mlp_timing_collect(lora_mlp_kernel_time* out, int max, int* count);
 /* Number of kernels this library has launched in this process (all devices). */
 int64_t lora_mlp_launch_count(void);
 
+/* ---------------------------------------------------------------------------
+ * Forward pass that allocates nothing.  (The pages have no counterpart: this
+ * entry point exists for how the library is called, not for the method.)
+ *
+ * Some callers cannot allocate device memory: a plugin running inside a host
+ * framework that owns all device memory and forbids allocations behind its
+ * allocator, a latency-critical loop where cudaMalloc's implicit device
+ * synchronisation cannot be afforded, or a deployment whose memory is
+ * budgeted up front.  For them this call does what lora_mlp_forward does
+ * with the same arguments, but takes no workspace: its scratch is a fixed
+ * device array of LORA_MLP_NOALLOC_SCRATCH_BYTES inside the library.  The
+ * caller still passes X, out, g, u and saved.
+ *  - Shapes whose forward workspace (lora_mlp_sizes) exceeds
+ *    LORA_MLP_NOALLOC_SCRATCH_BYTES are rejected with
+ *    LORA_MLP_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
+ *  - The array is reserved on a device when this entry point is first used
+ *    there and held until the process exits.  That first call on a device
+ *    also looks up the array's device address and caches it; make it before
+ *    any stream capture begins.
+ *  - Every call on a device shares the one array.  Calls whose work may
+ *    overlap on the GPU (unordered streams) race and corrupt each other's
+ *    results: order them, e.g. on one stream.  Each call clears the part of
+ *    the array that must start at zero, so nothing carries over between calls.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called. */
+#define LORA_MLP_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int lora_mlp_forward_noalloc(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out,
+                             void* g, void* u, void* saved, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,6 +38,7 @@ SYMBOLS = (
     "lora_mlp_timing_enable",
     "lora_mlp_timing_collect",
     "lora_mlp_launch_count",
+    "lora_mlp_forward_noalloc",
 )
 
 
@@ -92,9 +93,12 @@ def lib() -> ctypes.CDLL:
             L.lora_mlp_timing_enable.argtypes = [ctypes.c_int]
             L.lora_mlp_timing_collect.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int,
                                                   ctypes.POINTER(ctypes.c_int)]
+            L.lora_mlp_forward_noalloc.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
+                                                   vp, vp]
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
-            for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_backward", "lora_mlp_dequant_int4",
+            for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
+                         "lora_mlp_dequant_int4",
                          "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
@@ -127,6 +131,13 @@ def sizes(shape: Shape):
 def forward(shape: Shape, weights: Weights, X, out, g, u, saved, workspace, workspace_bytes, stream) -> int:
     return lib().lora_mlp_forward(ctypes.byref(shape), ctypes.byref(weights), X, out, g, u, saved, workspace,
                                   workspace_bytes, stream)
+
+
+def forward_noalloc(shape: Shape, weights: Weights, X, out, g, u, saved, stream) -> int:
+    return lib().lora_mlp_forward_noalloc(ctypes.byref(shape), ctypes.byref(weights), X, out, g, u, saved, stream)
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 def backward(shape: Shape, weights: Weights, X, g, u, saved, dOut, dX, grads: Grads, workspace,

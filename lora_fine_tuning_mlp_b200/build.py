@@ -13,7 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = [os.path.join(CSRC, "lora_mlp.cu")]
+SOURCES = [os.path.join(CSRC, "lora_mlp.cu"), os.path.join(CSRC, "noalloc.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "epilogue.cuh", "umma_gemm.cuh", "umma2_gemm.cuh", "aux_kernels.cuh")] + [
     os.path.join(ROOT, "include", "lora_mlp.h")]
 OUT = os.path.join(HERE, "liblora_mlp.so")
