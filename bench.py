@@ -50,6 +50,35 @@ def load_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
+def csrc_sha256() -> str:
+    """Hash of the CUDA sources, to tell whether a stored ncu figure still applies."""
+    import hashlib
+    d = os.path.join(ROOT, "lora_fine_tuning_mlp_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    with open(os.path.join(ROOT, "include", "lora_mlp.h"), "rb") as fh:
+        h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when there is none or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if rec.get("csrc_sha256") != csrc_sha256():
+        return None
+    return rec.get(workload, {}).get(kernel, {}).get("dram_bytes")
+
+
 def gemm_flops(cfg) -> dict:
     """Algorithmic flops of each tensor-core GEMM launch (2 per multiply-add)."""
     N, d, f, r = cfg.N, cfg.d, cfg.d_ff, cfg.r
@@ -337,7 +366,7 @@ def b200_arm(args, cfg):
         achieved = fl[dom] / (avg_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": ncu_traffic(cfg.name, dom),
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                 "flops_per_launch": fl[dom], "avg_launch_ms": avg_ms}
 
@@ -377,7 +406,7 @@ def b200_arm(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=("b200", "reference"))
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
