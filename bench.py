@@ -247,7 +247,7 @@ def config_dict(cfg):
             "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
             "l2": "no flush: inputs larger than L2 (frozen weights %.0f MB > 126 MB)" % (
                 3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6),
-            "parallelism": "replicas" }
+            "parallelism": "replicas"}
 
 
 def b200_arm(args, cfg):
@@ -256,14 +256,12 @@ def b200_arm(args, cfg):
 
     from lora_fine_tuning_mlp_b200 import _lib, api
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from lora_fine_tuning_mlp_b200 import replicas
+
+    rank, local, world = replicas.world()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", device=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -284,9 +282,7 @@ def b200_arm(args, cfg):
         o, saved = api.forward(x, w, out=out, workspace=wsf)
         api.backward(x, w, saved, g_out, dX=dX, grads=grads, workspace=wsb)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = replicas.barrier
 
     for _ in range(args.warmup):
         step()
@@ -312,44 +308,31 @@ def b200_arm(args, cfg):
     launches = _lib.launch_count() - launches0
     recs = _lib.timing_collect()
     _lib.timing_enable(False)
-    ms = t0.elapsed_time(t1)
-    ms_max = ms
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = replicas.max_over_ranks(t0.elapsed_time(t1), device=dev)
 
-    # ---- end-to-end through the public API with host buffers
-    Xh = torch.from_numpy(inp["X"].view("int16")).view(torch.bfloat16).pin_memory()
-    dOh = torch.from_numpy(inp["dOut"].view("int16")).view(torch.bfloat16).pin_memory()
-    gh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in grads.items()}
-    Xd, dOd = torch.empty_like(X), torch.empty_like(dOut)
-    h2d = Xh.numel() * 2 + dOh.numel() * 2
-    d2h = sum(v.numel() * 2 for v in gh.values())
+    # ---- end-to-end through the public API with host buffers: every step copies
+    # its X and dOut from pinned host memory (overlapped with the previous
+    # step's compute) and reads its six adapter gradients back to the host.
+    Xh = [torch.from_numpy(inp["X"].view("int16")).view(torch.bfloat16).pin_memory() for _ in range(2)]
+    dOh = [torch.from_numpy(inp["dOut"].view("int16")).view(torch.bfloat16).pin_memory() for _ in range(2)]
+    trainer = api.HostBatchTrainer(w, N, dev)
+    h2d, d2h = trainer.h2d_bytes(), trainer.d2h_bytes()
 
-    def e2e_step():
-        Xd.copy_(Xh, non_blocking=True)
-        dOd.copy_(dOh, non_blocking=True)
-        step(Xd, dOd)
-        for k in gh:
-            gh[k].copy_(grads[k], non_blocking=True)
+    def run_e2e(n):
+        for i in range(n):
+            nxt = (i + 1) % 2 if i + 1 < n else None
+            trainer.step(Xh[i % 2], dOh[i % 2], None if nxt is None else Xh[nxt], None if nxt is None else dOh[nxt])
 
-    for _ in range(2):
-        e2e_step()
+    run_e2e(3)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    run_e2e(args.steps)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ems = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ems], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
+    ems = replicas.max_over_ranks(e0.elapsed_time(e1), device=dev)
 
     # ---- per-kernel breakdown and the dominant kernel's roofline
     per = {}
@@ -370,11 +353,10 @@ def b200_arm(args, cfg):
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                 "flops_per_launch": fl[dom], "avg_launch_ms": avg_ms}
 
-    if world > 1:
-        dist.barrier()
+    barrier()
     if rank == 0:
         per_step_ms = ms_max / args.steps
-        value = world * N * args.steps / (ms_max * 1e-3)
+        value = replicas.job_throughput(N, args.steps, ms_max, world)
         tflops = world * cfg.flops() * args.steps / (ms_max * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -385,9 +367,10 @@ def b200_arm(args, cfg):
                 "measured_sustained": tflops / world / peaks["bf16_tflops_sustained"],
                 "nominal_2250": tflops / world / 2250.0},
             "roofline": roof,
-            "e2e": {"value": world * N * args.steps / (ems * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": replicas.job_throughput(N, args.steps, ems, world), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "what": "H2D of X and dOut from pinned host, forward+backward, D2H of the six adapter grads"},
+                    "what": "api.HostBatchTrainer: per step H2D of X and dOut from pinned host (overlapped with "
+                            "the previous step's compute), forward+backward, D2H of the six adapter grads"},
             "gpu_launches": launches,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
@@ -399,6 +382,7 @@ def b200_arm(args, cfg):
                                     "sample": f"{n} tokens of the {cfg.name} shapes, numpy fp64 oracle, {dt:.1f} s"}
         print(json.dumps(line), flush=True)
     if world > 1:
+        torch.cuda.synchronize()
         dist.destroy_process_group()
     return 0
 

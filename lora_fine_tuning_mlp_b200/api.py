@@ -222,3 +222,68 @@ def weights_from_host(inp: dict, alpha: float, device="cuda") -> MLPWeights:
 
 def to_device_bf16(a, device="cuda") -> torch.Tensor:
     return torch.from_numpy(a.view("int16")).view(BF16).to(device)
+
+
+class HostBatchTrainer:
+    """Forward + backward over batches that live in (pinned) host memory.
+
+    The host-to-device copy of the next batch runs on its own stream while the
+    current batch computes (two device buffers, ordered by CUDA events), and
+    each step's adapter gradients are copied back to pinned host memory.
+    Every step still moves its own inputs and result across PCIe; only the
+    overlap with compute is new.
+    """
+
+    def __init__(self, w: MLPWeights, N: int, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.w, self.N, self.dev = w, N, dev
+        d = w.d
+        self.X = [torch.empty((N, d), dtype=BF16, device=dev) for _ in range(2)]
+        self.dOut = [torch.empty((N, d), dtype=BF16, device=dev) for _ in range(2)]
+        self.out = torch.empty((N, d), dtype=BF16, device=dev)
+        self.dX = torch.empty((N, d), dtype=BF16, device=dev)
+        self.grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+        self.grads_host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in self.grads.items()}
+        self.wsf, self.wsb = Workspace(), Workspace()
+        self.copy_stream = torch.cuda.Stream(device=dev)
+        self.ready = [torch.cuda.Event(), torch.cuda.Event()]
+        self.free = [torch.cuda.Event(), torch.cuda.Event()]
+        self.slot = 0
+        self.primed = False
+
+    def _stage(self, slot, Xh, dOh):
+        with torch.cuda.stream(self.copy_stream):
+            self.copy_stream.wait_event(self.free[slot])
+            self.X[slot].copy_(Xh, non_blocking=True)
+            self.dOut[slot].copy_(dOh, non_blocking=True)
+            self.ready[slot].record(self.copy_stream)
+
+    def h2d_bytes(self) -> int:
+        return 2 * self.N * self.w.d * 2
+
+    def d2h_bytes(self) -> int:
+        return sum(v.numel() * v.element_size() for v in self.grads.values())
+
+    def step(self, Xh, dOh, next_Xh=None, next_dOh=None):
+        """One training step on host batch (Xh, dOh); if the next batch is
+        given, its copy is started so that it overlaps this step's compute.
+        Returns the dict of pinned host adapter gradients (valid once the
+        current stream has been synchronised)."""
+        cur = self.slot
+        if not self.primed:
+            self._stage(cur, Xh, dOh)
+            self.primed = True
+        nxt = cur ^ 1
+        if next_Xh is not None:
+            self._stage(nxt, next_Xh, next_dOh)
+        stream = torch.cuda.current_stream(self.dev)
+        stream.wait_event(self.ready[cur])
+        o, saved = forward(self.X[cur], self.w, out=self.out, workspace=self.wsf)
+        backward(self.X[cur], self.w, saved, self.dOut[cur], dX=self.dX, grads=self.grads, workspace=self.wsb)
+        self.free[cur].record(stream)
+        for k, v in self.grads.items():
+            self.grads_host[k].copy_(v, non_blocking=True)
+        self.slot = nxt
+        if next_Xh is None:
+            self.primed = False
+        return self.grads_host

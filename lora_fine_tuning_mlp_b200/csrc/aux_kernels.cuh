@@ -1,47 +1,10 @@
-// Small bandwidth-bound kernels around the GEMMs: the transpose of the
-// adapter B matrices into K-major operands, and the block-int4
-// dequantisation.
+// The block-int4 dequantisation of the frozen weights.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
 namespace lmlp {
-
-constexpr int kRedRows = 32;
-constexpr int kRedMaxCols = 256;
-
-// Up to three transposes out_i[c][r] = in_i[r][c] of bf16 [R_i, C] matrices
-// (the adapter B matrices, C = rank <= 256), 32 rows per block.
-struct TransposeJobs {
-    const __nv_bfloat16* in[3];
-    __nv_bfloat16* out[3];
-    int R[3];
-    int C;
-    int n;
-};
-
-__global__ void __launch_bounds__(256) transpose3_bf16_kernel(const TransposeJobs jobs) {
-    __shared__ __nv_bfloat16 tile[kRedRows][kRedMaxCols + 2];
-    int blk = blockIdx.x, job = 0;
-    while (job < jobs.n - 1 && blk >= (jobs.R[job] + kRedRows - 1) / kRedRows) {
-        blk -= (jobs.R[job] + kRedRows - 1) / kRedRows;
-        ++job;
-    }
-    const __nv_bfloat16* in = jobs.in[job];
-    __nv_bfloat16* out = jobs.out[job];
-    const int R = jobs.R[job], C = jobs.C;
-    const int r0 = blk * kRedRows;
-    for (int i = threadIdx.x; i < kRedRows * C; i += blockDim.x) {
-        const int rr = i / C, c = i - rr * C;
-        if (r0 + rr < R) tile[rr][c] = in[static_cast<long long>(r0 + rr) * C + c];
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kRedRows * C; i += blockDim.x) {
-        const int c = i / kRedRows, rr = i - c * kRedRows;
-        if (r0 + rr < R) out[static_cast<long long>(c) * R + r0 + rr] = tile[rr][c];
-    }
-}
 
 // Block-int4 weight element -> bf16: (fp32(q) * fp32(scale)) / 7 in IEEE fp32
 // (the product is exact; the divide is correctly rounded), then round to

@@ -45,11 +45,71 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Where an epilogue reads its fp32 accumulator row from (32 columns at a time).
+// TMEM: `tacc` = TMEM address of this warp's lane quarter at the tile's
+// accumulator buffer.  Warp-collective.
+struct TmemSrc {
+    uint32_t tacc;
+    __device__ __forceinline__ void load(int col, uint32_t (&v)[32]) const {
+        tmem_ld32(tacc + col, v);
+        tmem_ld_wait();
+    }
+    __device__ __forceinline__ void load2(int c0, uint32_t (&v0)[32], int c1, uint32_t (&v1)[32]) const {
+        tmem_ld32(tacc + c0, v0);
+        tmem_ld32(tacc + c1, v1);
+        tmem_ld_wait();
+    }
+};
+
+// The sum, in split order, of `splits` fp32 partial rows (split s at
+// base + s * split_stride): the accumulator of a tile whose K range was
+// divided between CTAs.  Per thread.
+struct PartialSrc {
+    const float* base;
+    long long split_stride;
+    int splits;
+    __device__ __forceinline__ void load(int col, uint32_t (&v)[32]) const {
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+        // Two splits' loads are in flight together (the usual case is two).
+        for (int sp0 = 0; sp0 < splits; sp0 += 2) {
+            float4 x[2][8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (sp0 + h < splits) {
+                    const float4* q = reinterpret_cast<const float4*>(base + (sp0 + h) * split_stride + col);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[h][i] = __ldcg(q + i);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (sp0 + h < splits) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[4 * i] += x[h][i].x;
+                        acc[4 * i + 1] += x[h][i].y;
+                        acc[4 * i + 2] += x[h][i].z;
+                        acc[4 * i + 3] += x[h][i].w;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(acc[i]);
+    }
+    __device__ __forceinline__ void load2(int c0, uint32_t (&v0)[32], int c1, uint32_t (&v1)[32]) const {
+        load(c0, v0);
+        load(c1, v1);
+    }
+};
+
 // One output tile row per thread: `row` (may be >= M: stores are skipped),
-// columns [col_base, col_base + bn).  `tacc` = TMEM address of this warp's
-// lane quarter at the tile's accumulator buffer (accumulator a at + a*bn).
-template <int NACC, int EPI>
-__device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, uint32_t tacc) {
+// columns [col_base, col_base + bn); accumulator a's column c is read from
+// `src` at a*bn + c.
+template <int NACC, int EPI, class Src>
+__device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src) {
     const bool row_ok = row < o.M;
     const int nchunks = bn >> 5;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -57,8 +117,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
         if (col0 >= o.N) break;  // warp-uniform
         if constexpr (EPI == EPI_BF16) {
             uint32_t v[32];
-            tmem_ld32(tacc + ch * 32, v);
-            tmem_ld_wait();
+            src.load(ch * 32, v);
             if (row_ok) {
                 __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.out0) + row * o.ld + col0;
 #pragma unroll
@@ -77,8 +136,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
 #pragma unroll
             for (int acc = 0; acc < NACC; ++acc) {
                 uint32_t v[32];
-                tmem_ld32(tacc + acc * bn + ch * 32, v);
-                tmem_ld_wait();
+                src.load(acc * bn + ch * 32, v);
                 if (row_ok) {
                     float* dst = static_cast<float*>(acc == 0 ? o.out0 : o.out1) + o.split_off + row * o.ld + col0;
 #pragma unroll
@@ -92,9 +150,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             }
         } else if constexpr (EPI == EPI_SWIGLU_FWD) {
             uint32_t vg[32], vu[32];
-            tmem_ld32(tacc + ch * 32, vg);
-            tmem_ld32(tacc + bn + ch * 32, vu);
-            tmem_ld_wait();
+            src.load2(ch * 32, vg, bn + ch * 32, vu);
             if (row_ok) {
                 const long long off = row * o.ld + col0;
                 __nv_bfloat16* gd = static_cast<__nv_bfloat16*>(o.out0) + off;
@@ -133,8 +189,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                 }
             }
             uint32_t v[32];
-            tmem_ld32(tacc + ch * 32, v);
-            tmem_ld_wait();
+            src.load(ch * 32, v);
             if (row_ok) {
                 __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(o.out0) + off;
                 __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(o.out1) + off;

@@ -43,6 +43,22 @@ constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a la
 constexpr int kMaxSplits = 32;
 constexpr size_t kAlign = 256;
 constexpr uint32_t kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
+// Compile-time tuning knobs (defaults are the measured best on B200).
+#ifndef LMLP_PAIR_GROUP_M
+#define LMLP_PAIR_GROUP_M 16  // CTA-pair raster: tiles walk down groups of this many 256-row M tiles
+#endif
+#ifndef LMLP_TAIL_SPLIT
+#define LMLP_TAIL_SPLIT 1  // split the last partial round of CTA-pair tiles in two K halves
+#endif
+// The tail split pays off for launches with a plain bf16 store epilogue (the
+// down and dX GEMMs: -55 us and -15 us per step on the Llama-3-8B shapes,
+// measured interleaved) but not for the SwiGLU epilogues (+31 us, +39 us),
+// so those launches run without it.
+#ifndef LMLP_TAIL_SPLIT_SWIGLU
+#define LMLP_TAIL_SPLIT_SWIGLU 0
+#endif
+constexpr int kTailMaxUnits = 74;        // tail-split units of one CTA-pair launch (one per cluster)
+constexpr size_t kTailPartFloats = static_cast<size_t>(kTailMaxUnits) * 2 * kBM * 256;
 
 std::atomic<int64_t> g_launches{0};
 
@@ -189,7 +205,12 @@ struct GemmBuilder {
     int b_k(const void* p, int64_t Nn, int64_t K, int64_t ld) {
         return map(p, K, Nn, ld, kBK, static_cast<uint32_t>(a.bn));
     }
-    Prob* prob(int64_t M, int64_t N, int splits) {
+    // B operand, MN-major: matrix [K, Nn] (Nn contiguous), read as B[n, k]; needs bn % 64 == 0.
+    int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) {
+        if (a.bn % 64) ok = false;
+        return map(p, Nn, K, ld, 64, kBK);
+    }
+    Prob* prob(int64_t M, int64_t N, int splits, bool a_mn = false, bool b_mn = false) {
         if (a.nprobs >= kMaxProbs) {
             ok = false;
             return &a.prob[0];
@@ -200,6 +221,8 @@ struct GemmBuilder {
         p.tiles_m = ceil_div(M, kBM);
         p.tiles_n = ceil_div(N, a.bn);
         p.splits = splits;
+        p.a_mn = a_mn ? 1 : 0;
+        p.b_mn = b_mn ? 1 : 0;
         return &p;
     }
     void seg(Prob* p, int amap, int b0, int b1, int64_t k_len) {
@@ -247,12 +270,12 @@ struct GemmBuilder {
     }
 };
 
-template <int NACC, bool A_MN, bool B_MN, int EPI>
+template <int NACC, int EPI>
 int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int* counters = nullptr) {
     b.finish(counters);
     if (!b.ok) return LORA_MLP_ERR_CUDA;
     GemmArgs& a = b.a;
-    a.b_bytes = static_cast<uint32_t>(B_MN ? (a.bn / 64) * 8192 : a.bn * 128);
+    a.b_bytes = static_cast<uint32_t>(a.bn * 128);  // K-major: bn rows x 128 B; MN-major: bn/64 chunks x 8 KB
     const uint32_t stage_bytes = kATileBytes + NACC * a.b_bytes;
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
     int stages = static_cast<int>(budget / stage_bytes);
@@ -260,7 +283,7 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + gemm_ctl_bytes();
-    auto kern = umma_gemm_kernel<NACC, A_MN, B_MN, EPI>;
+    auto kern = umma_gemm_kernel<NACC, EPI>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -285,7 +308,7 @@ struct PairBuilder {
 
     PairBuilder(int64_t M, int64_t N, int tile_n) {
         std::memset(&a, 0, sizeof(a));
-        a.group_m = 8;
+        a.group_m = LMLP_PAIR_GROUP_M;
         a.prob.M = static_cast<int>(M);
         a.prob.N = static_cast<int>(N);
         a.prob.tile_n = tile_n;
@@ -323,11 +346,29 @@ struct PairBuilder {
     }
 };
 
+// Tail split of a CTA-pair launch: with `clusters` clusters and `tiles`
+// tiles, the tiles of the last, partial round are each cut into two K
+// halves when enough clusters are free, so that round takes half a tile's
+// time.  More pieces would shorten it further but the CTA that finishes a
+// tile then has to add more partials, which costs more than it saves.
+// Returns the number of pieces (1 = no split).
+int pair_tail_splits(int tiles, int clusters, int nkb) {
+    if (clusters < 1 || tiles < 1 || nkb < 4) return 1;
+    const int tail = tiles % clusters;
+    if (tail == 0 || 2 * tail > clusters) return 1;
+    return 2;
+}
+
 template <bool B_MN, int EPI>
-int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name) {
+int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, float* tail_part, int* tail_ctr) {
     if (!b.ok) return LORA_MLP_ERR_CUDA;
     PairArgs& a = b.a;
-    a.total_units = a.prob.tiles_m * a.prob.tiles_n;
+    const int tiles = a.prob.tiles_m * a.prob.tiles_n;
+    a.total_units = tiles;
+    a.full_units = tiles;
+    a.tail_splits = 1;
+    a.tail_part = tail_part;
+    a.tail_ctr = tail_ctr;
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
     int stages = static_cast<int>(budget / kPairStageBytes);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
@@ -356,6 +397,17 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name) {
         if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = sms / 2;
         max_clusters[dev] = n;
     }
+    const int avail = std::min(max_clusters[dev], kTailMaxUnits);
+    const bool tail_ok = EPI == EPI_BF16 ? LMLP_TAIL_SPLIT != 0 : LMLP_TAIL_SPLIT_SWIGLU != 0;
+    if (tail_ok && tail_part != nullptr && tail_ctr != nullptr) {
+        const int S = pair_tail_splits(tiles, avail, a.prob.nkb);
+        if (S > 1) {
+            const int tail = tiles % avail;
+            a.full_units = tiles - tail;
+            a.tail_splits = S;
+            a.total_units = a.full_units + tail * S;
+        }
+    }
     int clusters = a.total_units < max_clusters[dev] ? a.total_units : max_clusters[dev];
     cfg.gridDim = dim3(2 * clusters, 1, 1);
     cudaError_t err;
@@ -364,17 +416,6 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name) {
         err = cudaLaunchKernelEx(&cfg, kern, a);
     }
     if (err != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    return last_launch_error();
-}
-
-// Transpose up to three adapter B matrices [R_i, C] -> [C, R_i] in one launch.
-int launch_transpose3(const TransposeJobs& jobs, cudaStream_t st) {
-    int blocks = 0;
-    for (int i = 0; i < jobs.n; ++i) blocks += ceil_div(jobs.R[i], kRedRows);
-    {
-        LaunchScope scope("transpose_B", st);
-        transpose3_bf16_kernel<<<blocks, 256, 0, st>>>(jobs);
-    }
     return last_launch_error();
 }
 
@@ -395,37 +436,68 @@ int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t
 }
 
 // ----------------------------------------------------------------------------- layout
-// Split-K factor for a skinny product with `tiles` output tiles and `nkb`
-// K blocks: minimise the estimated makespan of the persistent grid, i.e. the
-// number of unit rounds per SM times the K blocks of one unit, plus a small
-// per-unit cost.  Depends only on the shape (a fixed 148-CTA grid), so the
-// workspace size does not depend on the device.
-int splits_for(int64_t tiles, int64_t nkb) {
-    if (tiles < 1) tiles = 1;
-    int best = 1;
-    double best_cost = 1e30;
-    const int64_t smax = std::min<int64_t>(kMaxSplits, std::max<int64_t>(nkb, 1));
-    for (int64_t sp = 1; sp <= smax; ++sp) {
-        const int64_t rounds = (tiles * sp + kTargetCtas - 1) / kTargetCtas;
-        const double cost = static_cast<double>(rounds) * (static_cast<double>(nkb) / sp + 2.0);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = static_cast<int>(sp);
+// Split-K factors for the skinny problems of one launch.  All problems of a
+// launch are cut into units of about T K blocks (problem p gets
+// ceil(nkb_p / T) splits); T is chosen to minimise the estimated makespan of
+// the persistent grid, rounds(T) * (T + kUnitCost), where a round is one
+// unit per SM and kUnitCost (in K blocks) stands for a unit's epilogue and
+// split-K bookkeeping.  Depends only on the shape (a fixed 148-CTA grid), so
+// workspace sizes do not depend on the device.
+constexpr int64_t kUnitCost = 6;
+
+struct SkinnySpec {
+    int64_t M;      // output rows
+    int64_t ncols;  // partial columns (the valid N of the problem)
+    int64_t nkb;    // K blocks
+};
+
+void plan_splits(const SkinnySpec* sp, int n, int* out) {
+    int64_t max_kb = 1;
+    for (int i = 0; i < n; ++i) max_kb = std::max(max_kb, sp[i].nkb);
+    double best = 1e300;
+    int64_t best_T = max_kb;
+    for (int64_t T = 4; T <= max_kb + 4; T += (T < 64 ? 4 : 16)) {
+        int64_t units = 0, longest = 0;
+        for (int i = 0; i < n; ++i) {
+            const int64_t s = std::min<int64_t>(std::max<int64_t>((sp[i].nkb + T - 1) / T, 1), kMaxSplits);
+            units += ceil_div(sp[i].M, kBM) * s;
+            longest = std::max(longest, (sp[i].nkb + s - 1) / s);
+        }
+        const int64_t rounds = (units + kTargetCtas - 1) / kTargetCtas;
+        const double cost = static_cast<double>(rounds) * static_cast<double>(longest + kUnitCost);
+        if (cost < best - 1e-9) {
+            best = cost;
+            best_T = T;
         }
     }
-    return best;
+    for (int i = 0; i < n; ++i) {
+        const int64_t s = std::min<int64_t>(std::max<int64_t>((sp[i].nkb + best_T - 1) / best_T, 1), kMaxSplits);
+        out[i] = static_cast<int>(std::min<int64_t>(s, std::max<int64_t>(sp[i].nkb, 1)));
+    }
 }
+
+int64_t launch_tiles(const SkinnySpec* sp, int n) {
+    int64_t t = 0;
+    for (int i = 0; i < n; ++i) t += ceil_div(sp[i].M, kBM);
+    return t;
+}
+
+// The skinny launches of one forward + backward, in launch order.
+enum { SK_F0, SK_F2, SK_B0, SK_BMID, SK_B5, SK_COUNT };
+constexpr int kSkinnyProbs[SK_COUNT] = {1, 1, 2, 5, 1};
 
 struct Plan {
     int64_t N, d, d_ff, r, ldN;
     float s;
     bool int4;
-    int bn_r, bn_2r;
-    int sp_f0, sp_f2, sp_b0a, sp_b0b, sp_b2, sp_b3a, sp_b3b, sp_b5;
+    int bn_r, bn_r64, bn_2r;
+    SkinnySpec spec[SK_COUNT][kMaxProbs];
+    int splits[SK_COUNT][kMaxProbs];
+    size_t part_off[SK_COUNT][kMaxProbs];  // float offset of each problem's partials
     // forward workspace
-    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_w[3], f_total;
+    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_w[3], f_total;
     // backward workspace
-    size_t b_dg, b_du, b_h, b_bdT, b_bgT, b_buT, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_w[3], b_total;
+    size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_w[3], b_total;
     size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
     // saved
     size_t s_sgT, s_suT, s_sdT, s_total;
@@ -450,63 +522,73 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.s = static_cast<float>(static_cast<double>(sh.alpha) / static_cast<double>(sh.r));
     p.int4 = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64;
     p.bn_r = static_cast<int>(round_up(sh.r, 32));
+    p.bn_r64 = static_cast<int>(round_up(sh.r, 64));
     p.bn_2r = static_cast<int>(round_up(2 * sh.r, 32));
-    const int64_t tm_N = ceil_div(p.N, kBM);
-    p.sp_f0 = splits_for(tm_N, ceil_div(p.d, kBK));
-    p.sp_f2 = splits_for(tm_N, ceil_div(p.d_ff, kBK));
-    p.sp_b0a = splits_for(tm_N, ceil_div(p.d, kBK));
-    p.sp_b0b = splits_for(ceil_div(p.d, kBM), ceil_div(p.N, kBK));
-    p.sp_b2 = splits_for(ceil_div(p.d_ff, kBM), ceil_div(p.N, kBK));
-    p.sp_b3a = splits_for(2 * tm_N, ceil_div(p.d_ff, kBK));
-    p.sp_b3b = splits_for(2 * ceil_div(p.d_ff, kBM), ceil_div(p.N, kBK));
-    p.sp_b5 = splits_for(ceil_div(p.d, kBM), ceil_div(p.N, kBK));
+    const int64_t N = p.N, d = p.d, dff = p.d_ff, r = p.r;
+    const int64_t kb_d = ceil_div(d, kBK), kb_f = ceil_div(dff, kBK), kb_n = ceil_div(N, kBK);
+    // F0: [S_g|S_u] (two accumulators, 2r partial columns); F2: S_d
+    p.spec[SK_F0][0] = {N, 2 * r, kb_d};
+    p.spec[SK_F2][0] = {N, r, kb_f};
+    // B0: T_d (rows = tokens) and dBd (rows = d)
+    p.spec[SK_B0][0] = {N, r, kb_d};
+    p.spec[SK_B0][1] = {d, r, kb_n};
+    // B-mid: T_g, T_u (longest units first), dAd, dBg, dBu
+    p.spec[SK_BMID][0] = {N, r, kb_f};
+    p.spec[SK_BMID][1] = {N, r, kb_f};
+    p.spec[SK_BMID][2] = {dff, r, kb_n};
+    p.spec[SK_BMID][3] = {dff, r, kb_n};
+    p.spec[SK_BMID][4] = {dff, r, kb_n};
+    // B5: [dAg; dAu]^T (2r partial columns)
+    p.spec[SK_B5][0] = {d, 2 * r, kb_n};
+    size_t part_f = 0, part_b = 0;
+    int64_t max_tiles = 0;
+    for (int l = 0; l < SK_COUNT; ++l) {
+        plan_splits(p.spec[l], kSkinnyProbs[l], p.splits[l]);
+        size_t off = 0;
+        for (int i = 0; i < kSkinnyProbs[l]; ++i) {
+            p.part_off[l][i] = off;
+            off += static_cast<size_t>(p.splits[l][i]) * p.spec[l][i].M * p.spec[l][i].ncols;
+        }
+        if (l <= SK_F2) part_f = std::max(part_f, off);
+        else part_b = std::max(part_b, off);
+        max_tiles = std::max(max_tiles, launch_tiles(p.spec[l], kSkinnyProbs[l]));
+    }
+    p.ctr_bytes = static_cast<size_t>(std::max<int64_t>(max_tiles, 2 * kTailMaxUnits) + 8) * sizeof(int);
+
     const size_t bf = 2, f32 = 4;
-    const size_t N = p.N, d = p.d, dff = p.d_ff, r = p.r, ldN = p.ldN;
-    const size_t wsz[3] = {dff * d * bf, dff * d * bf, d * dff * bf};
+    const size_t Nz = N, dz = d, fz = dff, rz = r, ldN = p.ldN;
+    const size_t wsz[3] = {fz * dz * bf, fz * dz * bf, dz * fz * bf};
 
     Carver f;
-    p.f_h = f.take(N * dff * bf);
-    p.f_sgu = f.take(N * 2 * r * bf);
-    p.f_sd = f.take(N * r * bf);
-    size_t part = p.sp_f0 * N * 2 * r;
-    part = std::max(part, p.sp_f2 * N * r);
-    p.f_part = f.take(part * f32);
-    const size_t ctr_slots = 2 * static_cast<size_t>(std::max<int64_t>(
-                                     std::max<int64_t>(ceil_div(p.N, kBM), ceil_div(p.d_ff, kBM)), ceil_div(p.d, kBM))) +
-                             8;
-    p.ctr_bytes = ctr_slots * sizeof(int);
+    p.f_h = f.take(Nz * fz * bf);
+    p.f_sgu = f.take(Nz * 2 * rz * bf);
+    p.f_sd = f.take(Nz * rz * bf);
+    p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
+    p.f_tail = f.take(kTailPartFloats * f32);
     for (int i = 0; i < 3; ++i) p.f_w[i] = p.int4 ? f.take(wsz[i]) : 0;
     p.f_total = f.off;
 
     Carver b;
-    p.b_dg = b.take(N * dff * bf);
-    p.b_du = b.take(N * dff * bf);
-    p.b_h = b.take(N * dff * bf);
-    p.b_bdT = b.take(r * d * bf);
-    p.b_bgT = b.take(r * dff * bf);
-    p.b_buT = b.take(r * dff * bf);
-    p.b_td = b.take(N * r * bf);
-    p.b_tdT = b.take(r * ldN * bf);
-    p.b_tgu = b.take(N * 2 * r * bf);
-    p.b_tguT = b.take(2 * r * ldN * bf);
-    size_t bpart = p.sp_b0a * N * r;
-    bpart = std::max(bpart, p.sp_b0b * d * r);
-    bpart = std::max(bpart, p.sp_b2 * dff * r);
-    bpart = std::max(bpart, p.sp_b3a * N * 2 * r);
-    bpart = std::max(bpart, p.sp_b3b * dff * 2 * r);
-    bpart = std::max(bpart, p.sp_b5 * d * 2 * r);
-    p.b_part = b.take(bpart * f32);
+    p.b_dg = b.take(Nz * fz * bf);
+    p.b_du = b.take(Nz * fz * bf);
+    p.b_h = b.take(Nz * fz * bf);
+    p.b_td = b.take(Nz * rz * bf);
+    p.b_tdT = b.take(rz * ldN * bf);
+    p.b_tgu = b.take(Nz * 2 * rz * bf);
+    p.b_tguT = b.take(2 * rz * ldN * bf);
+    p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
+    p.b_tail = b.take(kTailPartFloats * f32);
     for (int i = 0; i < 3; ++i) p.b_w[i] = p.int4 ? b.take(wsz[i]) : 0;
     p.b_total = b.off;
 
-    Carver s;
-    p.s_sgT = s.take(r * ldN * bf);
-    p.s_suT = p.s_sgT + r * ldN * bf;  // contiguous with S_g^T: [S_g^T; S_u^T] is one [2r, ldN] matrix
-    s.take(r * ldN * bf);
-    p.s_sdT = s.take(r * ldN * bf);
-    p.s_total = s.off;
+    Carver sv;
+    p.s_sgT = sv.take(rz * ldN * bf);
+    p.s_suT = p.s_sgT + rz * ldN * bf;  // contiguous with S_g^T: [S_g^T; S_u^T] is one [2r, ldN] matrix
+    sv.take(rz * ldN * bf);
+    p.s_sdT = sv.take(rz * ldN * bf);
+    p.s_total = sv.off;
     return p;
 }
 
@@ -606,6 +688,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     __nv_bfloat16* Sd = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_sd);
     float* part = reinterpret_cast<float*>(ws + pl.f_part);
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
+    float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
     const void* W[3];
     LMLP_TRY(frozen_weights(pl, w, ws, pl.f_w, di.sms, st, W));
@@ -615,14 +698,14 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         const int ax = b.a_k(X, N, d, d);
         const int bg = b.b_k(w->Ag, r, d, d);
         const int bu = b.b_k(w->Au, r, d, d);
-        Prob* p = b.prob(N, r, pl.sp_f0);
+        Prob* p = b.prob(N, r, pl.splits[SK_F0][0]);
         b.seg(p, ax, bg, bu, d);
         p->out0 = part;
         p->out1 = part + r;
         p->ld = 2 * r;
         p->split_stride = N * 2 * r;
         b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
-        LMLP_TRY((launch_gemm<2, false, false, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
+        LMLP_TRY((launch_gemm<2, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
         PairBuilder b(N, dff, 128);
@@ -638,19 +721,19 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.out1 = u;
         b.a.prob.out2 = h;
         b.a.prob.ld = dff;
-        LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu")));
+        LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
     }
     {  // F2: S_d = s h Ad^T  -> Sd [N, r] and saved S_d^T [r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ah = b.a_k(h, N, dff, dff);
         const int bad = b.b_k(w->Ad, r, dff, dff);
-        Prob* p = b.prob(N, r, pl.sp_f2);
+        Prob* p = b.prob(N, r, pl.splits[SK_F2][0]);
         b.seg(p, ah, bad, -1, dff);
         p->out0 = part;
         p->ld = r;
         p->split_stride = N * r;
         b.fin(p, pl.s, static_cast<int>(r), Sd, r, sv + pl.s_sdT, nullptr, pl.ldN, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
     }
     {  // F3: out = h Wd^T + S_d Bd^T
         PairBuilder b(N, d, 256);
@@ -662,7 +745,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.seg(asd, bbd, bbd, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = out;
         b.a.prob.ld = d;
-        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down")));
+        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down", tailp, ctr)));
     }
     return LORA_MLP_OK;
 }
@@ -686,15 +769,13 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_dg);
     __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_du);
     __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_h);
-    __nv_bfloat16* BdT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_bdT);
-    __nv_bfloat16* BgT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_bgT);
-    __nv_bfloat16* BuT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_buT);
     __nv_bfloat16* Td = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_td);
     __nv_bfloat16* TdT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tdT);
     __nv_bfloat16* Tgu = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tgu);
     __nv_bfloat16* TguT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tguT);
     float* part = reinterpret_cast<float*>(ws + pl.b_part);
     int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
+    float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
@@ -703,44 +784,26 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     LMLP_TRY(frozen_weights(pl, w, ws, pl.b_w, di.sms, st, W));
 
     // adapter B matrices as K-major operands of the rank-r projections
-    {
-        TransposeJobs jobs{};
-        jobs.n = 3;
-        jobs.C = static_cast<int>(r);
-        const void* ins[3] = {w->Bd, w->Bg, w->Bu};
-        void* outs[3] = {BdT, BgT, BuT};
-        const int64_t rows[3] = {d, dff, dff};
-        for (int i = 0; i < 3; ++i) {
-            jobs.in[i] = static_cast<const __nv_bfloat16*>(ins[i]);
-            jobs.out[i] = static_cast<__nv_bfloat16*>(outs[i]);
-            jobs.R[i] = static_cast<int>(rows[i]);
-        }
-        LMLP_TRY(launch_transpose3(jobs, st));
-    }
-
-    {  // B0a: T_d = s dOut Bd  -> Td [N, r] and Td^T [r, ldN]
-        GemmBuilder b(pl.bn_r);
-        const int a = b.a_k(dOut, N, d, d);
-        const int bb = b.b_k(BdT, r, d, d);
-        Prob* p = b.prob(N, r, pl.sp_b0a);
-        b.seg(p, a, bb, -1, d);
-        p->out0 = part;
-        p->ld = r;
-        p->split_stride = N * r;
-        b.fin(p, pl.s, static_cast<int>(r), Td, r, TdT, nullptr, ldN, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B0_lowrank_out", ctr)));
-    }
-    {  // B0b: dBd = dOut^T S_d
-        GemmBuilder b(pl.bn_r);
-        const int a = b.a_mn(dOut, N, d, d);
-        const int bb = b.b_k(SdT, r, N, ldN);
-        Prob* p = b.prob(d, r, pl.sp_b0b);
-        b.seg(p, a, bb, -1, N);
-        p->out0 = part;
-        p->ld = r;
-        p->split_stride = d * r;
-        b.fin(p, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B0_dBd", ctr)));
+    {  // B0: T_d = s dOut Bd -> Td [N, r], Td^T [r, ldN];  dBd = dOut^T S_d
+        const int* sp = pl.splits[SK_B0];
+        GemmBuilder b(pl.bn_r64);
+        const int a0 = b.a_k(dOut, N, d, d);
+        const int b0 = b.b_mn(w->Bd, d, r, r);
+        const int a1 = b.a_mn(dOut, N, d, d);
+        const int b1 = b.b_k(SdT, r, N, ldN);
+        Prob* p0 = b.prob(N, r, sp[0], false, true);
+        b.seg(p0, a0, b0, -1, d);
+        p0->out0 = part + pl.part_off[SK_B0][0];
+        p0->ld = r;
+        p0->split_stride = N * r;
+        b.fin(p0, pl.s, static_cast<int>(r), Td, r, TdT, nullptr, ldN, static_cast<int>(r));
+        Prob* p1 = b.prob(d, r, sp[1], true, false);
+        b.seg(p1, a1, b1, -1, N);
+        p1->out0 = part + pl.part_off[SK_B0][1];
+        p1->ld = r;
+        p1->split_stride = d * r;
+        b.fin(p1, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B0_lowrank_out_dBd", ctr)));
     }
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
         PairBuilder b(N, dff, 256);
@@ -757,59 +820,54 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p.out1 = du;
         p.out2 = hb;
         p.ld = dff;
-        LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd")));
+        LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
     }
-    {  // B2: dAd = T_d^T h  (written transposed: dAd [r, d_ff])
-        GemmBuilder b(pl.bn_r);
-        const int a = b.a_mn(hb, N, dff, dff);
-        const int bb = b.b_k(TdT, r, N, ldN);
-        Prob* p = b.prob(dff, r, pl.sp_b2);
-        b.seg(p, a, bb, -1, N);
-        p->out0 = part;
-        p->ld = r;
-        p->split_stride = dff * r;
-        b.fin(p, 1.0f, static_cast<int>(r), nullptr, 0, grads->dAd, nullptr, dff, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B2_dAd", ctr)));
-    }
-    {  // B3a: T_g = s dg Bg, T_u = s du Bu  -> Tgu [N, 2r] and Tgu^T [2r, ldN]
-        GemmBuilder b(pl.bn_r);
-        const int ag = b.a_k(dg, N, dff, dff);
-        const int au = b.a_k(du, N, dff, dff);
-        const int bg = b.b_k(BgT, r, dff, dff);
-        const int bu = b.b_k(BuT, r, dff, dff);
-        Prob* p0 = b.prob(N, r, pl.sp_b3a);
-        b.seg(p0, ag, bg, -1, dff);
-        p0->out0 = part;
-        p0->ld = 2 * r;
-        p0->split_stride = N * 2 * r;
-        b.fin(p0, pl.s, static_cast<int>(r), Tgu, 2 * r, TguT, nullptr, ldN, static_cast<int>(r));
-        Prob* p1 = b.prob(N, r, pl.sp_b3a);
-        b.seg(p1, au, bu, -1, dff);
-        p1->out0 = part + r;
-        p1->ld = 2 * r;
-        p1->split_stride = N * 2 * r;
-        b.fin(p1, pl.s, static_cast<int>(r), Tgu + r, 2 * r, TguT + r * ldN, nullptr, ldN, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, false, false, EPI_F32>(b, di.sms, st, "B3_lowrank_gu", ctr)));
-    }
-    {  // B3b: dBg = dg^T S_g, dBu = du^T S_u
-        GemmBuilder b(pl.bn_r);
-        const int ag = b.a_mn(dg, N, dff, dff);
-        const int au = b.a_mn(du, N, dff, dff);
-        const int bg = b.b_k(SgT, r, N, ldN);
-        const int bu = b.b_k(SuT, r, N, ldN);
-        Prob* p0 = b.prob(dff, r, pl.sp_b3b);
-        b.seg(p0, ag, bg, -1, N);
-        p0->out0 = part;
-        p0->ld = 2 * r;
-        p0->split_stride = dff * 2 * r;
-        b.fin(p0, 1.0f, static_cast<int>(r), grads->dBg, r, nullptr, nullptr, 0, static_cast<int>(r));
-        Prob* p1 = b.prob(dff, r, pl.sp_b3b);
-        b.seg(p1, au, bu, -1, N);
-        p1->out0 = part + r;
-        p1->ld = 2 * r;
-        p1->split_stride = dff * 2 * r;
-        b.fin(p1, 1.0f, static_cast<int>(r), grads->dBu, r, nullptr, nullptr, 0, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B3_dBgu", ctr)));
+    {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
+       //        dAd = T_d^T h (written transposed);  dBg = dg^T S_g, dBu = du^T S_u
+        const int* sp = pl.splits[SK_BMID];
+        const size_t* po = pl.part_off[SK_BMID];
+        GemmBuilder b(pl.bn_r64);
+        const int adg_k = b.a_k(dg, N, dff, dff);
+        const int adu_k = b.a_k(du, N, dff, dff);
+        const int bbg = b.b_mn(w->Bg, dff, r, r);
+        const int bbu = b.b_mn(w->Bu, dff, r, r);
+        const int ah = b.a_mn(hb, N, dff, dff);
+        const int btd = b.b_k(TdT, r, N, ldN);
+        const int adg_m = b.a_mn(dg, N, dff, dff);
+        const int adu_m = b.a_mn(du, N, dff, dff);
+        const int bsg = b.b_k(SgT, r, N, ldN);
+        const int bsu = b.b_k(SuT, r, N, ldN);
+        Prob* tg = b.prob(N, r, sp[0], false, true);
+        b.seg(tg, adg_k, bbg, -1, dff);
+        tg->out0 = part + po[0];
+        tg->ld = r;
+        tg->split_stride = N * r;
+        b.fin(tg, pl.s, static_cast<int>(r), Tgu, 2 * r, TguT, nullptr, ldN, static_cast<int>(r));
+        Prob* tu = b.prob(N, r, sp[1], false, true);
+        b.seg(tu, adu_k, bbu, -1, dff);
+        tu->out0 = part + po[1];
+        tu->ld = r;
+        tu->split_stride = N * r;
+        b.fin(tu, pl.s, static_cast<int>(r), Tgu + r, 2 * r, TguT + r * ldN, nullptr, ldN, static_cast<int>(r));
+        Prob* pad = b.prob(dff, r, sp[2], true, false);
+        b.seg(pad, ah, btd, -1, N);
+        pad->out0 = part + po[2];
+        pad->ld = r;
+        pad->split_stride = dff * r;
+        b.fin(pad, 1.0f, static_cast<int>(r), nullptr, 0, grads->dAd, nullptr, dff, static_cast<int>(r));
+        Prob* pbg = b.prob(dff, r, sp[3], true, false);
+        b.seg(pbg, adg_m, bsg, -1, N);
+        pbg->out0 = part + po[3];
+        pbg->ld = r;
+        pbg->split_stride = dff * r;
+        b.fin(pbg, 1.0f, static_cast<int>(r), grads->dBg, r, nullptr, nullptr, 0, static_cast<int>(r));
+        Prob* pbu = b.prob(dff, r, sp[4], true, false);
+        b.seg(pbu, adu_m, bsu, -1, N);
+        pbu->out0 = part + po[4];
+        pbu->ld = r;
+        pbu->split_stride = dff * r;
+        b.fin(pbu, 1.0f, static_cast<int>(r), grads->dBu, r, nullptr, nullptr, 0, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B_mid_lowrank_grads", ctr)));
     }
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
         PairBuilder b(N, d, 256);
@@ -827,19 +885,19 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.seg(atu, bau, bau, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = dX;
         b.a.prob.ld = d;
-        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX")));
+        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX", tailp, ctr)));
     }
     {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]  (written transposed: dAg, dAu [r, d])
         GemmBuilder b(pl.bn_2r);
         const int a = b.a_mn(X, N, d, d);
         const int bb = b.b_k(TguT, 2 * r, N, ldN);
-        Prob* p = b.prob(d, 2 * r, pl.sp_b5);
+        Prob* p = b.prob(d, 2 * r, pl.splits[SK_B5][0], true, false);
         b.seg(p, a, bb, -1, N);
         p->out0 = part;
         p->ld = 2 * r;
         p->split_stride = d * 2 * r;
         b.fin(p, 1.0f, static_cast<int>(2 * r), nullptr, 0, grads->dAg, grads->dAu, d, static_cast<int>(r));
-        LMLP_TRY((launch_gemm<1, true, false, EPI_F32>(b, di.sms, st, "B5_dA_in", ctr)));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B5_dA_in", ctr)));
     }
     return LORA_MLP_OK;
 }

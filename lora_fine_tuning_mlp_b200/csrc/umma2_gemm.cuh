@@ -60,23 +60,57 @@ struct PairProb {
     long long ld;
 };
 
+// Tail split (stream-K for the last partial wave): the first `full_units`
+// tiles run whole; each of the remaining tiles is cut into `tail_splits`
+// K ranges run by different clusters, so the last round takes a fraction of
+// a tile's time instead of a whole one.  Each CTA of such a unit stores its
+// fp32 accumulator rows in `tail_part`; the CTA that finishes a (tile, rank)
+// last (counter in `tail_ctr`) adds the partials in split order and runs the
+// real epilogue on the sum.
 struct alignas(64) PairArgs {
     CUtensorMap maps[kMaxMaps];
     PairProb prob;
     int total_units;
+    int full_units;
+    int tail_splits;
     int stages;
     int group_m;
+    float* tail_part;  // [tail tile][split][rank][128 rows][256 columns]
+    int* tail_ctr;     // [tail tile][rank], zero before the launch
 };
 
-__device__ __forceinline__ void pair_decode(const PairArgs& a, int u, int& mb, int& nb) {
+struct PairUnit {
+    int mb, nb, kb0, kb1;
+    int tail;  // -1 for a whole tile, else the tail tile index
+    int ks;
+};
+
+__device__ __forceinline__ PairUnit pair_decode(const PairArgs& a, int u) {
     const PairProb& P = a.prob;
+    PairUnit r;
+    int tile;
+    if (u < a.full_units) {
+        tile = u;
+        r.tail = -1;
+        r.ks = 0;
+        r.kb0 = 0;
+        r.kb1 = P.nkb;
+    } else {
+        const int v = u - a.full_units;
+        r.tail = v / a.tail_splits;
+        r.ks = v - r.tail * a.tail_splits;
+        tile = a.full_units + r.tail;
+        r.kb0 = static_cast<int>((static_cast<long long>(r.ks) * P.nkb) / a.tail_splits);
+        r.kb1 = static_cast<int>((static_cast<long long>(r.ks + 1) * P.nkb) / a.tail_splits);
+    }
     const int per_group = a.group_m * P.tiles_n;
-    const int grp = u / per_group;
+    const int grp = tile / per_group;
     const int first_m = grp * a.group_m;
     const int gsz = min(a.group_m, P.tiles_m - first_m);
-    const int local = u - grp * per_group;
-    mb = first_m + local % gsz;
-    nb = local / gsz;
+    const int local = tile - grp * per_group;
+    r.mb = first_m + local % gsz;
+    r.nb = local / gsz;
+    return r;
 }
 
 template <bool B_MN>
@@ -87,10 +121,10 @@ __device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, 
     int stage = 0;
     uint32_t phase = 0;
     for (int u = cid; u < a.total_units; u += ncl) {
-        int mb, nb;
-        pair_decode(a, u, mb, nb);
+        const PairUnit t = pair_decode(a, u);
+        const int mb = t.mb, nb = t.nb;
         int seg = 0, seg_kb0 = 0;
-        for (int kb = 0; kb < P.nkb; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
             while (kb >= seg_kb0 + P.seg[seg].kblocks) {
                 seg_kb0 += P.seg[seg].kblocks;
                 ++seg;
@@ -131,12 +165,13 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     int abuf = 0;
     uint32_t aphase = 0;
     for (int u = cid; u < a.total_units; u += ncl) {
+        const PairUnit t = pair_decode(a, u);
         if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
         tc_fence_after();
         const uint32_t d = tmem_base + abuf * 256u;
         bool started = false;
         int seg = 0, seg_kb0 = 0;
-        for (int kb = 0; kb < P.nkb; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
             while (kb >= seg_kb0 + P.seg[seg].kblocks) {
                 seg_kb0 += P.seg[seg].kblocks;
                 ++seg;
@@ -191,19 +226,52 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     int abuf = 0;
     uint32_t aphase = 0;
     for (int u = cid; u < a.total_units; u += ncl) {
-        int mb, nb;
-        pair_decode(a, u, mb, nb);
+        const PairUnit t = pair_decode(a, u);
         if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
         tc_fence_after();
-        const int row = mb * kPairBM + static_cast<int>(rank) * kBM + quarter * 32 + lane;
+        const int lrow = quarter * 32 + lane;  // row within this CTA's 128
+        const int row = t.mb * kPairBM + static_cast<int>(rank) * kBM + lrow;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * 256u;
-        epilogue_tile<NACC, EPI>(o, row, nb * P.tile_n, bn, tacc);
+        float* part = nullptr;
+        if (t.tail < 0) {
+            epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, TmemSrc{tacc});
+        } else {
+            // this split's accumulator rows -> fp32 partial
+            part = a.tail_part + ((static_cast<long long>(t.tail) * a.tail_splits + t.ks) * 2 + rank) * (kBM * 256ll) +
+                   lrow * 256ll;
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t v[32];
+                tmem_ld32(tacc + ch * 32, v);
+                tmem_ld_wait();
+                uint4* dst = reinterpret_cast<uint4*>(part + ch * 32);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(c.acce + 8u * abuf, 0));
         if (++abuf == 2) {
             abuf = 0;
             aphase ^= 1u;
+        }
+        if (t.tail >= 0) {
+            __threadfence();
+            epi_bar();
+            if (threadIdx.x == 64) {
+                int* ctr = a.tail_ctr + t.tail * 2 + rank;
+                const int old = atomicAdd(ctr, 1);
+                const int last = old == a.tail_splits - 1;
+                if (last) *ctr = 0;
+                *c.fin_flag = last;
+            }
+            epi_bar();
+            if (*c.fin_flag) {
+                __threadfence();
+                const long long split_stride = 2ll * kBM * 256;
+                PartialSrc src{part - static_cast<long long>(t.ks) * split_stride, split_stride, a.tail_splits};
+                epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, src);
+            }
         }
     }
 }

@@ -36,7 +36,7 @@ constexpr int kBK = 64;
 constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxMaps = 12;
 constexpr int kMaxSegs = 4;
-constexpr int kMaxProbs = 2;
+constexpr int kMaxProbs = 5;
 constexpr int kMaxStages = 12;
 constexpr int kGemmThreads = 192;
 
@@ -50,6 +50,7 @@ struct Seg {
 struct Prob {
     int M, N;
     int tiles_m, tiles_n, splits, nkb, nsegs, unit0;
+    int a_mn, b_mn;  // operand majorness: 0 = K-major, 1 = MN-major (B MN-major needs bn % 64 == 0)
     Seg seg[kMaxSegs];
     void* out0;
     void* out1;
@@ -91,7 +92,9 @@ struct Unit {
 
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
     Unit r;
-    r.p = (a.nprobs > 1 && u >= a.prob[1].unit0) ? 1 : 0;
+    r.p = 0;
+    for (int i = 1; i < a.nprobs; ++i)
+        if (u >= a.prob[i].unit0) r.p = i;
     const Prob& P = a.prob[r.p];
     const int lu = u - P.unit0;
     const int tile = lu / P.splits;
@@ -136,73 +139,95 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 // ---------------------------------------------------------------------------
 // roles
 
-template <int NACC, bool A_MN, bool B_MN>
+// Loads are issued in bursts of up to kLoadBurst consecutive K blocks: the
+// producer first waits until that many stages are free, then issues their
+// copies back to back, so the DRAM pages of each A row are requested
+// together rather than one 128-byte piece at a time.
+constexpr int kLoadBurst = 4;
+
+template <int NACC>
 __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
                                               const SmemCtl& c) {
     int stage = 0;
     uint32_t phase = 0;
+    const int burst = a.stages >= 2 * kLoadBurst ? kLoadBurst : 1;
     for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
         const Unit t = decode_unit(a, u);
         const Prob& P = a.prob[t.p];
         int seg = 0, seg_kb0 = 0;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
-                seg_kb0 += P.seg[seg].kblocks;
-                ++seg;
-            }
-            const Seg& S = P.seg[seg];
-            const int k0 = (kb - seg_kb0) * kBK;
-            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c.abort_flag)) return;
-            uint32_t bytes = kATileBytes;
-#pragma unroll
-            for (int acc = 0; acc < NACC; ++acc)
-                if (S.b_map[acc] >= 0) bytes += a.b_bytes;
-            const uint32_t fb = c.full + 8u * stage;
-            mbar_arrive_expect_tx(fb, bytes);
-            const uint32_t sA = smem_base + stage * stage_bytes;
-            const CUtensorMap* am = &a.maps[S.a_map];
-            if (A_MN) {
-                tma_load_2d(sA, am, fb, t.mb * kBM, k0);
-                tma_load_2d(sA + 8192u, am, fb, t.mb * kBM + 64, k0);
-            } else {
-                tma_load_2d(sA, am, fb, k0, t.mb * kBM);
-            }
-#pragma unroll
-            for (int acc = 0; acc < NACC; ++acc) {
-                if (S.b_map[acc] < 0) continue;
-                const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
-                const CUtensorMap* bm = &a.maps[S.b_map[acc]];
-                if (B_MN) {
-                    for (int j = 0; j < a.bn / 64; ++j) tma_load_2d(sB + 8192u * j, bm, fb, t.nb * a.bn + 64 * j, k0);
-                } else {
-                    tma_load_2d(sB, bm, fb, k0, t.nb * a.bn);
+        for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += burst) {
+            const int cnt = min(burst, t.kb1 - kb0);
+            {
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < cnt; ++i) {
+                    if (!wait_or_abort(c.empty + 8u * st, ph ^ 1u, c.abort_flag)) return;
+                    if (++st == a.stages) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
-            if (++stage == a.stages) {
-                stage = 0;
-                phase ^= 1u;
+            for (int kb = kb0; kb < kb0 + cnt; ++kb) {
+                while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                    seg_kb0 += P.seg[seg].kblocks;
+                    ++seg;
+                }
+                const Seg& S = P.seg[seg];
+                const int k0 = (kb - seg_kb0) * kBK;
+                uint32_t bytes = kATileBytes;
+#pragma unroll
+                for (int acc = 0; acc < NACC; ++acc)
+                    if (S.b_map[acc] >= 0) bytes += a.b_bytes;
+                const uint32_t fb = c.full + 8u * stage;
+                mbar_arrive_expect_tx(fb, bytes);
+                const uint32_t sA = smem_base + stage * stage_bytes;
+                const CUtensorMap* am = &a.maps[S.a_map];
+                if (P.a_mn) {
+                    tma_load_2d(sA, am, fb, t.mb * kBM, k0);
+                    tma_load_2d(sA + 8192u, am, fb, t.mb * kBM + 64, k0);
+                } else {
+                    tma_load_2d(sA, am, fb, k0, t.mb * kBM);
+                }
+#pragma unroll
+                for (int acc = 0; acc < NACC; ++acc) {
+                    if (S.b_map[acc] < 0) continue;
+                    const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
+                    const CUtensorMap* bm = &a.maps[S.b_map[acc]];
+                    if (P.b_mn) {
+                        for (int j = 0; j < a.bn / 64; ++j)
+                            tma_load_2d(sB + 8192u * j, bm, fb, t.nb * a.bn + 64 * j, k0);
+                    } else {
+                        tma_load_2d(sB, bm, fb, k0, t.nb * a.bn);
+                    }
+                }
+                if (++stage == a.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     }
 }
 
-template <int NACC, bool A_MN, bool B_MN>
+template <int NACC>
 __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
                                          uint32_t tmem_base, const SmemCtl& c) {
     int stage = 0;
     uint32_t phase = 0;
     int abuf = 0;
     uint32_t aphase = 0;
-    const uint32_t idesc = idesc_bf16(static_cast<uint32_t>(a.bn), A_MN, B_MN);
-    // Two accumulators fed by the same segment sit side by side in TMEM and
-    // their B tiles side by side in smem, so one UMMA of N = 2*bn does both
-    // (A is read from smem once instead of twice).
-    const bool pair_ok = NACC == 2 && !B_MN && 2 * a.bn <= 256;
-    const uint32_t idesc_pair = idesc_bf16(static_cast<uint32_t>(2 * a.bn), A_MN, B_MN);
     const uint32_t acc_cols = NACC * a.bn;
     for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
         const Unit t = decode_unit(a, u);
         const Prob& P = a.prob[t.p];
+        const bool a_mn = P.a_mn != 0, b_mn = P.b_mn != 0;
+        const uint32_t idesc = idesc_bf16(static_cast<uint32_t>(a.bn), a_mn, b_mn);
+        // Two accumulators fed by the same segment sit side by side in TMEM and
+        // their B tiles side by side in smem, so one UMMA of N = 2*bn does both
+        // (A is read from smem once instead of twice).
+        const bool pair_ok = NACC == 2 && !b_mn && 2 * a.bn <= 256;
+        const uint32_t idesc_pair = idesc_bf16(static_cast<uint32_t>(2 * a.bn), a_mn, b_mn);
         if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
         tc_fence_after();
         uint32_t started = 0;
@@ -223,7 +248,7 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
                 const uint32_t sB = sA + kATileBytes;
                 const uint32_t d = tmem_base + abuf * acc_cols;
                 for (int k = 0; k < nk; ++k) {
-                    const uint64_t ad = A_MN ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
+                    const uint64_t ad = a_mn ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
                                              : sw128_desc(sA + 32u * k, 16u, 1024u);
                     const uint64_t bd = sw128_desc(sB + 32u * k, 16u, 1024u);
                     umma_bf16(d, ad, bd, idesc_pair, (started & 1u) | (k > 0 ? 1u : 0u));
@@ -242,9 +267,9 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
                 const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
                 const uint32_t d = tmem_base + abuf * acc_cols + acc * a.bn;
                 for (int k = 0; k < nk; ++k) {
-                    const uint64_t ad = A_MN ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
+                    const uint64_t ad = a_mn ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
                                              : sw128_desc(sA + 32u * k, 16u, 1024u);
-                    const uint64_t bd = B_MN ? sw128_desc(sB + 2048u * k, 8192u, 1024u)
+                    const uint64_t bd = b_mn ? sw128_desc(sB + 2048u * k, 8192u, 1024u)
                                              : sw128_desc(sB + 32u * k, 16u, 1024u);
                     umma_bf16(d, ad, bd, idesc, ((started >> acc) & 1u) | (k > 0 ? 1u : 0u));
                 }
@@ -290,11 +315,25 @@ __device__ __forceinline__ void splitk_finalize(const Prob& P, const Unit& t, in
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-        for (int sp = 0; sp < P.splits; ++sp) {
-            const float4* q = reinterpret_cast<const float4*>(src + sp * P.split_stride + j);
-            const float4 a0 = __ldcg(q), a1 = __ldcg(q + 1);
-            acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
-            acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+        // Loads of up to 8 splits are issued before their (in-order) adds, so a
+        // tile with many splits costs a few L2 round trips, not one per split.
+        for (int sp0 = 0; sp0 < P.splits; sp0 += 8) {
+            float4 v[8][2];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (sp0 + q < P.splits) {
+                    const float4* src4 = reinterpret_cast<const float4*>(src + (sp0 + q) * P.split_stride + j);
+                    v[q][0] = __ldcg(src4);
+                    v[q][1] = __ldcg(src4 + 1);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (sp0 + q < P.splits) {
+                    acc[0] += v[q][0].x; acc[1] += v[q][0].y; acc[2] += v[q][0].z; acc[3] += v[q][0].w;
+                    acc[4] += v[q][1].x; acc[5] += v[q][1].y; acc[6] += v[q][1].z; acc[7] += v[q][1].w;
+                }
+            }
         }
         uint32_t w[4];
 #pragma unroll
@@ -337,7 +376,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
         o.N = P.N;
         const int row = t.mb * kBM + quarter * 32 + lane;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * acc_cols;
-        epilogue_tile<NACC, EPI>(o, row, t.nb * a.bn, a.bn, tacc);
+        epilogue_tile<NACC, EPI>(o, row, t.nb * a.bn, a.bn, TmemSrc{tacc});
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(c.acce + 8u * abuf);
@@ -376,7 +415,7 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int nacc, int bn) {
     return cols;
 }
 
-template <int NACC, bool A_MN, bool B_MN, int EPI>
+template <int NACC, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -414,11 +453,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(ctl_ptr + (c.tmem_slot - ctl));
 
     if (warp == 0) {
-        if (lane == 0) producer_loop<NACC, A_MN, B_MN>(args, base, stage_bytes, c);
+        if (lane == 0) producer_loop<NACC>(args, base, stage_bytes, c);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            mma_loop<NACC, A_MN, B_MN>(args, base, stage_bytes, tmem_base, c);
+            mma_loop<NACC>(args, base, stage_bytes, tmem_base, c);
             // Drain: wait until every MMA issued by this thread has finished
             // before TMEM is released (matters only after an abort).
             umma_commit(c.drain);

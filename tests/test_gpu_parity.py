@@ -161,3 +161,31 @@ def test_autograd_function_matches_api():
     assert np.array_equal(X.grad.float().double().cpu().numpy(), ref["dX"])
     for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd"):
         assert np.array_equal(getattr(w, k).grad.float().double().cpu().numpy(), ref["d" + k]), k
+
+
+def test_host_batch_trainer_matches_device_path():
+    """Host batches through the overlapped-copy trainer give the same gradients
+    as the device-resident calls, batch after batch."""
+    cfg_a = synth.custom(512, 256, 512, 16, 16.0, seed_index=34)
+    inp_a = synth.make_inputs(cfg_a)
+    inp_b = synth.make_inputs(synth.custom(512, 256, 512, 16, 16.0, seed_index=35))
+    dev = torch.device("cuda:0")
+    w = api.weights_from_host(inp_a, cfg_a.alpha, dev)
+    host = [(torch.from_numpy(i["X"].view("int16")).view(torch.bfloat16).pin_memory(),
+             torch.from_numpy(i["dOut"].view("int16")).view(torch.bfloat16).pin_memory()) for i in (inp_a, inp_b)]
+    trainer = api.HostBatchTrainer(w, cfg_a.N, dev)
+    order = [0, 1, 0, 1]
+    got = []
+    for i, b in enumerate(order):
+        nxt = host[order[i + 1]] if i + 1 < len(order) else (None, None)
+        g = trainer.step(host[b][0], host[b][1], nxt[0], nxt[1])
+        torch.cuda.synchronize()
+        got.append({k: v.clone() for k, v in g.items()})
+    for i, b in enumerate(order):
+        X = host[b][0].to(dev)
+        dOut = host[b][1].to(dev)
+        _, saved = api.forward(X, w)
+        _, ref = api.backward(X, w, saved, dOut)
+        torch.cuda.synchronize()
+        for k in ref:
+            assert torch.equal(got[i][k], ref[k].cpu()), (i, k)
