@@ -36,7 +36,19 @@ struct EpiOut {
     int M, N;             // valid rows / columns
 };
 
-__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+#ifndef LMLP_FAST_SIGMOID
+#define LMLP_FAST_SIGMOID 1
+#endif
+// sigmoid(x) = 1 / (1 + e^-x) with CUDA's fast exp and fast divide
+// intrinsics (for large |x| the result saturates to 0 or 1); the forward and
+// the backward epilogues share this one definition, so both form the same h.
+__device__ __forceinline__ float sigmoid_f(float x) {
+#if LMLP_FAST_SIGMOID
+    return __fdividef(1.0f, 1.0f + __expf(-x));
+#else
+    return __frcp_rn(1.0f + __expf(-x));
+#endif
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -108,10 +120,86 @@ struct PartialSrc {
 // One output tile row per thread: `row` (may be >= M: stores are skipped),
 // columns [col_base, col_base + bn); accumulator a's column c is read from
 // `src` at a*bn + c.
+// SwiGLU backward for 8 consecutive columns: dH (fp32) with g, u (bf16 pairs).
+__device__ __forceinline__ void swiglu_bwd8(const uint32_t* dh, const uint4& gq, const uint4& uq, uint4& dgq,
+                                            uint4& duq, uint4& hq) {
+    const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+    uint32_t dgw[4], duw[4], hw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float dg2[2], du2[2], h2[2];
+#pragma unroll
+        for (int hsel = 0; hsel < 2; ++hsel) {
+            const float gx = hsel ? bf16_hi(gw[e]) : bf16_lo(gw[e]);
+            const float ux = hsel ? bf16_hi(uw[e]) : bf16_lo(uw[e]);
+            const float d = __uint_as_float(dh[2 * e + hsel]);
+            const float sg = sigmoid_f(gx);
+            const float sl = gx * sg;
+            du2[hsel] = d * sl;
+            dg2[hsel] = d * ux * sg * (1.0f + gx * (1.0f - sg));
+            h2[hsel] = sl * ux;
+        }
+        dgw[e] = pack_bf16(dg2[0], dg2[1]);
+        duw[e] = pack_bf16(du2[0], du2[1]);
+        hw[e] = pack_bf16(h2[0], h2[1]);
+    }
+    dgq = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+    duq = make_uint4(duw[0], duw[1], duw[2], duw[3]);
+    hq = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+}
+
 template <int NACC, int EPI, class Src>
 __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src) {
     const bool row_ok = row < o.M;
     const int nchunks = bn >> 5;
+    if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // g and u of the next 32 columns are loaded while this chunk computes.
+        const __nv_bfloat16* g_row = static_cast<const __nv_bfloat16*>(o.in0) + row * o.ld;
+        const __nv_bfloat16* u_row = static_cast<const __nv_bfloat16*>(o.in1) + row * o.ld;
+        uint4 gv[4], uv[4], gn[4], un[4];
+        auto load_gu = [&](int c0, uint4(&gq)[4], uint4(&uq)[4]) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (row_ok && c0 + 8 * q < o.N) {
+                    gq[q] = *reinterpret_cast<const uint4*>(g_row + c0 + 8 * q);
+                    uq[q] = *reinterpret_cast<const uint4*>(u_row + c0 + 8 * q);
+                } else {
+                    gq[q] = make_uint4(0, 0, 0, 0);
+                    uq[q] = make_uint4(0, 0, 0, 0);
+                }
+            }
+        };
+        load_gu(col_base, gv, uv);
+        for (int ch = 0; ch < nchunks; ++ch) {
+            const int col0 = col_base + ch * 32;
+            if (col0 >= o.N) break;  // warp-uniform
+            if (ch + 1 < nchunks) load_gu(col0 + 32, gn, un);
+            uint32_t v[32];
+            src.load(ch * 32, v);
+            if (row_ok) {
+                const long long off = row * o.ld + col0;
+                __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(o.out0) + off;
+                __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(o.out1) + off;
+                __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(o.out2) + off;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (col0 + 8 * q < o.N) {
+                        uint4 dgq, duq, hq;
+                        swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq, duq, hq);
+                        *reinterpret_cast<uint4*>(dgd + 8 * q) = dgq;
+                        *reinterpret_cast<uint4*>(dud + 8 * q) = duq;
+                        *reinterpret_cast<uint4*>(hd + 8 * q) = hq;
+                    }
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                gv[q] = gn[q];
+                uv[q] = un[q];
+            }
+        }
+    } else {
     for (int ch = 0; ch < nchunks; ++ch) {
         const int col0 = col_base + ch * 32;
         if (col0 >= o.N) break;  // warp-uniform
@@ -175,56 +263,8 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                     }
                 }
             }
-        } else {  // EPI_SWIGLU_BWD
-            uint4 gv[4], uv[4];
-            const long long off = row * o.ld + col0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (row_ok && col0 + 8 * q < o.N) {
-                    gv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o.in0) + off + 8 * q);
-                    uv[q] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o.in1) + off + 8 * q);
-                } else {
-                    gv[q] = make_uint4(0, 0, 0, 0);
-                    uv[q] = make_uint4(0, 0, 0, 0);
-                }
-            }
-            uint32_t v[32];
-            src.load(ch * 32, v);
-            if (row_ok) {
-                __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(o.out0) + off;
-                __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(o.out1) + off;
-                __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(o.out2) + off;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (col0 + 8 * q < o.N) {
-                        const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-                        const uint32_t uw[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
-                        uint32_t dgw[4], duw[4], hw[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float dg2[2], du2[2], h2[2];
-#pragma unroll
-                            for (int hsel = 0; hsel < 2; ++hsel) {
-                                const float gx = hsel ? bf16_hi(gw[e]) : bf16_lo(gw[e]);
-                                const float ux = hsel ? bf16_hi(uw[e]) : bf16_lo(uw[e]);
-                                const float dh = __uint_as_float(v[8 * q + 2 * e + hsel]);
-                                const float sg = sigmoid_f(gx);
-                                const float sl = gx * sg;
-                                du2[hsel] = dh * sl;
-                                dg2[hsel] = dh * ux * sg * (1.0f + gx * (1.0f - sg));
-                                h2[hsel] = sl * ux;
-                            }
-                            dgw[e] = pack_bf16(dg2[0], dg2[1]);
-                            duw[e] = pack_bf16(du2[0], du2[1]);
-                            hw[e] = pack_bf16(h2[0], h2[1]);
-                        }
-                        *reinterpret_cast<uint4*>(dgd + 8 * q) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                        *reinterpret_cast<uint4*>(dud + 8 * q) = make_uint4(duw[0], duw[1], duw[2], duw[3]);
-                        *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    }
-                }
-            }
         }
+    }
     }
 }
 
