@@ -139,6 +139,15 @@ int lora_mlp_timing_collect(lora_mlp_kernel_time* out, int max, int* count);
 /* Number of kernels this library has launched in this process (all devices). */
 int64_t lora_mlp_launch_count(void);
 
+/* Test hook for the failure path.  While enabled, every GEMM launch makes its
+ * epilogue wait on a barrier that nothing signals, and every barrier wait of
+ * the library's kernels gives up after `wait_cycles` SM cycles (default
+ * limit otherwise: 4e9 cycles, about 2 s).  The kernels then record
+ * LORA_MLP_ERR_DEVICE_TIMEOUT for lora_mlp_device_status, wind down without
+ * trapping (outputs are then garbage) and leave the CUDA context usable.
+ * enable = 0 restores normal operation.  Process-wide; not for production. */
+int lora_mlp_debug_force_timeout(int enable, int64_t wait_cycles);
+
 /* ---------------------------------------------------------------------------
  * Forward pass that allocates nothing.  (The pages have no counterpart: this
  * entry point exists for how the library is called, not for the method.)

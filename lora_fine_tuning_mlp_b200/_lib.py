@@ -39,6 +39,7 @@ SYMBOLS = (
     "lora_mlp_timing_collect",
     "lora_mlp_launch_count",
     "lora_mlp_forward_noalloc",
+    "lora_mlp_debug_force_timeout",
 )
 
 
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
                                                   ctypes.POINTER(ctypes.c_int)]
             L.lora_mlp_forward_noalloc.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
                                                    vp, vp]
+            L.lora_mlp_debug_force_timeout.argtypes = [ctypes.c_int, i64]
+            L.lora_mlp_debug_force_timeout.restype = ctypes.c_int
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
@@ -165,6 +168,10 @@ def timing_collect(max_records: int = 4096):
     n = ctypes.c_int(0)
     check(lib().lora_mlp_timing_collect(buf, max_records, ctypes.byref(n)), "lora_mlp_timing_collect")
     return [(buf[i].name.decode(), float(buf[i].ms)) for i in range(min(n.value, max_records))]
+
+
+def debug_force_timeout(enable: bool, wait_cycles: int = 0) -> None:
+    check(lib().lora_mlp_debug_force_timeout(1 if enable else 0, int(wait_cycles)), "lora_mlp_debug_force_timeout")
 
 
 def launch_count() -> int:

@@ -50,6 +50,27 @@ __device__ __forceinline__ float sigmoid_f(float x) {
 #endif
 }
 
+#ifndef LMLP_STREAMING_EPILOGUE
+#define LMLP_STREAMING_EPILOGUE 1
+#endif
+// Epilogue traffic (activations written once, g/u read once) is marked
+// evict-first so that it does not push the GEMM operands that other tiles are
+// still reading out of L2.
+__device__ __forceinline__ void st_out(void* p, const uint4& v) {
+#if LMLP_STREAMING_EPILOGUE
+    __stcs(reinterpret_cast<uint4*>(p), v);
+#else
+    *reinterpret_cast<uint4*>(p) = v;
+#endif
+}
+__device__ __forceinline__ uint4 ld_in(const void* p) {
+#if LMLP_STREAMING_EPILOGUE
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+#else
+    return *reinterpret_cast<const uint4*>(p);
+#endif
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -162,8 +183,8 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if (row_ok && c0 + 8 * q < o.N) {
-                    gq[q] = *reinterpret_cast<const uint4*>(g_row + c0 + 8 * q);
-                    uq[q] = *reinterpret_cast<const uint4*>(u_row + c0 + 8 * q);
+                    gq[q] = ld_in(g_row + c0 + 8 * q);
+                    uq[q] = ld_in(u_row + c0 + 8 * q);
                 } else {
                     gq[q] = make_uint4(0, 0, 0, 0);
                     uq[q] = make_uint4(0, 0, 0, 0);
@@ -187,9 +208,9 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                     if (col0 + 8 * q < o.N) {
                         uint4 dgq, duq, hq;
                         swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq, duq, hq);
-                        *reinterpret_cast<uint4*>(dgd + 8 * q) = dgq;
-                        *reinterpret_cast<uint4*>(dud + 8 * q) = duq;
-                        *reinterpret_cast<uint4*>(hd + 8 * q) = hq;
+                        st_out(dgd + 8 * q, dgq);
+                        st_out(dud + 8 * q, duq);
+                        st_out(hd + 8 * q, hq);
                     }
                 }
             }
@@ -216,7 +237,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                         w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
                         w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
                         w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                        *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+                        st_out(dst + 8 * q, w);
                     }
                 }
             }
@@ -257,9 +278,9 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                             const float h1 = g1 * sigmoid_f(g1) * bf16_hi(uw[e]);
                             hw[e] = pack_bf16(h0, h1);
                         }
-                        *reinterpret_cast<uint4*>(gd + 8 * q) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
-                        *reinterpret_cast<uint4*>(ud + 8 * q) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
-                        *reinterpret_cast<uint4*>(hd + 8 * q) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        st_out(gd + 8 * q, make_uint4(gw[0], gw[1], gw[2], gw[3]));
+                        st_out(ud + 8 * q, make_uint4(uw[0], uw[1], uw[2], uw[3]));
+                        st_out(hd + 8 * q, make_uint4(hw[0], hw[1], hw[2], hw[3]));
                     }
                 }
             }

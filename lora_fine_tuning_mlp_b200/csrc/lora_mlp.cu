@@ -61,6 +61,8 @@ constexpr int kTailMaxUnits = 74;        // tail-split units of one CTA-pair lau
 constexpr size_t kTailPartFloats = static_cast<size_t>(kTailMaxUnits) * 2 * kBM * 256;
 
 std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_force_timeout{0};
+std::atomic<long long> g_wait_limit{kWaitLimitCycles};
 
 // ----------------------------------------------------------------------------- device info
 struct DevInfo {
@@ -292,6 +294,8 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
             return LORA_MLP_ERR_CUDA;
         attr_set[dev] = true;
     }
+    a.wait_limit = g_wait_limit.load();
+    a.force_timeout = g_force_timeout.load();
     const int grid = b.units < sms ? b.units : sms;
     {
         LaunchScope scope(name, st);
@@ -408,6 +412,8 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
             a.total_units = a.full_units + tail * S;
         }
     }
+    a.wait_limit = g_wait_limit.load();
+    a.force_timeout = g_force_timeout.load();
     int clusters = a.total_units < max_clusters[dev] ? a.total_units : max_clusters[dev];
     cfg.gridDim = dim3(2 * clusters, 1, 1);
     cudaError_t err;
@@ -968,5 +974,12 @@ int lora_mlp_timing_collect(lora_mlp_kernel_time* out, int max, int* count) {
 }
 
 int64_t lora_mlp_launch_count(void) { return g_launches.load(); }
+
+int lora_mlp_debug_force_timeout(int enable, int64_t wait_cycles) {
+    if (enable && wait_cycles < 1) return LORA_MLP_ERR_INVALID_ARG;
+    g_wait_limit.store(enable ? static_cast<long long>(wait_cycles) : kWaitLimitCycles);
+    g_force_timeout.store(enable ? 1 : 0);
+    return LORA_MLP_OK;
+}
 
 }  // extern "C"

@@ -6,9 +6,10 @@
 
 namespace lmlp {
 
-// Every spin on an mbarrier gives up after this many SM clock cycles
-// (about 2 s at 1.9 GHz), records LORA_MLP_ERR_DEVICE_TIMEOUT in the device
-// status word and lets the CTA wind down instead of hanging the GPU.
+// Every spin on an mbarrier gives up after a limit of SM clock cycles (by
+// default this many, about 2 s at 1.9 GHz), records
+// LORA_MLP_ERR_DEVICE_TIMEOUT in the device status word and lets the CTA
+// wind down instead of hanging the GPU.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -40,17 +41,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-// Returns false if the limit expired.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) return false;
-    }
-    return true;
-}
-
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -77,6 +77,8 @@ struct alignas(64) PairArgs {
     int group_m;
     float* tail_part;  // [tail tile][split][rank][128 rows][256 columns]
     int* tail_ctr;     // [tail tile][rank], zero before the launch
+    long long wait_limit;  // SM cycles a barrier wait may spin before the kernel gives up
+    int force_timeout;     // test hook: the epilogue waits on a barrier nothing signals
 };
 
 struct PairUnit {
@@ -131,7 +133,7 @@ __device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, 
             }
             const PairSeg& S = P.seg[seg];
             const int k0 = (kb - seg_kb0) * kBK;
-            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c.abort_flag)) return;
+            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c)) return;
             const uint32_t fb_local = c.full + 8u * stage;
             if (leader) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
             const uint32_t fb = mapa_shared(fb_local, 0);
@@ -166,7 +168,7 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     uint32_t aphase = 0;
     for (int u = cid; u < a.total_units; u += ncl) {
         const PairUnit t = pair_decode(a, u);
-        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
+        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c)) return;
         tc_fence_after();
         const uint32_t d = tmem_base + abuf * 256u;
         bool started = false;
@@ -179,7 +181,7 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
             const PairSeg& S = P.seg[seg];
             const int k0 = (kb - seg_kb0) * kBK;
             const int nk = (min(kBK, S.k_len - k0) + 15) >> 4;
-            if (!wait_or_abort(c.full + 8u * stage, phase, c.abort_flag)) return;
+            if (!wait_or_abort(c.full + 8u * stage, phase, c)) return;
             tc_fence_after();
             const uint32_t sA = base + stage * kPairStageBytes;
             const uint32_t sB = sA + kATileBytes;
@@ -225,9 +227,13 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     const int bn = 256 / NACC;
     int abuf = 0;
     uint32_t aphase = 0;
+    if (a.force_timeout) {
+        wait_or_abort(c.never, 0, c);
+        return;
+    }
     for (int u = cid; u < a.total_units; u += ncl) {
         const PairUnit t = pair_decode(a, u);
-        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
+        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c)) return;
         tc_fence_after();
         const int lrow = quarter * 32 + lane;  // row within this CTA's 128
         const int row = t.mb * kPairBM + static_cast<int>(rank) * kBM + lrow;
@@ -284,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
     const uint32_t ctl = base + args.stages * kPairStageBytes;
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
-    const SmemCtl c = make_ctl(ctl, ctl_ptr);
+    const SmemCtl c = make_ctl(ctl, ctl_ptr, args.wait_limit);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -301,6 +307,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
             mbar_init(c.acce + 8u * b, 8);  // 4 epilogue warps in each CTA of the pair
         }
         mbar_init(c.drain, 1);
+        mbar_init(c.never, 1);
         *c.abort_flag = 0;
         fence_mbar_init();
     }
@@ -323,7 +330,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
             umma_commit_pair(c.drain, 1);
             const long long t0 = clock64();
             while (!mbar_try_wait(c.drain, 0)) {
-                if (clock64() - t0 > kWaitLimitCycles) break;
+                if (clock64() - t0 > c.wait_limit) break;
             }
         }
         __syncwarp();

@@ -84,6 +84,8 @@ struct alignas(64) GemmArgs {
     int stages;
     int group_m;       // raster: consecutive tiles walk down groups of this many M tiles
     uint32_t b_bytes;  // one B tile: bn rows (or bn/64 MN chunks) x 128 B
+    long long wait_limit;  // SM cycles a barrier wait may spin before the kernel gives up
+    int force_timeout;     // test hook: the epilogue waits on a barrier nothing signals
 };
 
 struct Unit {
@@ -114,20 +116,21 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
 __device__ int g_lmlp_status;  // LORA_MLP_ERR_DEVICE_TIMEOUT once any bounded wait expired
 
 struct SmemCtl {
-    uint32_t full, empty, accf, acce, drain;  // barrier array bases (shared addresses)
+    uint32_t full, empty, accf, acce, drain, never;  // barrier addresses (shared); `never` is never arrived on
     uint32_t tmem_slot;
     volatile int* abort_flag;
     volatile int* fin_flag;
+    long long wait_limit;  // SM cycles a wait may spin before giving up
 };
 
 // Bounded wait that also gives up as soon as another role of this CTA gave up.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, const SmemCtl& c) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort_flag = 1;
+        if (*c.abort_flag) return false;
+        if (clock64() - t0 > c.wait_limit) {
+            *c.abort_flag = 1;
             atomicExch(&g_lmlp_status, -7 /* LORA_MLP_ERR_DEVICE_TIMEOUT */);
             return false;
         }
@@ -161,7 +164,7 @@ __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_b
                 int st = stage;
                 uint32_t ph = phase;
                 for (int i = 0; i < cnt; ++i) {
-                    if (!wait_or_abort(c.empty + 8u * st, ph ^ 1u, c.abort_flag)) return;
+                    if (!wait_or_abort(c.empty + 8u * st, ph ^ 1u, c)) return;
                     if (++st == a.stages) {
                         st = 0;
                         ph ^= 1u;
@@ -228,7 +231,7 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
         // (A is read from smem once instead of twice).
         const bool pair_ok = NACC == 2 && !b_mn && 2 * a.bn <= 256;
         const uint32_t idesc_pair = idesc_bf16(static_cast<uint32_t>(2 * a.bn), a_mn, b_mn);
-        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c.abort_flag)) return;
+        if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c)) return;
         tc_fence_after();
         uint32_t started = 0;
         int seg = 0, seg_kb0 = 0;
@@ -241,7 +244,7 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
             const int k0 = (kb - seg_kb0) * kBK;
             const int kvalid = min(kBK, S.k_len - k0);
             const int nk = (kvalid + 15) >> 4;
-            if (!wait_or_abort(c.full + 8u * stage, phase, c.abort_flag)) return;
+            if (!wait_or_abort(c.full + 8u * stage, phase, c)) return;
             tc_fence_after();
             const uint32_t sA = smem_base + stage * stage_bytes;
             if (pair_ok && S.b_map[0] >= 0 && S.b_map[1] >= 0 && (started == 0u || started == 3u)) {
@@ -359,10 +362,14 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
     int abuf = 0;
     uint32_t aphase = 0;
     const uint32_t acc_cols = NACC * a.bn;
+    if (a.force_timeout) {
+        wait_or_abort(c.never, 0, c);
+        return;
+    }
     for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
         const Unit t = decode_unit(a, u);
         const Prob& P = a.prob[t.p];
-        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c.abort_flag)) return;
+        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c)) return;
         tc_fence_after();
         EpiOut o;
         o.out0 = P.out0;
@@ -393,17 +400,19 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
 // ---------------------------------------------------------------------------
 // kernel
 
-__host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 5) + 16u; }
+__host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 6) + 16u; }
 
 // Barrier/flag block that follows the operand stages in shared memory.
-__device__ __forceinline__ SmemCtl make_ctl(uint32_t ctl, uint8_t* ctl_ptr) {
+__device__ __forceinline__ SmemCtl make_ctl(uint32_t ctl, uint8_t* ctl_ptr, long long wait_limit) {
     SmemCtl c;
     c.full = ctl;
     c.empty = ctl + 8u * kMaxStages;
     c.accf = ctl + 8u * (2 * kMaxStages);
     c.acce = c.accf + 16u;
     c.drain = c.acce + 16u;
-    c.tmem_slot = c.drain + 8u;
+    c.never = c.drain + 8u;
+    c.tmem_slot = c.never + 8u;
+    c.wait_limit = wait_limit;
     c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
     c.fin_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 8u - ctl));
     return c;
@@ -424,7 +433,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
     const uint32_t ctl = base + args.stages * stage_bytes;
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
-    const SmemCtl c = make_ctl(ctl, ctl_ptr);
+    const SmemCtl c = make_ctl(ctl, ctl_ptr, args.wait_limit);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -440,6 +449,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
             mbar_init(c.acce + 8u * b, 4);
         }
         mbar_init(c.drain, 1);
+        mbar_init(c.never, 1);
         *c.abort_flag = 0;
         fence_mbar_init();
     }
@@ -463,7 +473,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
             umma_commit(c.drain);
             const long long t0 = clock64();
             while (!mbar_try_wait(c.drain, 0)) {
-                if (clock64() - t0 > kWaitLimitCycles) break;
+                if (clock64() - t0 > c.wait_limit) break;
             }
         }
         __syncwarp();
