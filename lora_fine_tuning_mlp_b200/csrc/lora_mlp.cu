@@ -427,15 +427,15 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
 
 int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
                    cudaStream_t st) {
-    const long long words = rows * cols / 8;
-    long long blocks = (words + 255) / 256;
+    const long long nblk = rows * cols / 64;
+    long long blocks = (nblk + 255) / 256;
     const long long cap = static_cast<long long>(sms) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     {
         LaunchScope scope("dequant_int4", st);
         dequant_int4_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
-            static_cast<const uint32_t*>(packed), static_cast<const __half*>(scales), rows, cols,
+            static_cast<const uint4*>(packed), static_cast<const __half*>(scales), rows, cols,
             static_cast<__nv_bfloat16*>(w));
     }
     return last_launch_error();
@@ -501,9 +501,9 @@ struct Plan {
     int splits[SK_COUNT][kMaxProbs];
     size_t part_off[SK_COUNT][kMaxProbs];  // float offset of each problem's partials
     // forward workspace
-    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_w[3], f_total;
+    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_w[2], f_total;  // f_w: int4 dequant buffers
     // backward workspace
-    size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_w[3], b_total;
+    size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_w[2], b_total;
     size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
     // saved
     size_t s_sgT, s_suT, s_sdT, s_total;
@@ -563,7 +563,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
 
     const size_t bf = 2, f32 = 4;
     const size_t Nz = N, dz = d, fz = dff, rz = r, ldN = p.ldN;
-    const size_t wsz[3] = {fz * dz * bf, fz * dz * bf, dz * fz * bf};
+    const size_t wsz = fz * dz * bf;  // one dequantised frozen weight (all three have d*d_ff elements)
 
     Carver f;
     p.f_h = f.take(Nz * fz * bf);
@@ -572,7 +572,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
     p.f_tail = f.take(kTailPartFloats * f32);
-    for (int i = 0; i < 3; ++i) p.f_w[i] = p.int4 ? f.take(wsz[i]) : 0;
+    for (int i = 0; i < 2; ++i) p.f_w[i] = p.int4 ? f.take(wsz) : 0;
     p.f_total = f.off;
 
     Carver b;
@@ -586,7 +586,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
-    for (int i = 0; i < 3; ++i) p.b_w[i] = p.int4 ? b.take(wsz[i]) : 0;
+    for (int i = 0; i < 2; ++i) p.b_w[i] = p.int4 ? b.take(wsz) : 0;
     p.b_total = b.off;
 
     Carver sv;
@@ -640,23 +640,22 @@ int check_weights(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
         if (rc_ != LORA_MLP_OK) return rc_; \
     } while (0)
 
-// Resolve the frozen weights to bf16 pointers (dequantising int4 into the workspace).
-int frozen_weights(const Plan& pl, const lora_mlp_weights* w, uint8_t* ws, const size_t off[3], int sms,
-                   cudaStream_t st, const void* out[3]) {
+// The bf16 frozen weight `which` (0 = Wg, 1 = Wu, 2 = Wd): the caller's
+// buffer, or for int4 weights a just-in-time dequantisation into workspace
+// buffer `slot` (two buffers serve the whole pass: gate and up together,
+// then down).
+int frozen_weight(const Plan& pl, const lora_mlp_weights* w, int which, uint8_t* ws, const size_t* off, int slot,
+                  int sms, cudaStream_t st, const void** out) {
+    const void* bf[3] = {w->Wg, w->Wu, w->Wd};
     if (!pl.int4) {
-        out[0] = w->Wg;
-        out[1] = w->Wu;
-        out[2] = w->Wd;
+        *out = bf[which];
         return LORA_MLP_OK;
     }
-    const void* q[3] = {w->Wg, w->Wu, w->Wd};
     const void* sc[3] = {w->Sg, w->Su, w->Sd};
-    const int64_t rows[3] = {pl.d_ff, pl.d_ff, pl.d};
-    const int64_t cols[3] = {pl.d, pl.d, pl.d_ff};
-    for (int i = 0; i < 3; ++i) {
-        LMLP_TRY(launch_dequant(q[i], sc[i], rows[i], cols[i], ws + off[i], sms, st));
-        out[i] = ws + off[i];
-    }
+    const int64_t rows = which == 2 ? pl.d : pl.d_ff;
+    const int64_t cols = which == 2 ? pl.d_ff : pl.d;
+    LMLP_TRY(launch_dequant(bf[which], sc[which], rows, cols, ws + off[slot], sms, st));
+    *out = ws + off[slot];
     return LORA_MLP_OK;
 }
 
@@ -696,8 +695,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    const void* W[3];
-    LMLP_TRY(frozen_weights(pl, w, ws, pl.f_w, di.sms, st, W));
+    const void* W[3] = {nullptr, nullptr, nullptr};
 
     {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
@@ -713,6 +711,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
         LMLP_TRY((launch_gemm<2, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
+    LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, st, &W[0]));
+    LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, st, &W[1]));
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
         PairBuilder b(N, dff, 128);
         const int ax = b.a_k(X, N, d, d);
@@ -741,6 +741,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(r), Sd, r, sv + pl.s_sdT, nullptr, pl.ldN, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
     }
+    LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, st, &W[2]));
     {  // F3: out = h Wd^T + S_d Bd^T
         PairBuilder b(N, d, 256);
         const int ah = b.a_k(h, N, dff, dff);
@@ -786,8 +787,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
-    const void* W[3];
-    LMLP_TRY(frozen_weights(pl, w, ws, pl.b_w, di.sms, st, W));
+    const void* W[3] = {nullptr, nullptr, nullptr};
 
     // adapter B matrices as K-major operands of the rank-r projections
     {  // B0: T_d = s dOut Bd -> Td [N, r], Td^T [r, ldN];  dBd = dOut^T S_d
@@ -811,6 +811,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.fin(p1, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B0_lowrank_out_dBd", ctr)));
     }
+    LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, st, &W[2]));
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
         PairBuilder b(N, dff, 256);
         const int a = b.a_k(dOut, N, d, d);
@@ -875,6 +876,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.fin(pbu, 1.0f, static_cast<int>(r), grads->dBu, r, nullptr, nullptr, 0, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B_mid_lowrank_grads", ctr)));
     }
+    LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 0, di.sms, st, &W[0]));
+    LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 1, di.sms, st, &W[1]));
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
         PairBuilder b(N, d, 256);
         const int adg = b.a_k(dg, N, dff, dff);

@@ -61,7 +61,8 @@ def test_int4_workspace_holds_dequantised_weights(L):
     assert e.value.code == _lib.ERR_UNSUPPORTED_SHAPE
     f1, b1, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=1))
     f0b, b0b, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=0))
-    assert f1 - f0b >= 3 * 256 * 768 * 2 and b1 - b0b >= 3 * 256 * 768 * 2
+    # two dequantised weights at a time (gate and up together, then down)
+    assert f1 - f0b >= 2 * 256 * 768 * 2 and b1 - b0b >= 2 * 256 * 768 * 2
 
 
 @pytest.mark.parametrize("kw,code", [

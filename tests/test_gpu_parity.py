@@ -128,6 +128,23 @@ def test_dequant_bits_match_oracle():
     assert np.array_equal(got_bits, oracle.dequant_int4(q, sc))
 
 
+def test_dequant_bits_every_code_for_many_scales():
+    """All 16 codes against finite scales of every kind: positive, negative,
+    +-0, subnormal, the largest fp16."""
+    rng = np.random.default_rng(36)
+    sc = list(rng.uniform(-8, 8, 200).astype(np.float16))
+    sc += [np.float16(x) for x in (0.0, -0.0, 6e-8, -6e-8, 1e-5, 65504.0, -65504.0, 1.0, 7.0, 0.1)]
+    rows = len(sc)
+    codes = np.tile(np.arange(-8, 8), (rows, 4))
+    nib = (codes & 0xF).astype(np.uint8)
+    q = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.array(sc, dtype=np.float16).reshape(rows, 1)
+    dev = torch.device("cuda:0")
+    got = api.dequant_int4(torch.from_numpy(q).to(dev), torch.from_numpy(scales).to(dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), oracle.dequant_int4(q, scales))
+
+
 def test_int4_path_matches_dequantised_bf16_path_bitwise_and_oracle():
     cfg = synth.custom(384, 256, 512, 16, 16.0, int4=True, seed_index=32)
     inp = synth.make_inputs(cfg)
