@@ -170,8 +170,59 @@ __device__ __forceinline__ void swiglu_bwd8(const uint32_t* dh, const uint4& gq,
     hq = make_uint4(hw[0], hw[1], hw[2], hw[3]);
 }
 
+// Per-warp staging area of the coalesced store: 32 rows of 64 B, padded to
+// 80 B so that both the row-per-lane writes and the row-contiguous reads
+// touch every bank evenly.
+constexpr uint32_t kStageRowBytes = 80;
+constexpr uint32_t kStageWarpBytes = 32 * kStageRowBytes;
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Writes one 32-column bf16 chunk of the warp's 32 rows (lane = row; v = this
+// row's 32 values) to global memory.  With a staging area (stg != 0) the
+// block is transposed through shared memory so that four lanes store 64
+// contiguous bytes of one row: every store fills whole 32-byte sectors.
+// Warp-collective; rows >= M and columns >= N are not stored.
+__device__ __forceinline__ void emit_chunk(__nv_bfloat16* base, long long ld, int row, int col0, int M, int N,
+                                           const uint4 (&v)[4], uint32_t stg) {
+    const int lane = threadIdx.x & 31;
+    if (stg == 0) {
+        if (row < M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (col0 + 8 * q < N) st_out(base + row * ld + col0 + 8 * q, v[q]);
+        }
+        return;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sts128(stg + lane * kStageRowBytes + q * 16, v[q]);
+    __syncwarp();
+    const int row0 = row - lane;
+    const int c = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = i * 8 + (lane >> 2);
+        const uint4 w = lds128(stg + r * kStageRowBytes + c * 16);
+        if (row0 + r < M && col0 + 8 * c < N) st_out(base + (row0 + r) * ld + col0 + 8 * c, w);
+    }
+}
+
+// One output tile row per thread: `row` (may be >= M: stores are skipped),
+// columns [col_base, col_base + bn); accumulator a's column c is read from
+// `src` at a*bn + c.  `stg`: this warp's staging area (0 = store directly).
 template <int NACC, int EPI, class Src>
-__device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src) {
+__device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src,
+                                              uint32_t stg = 0) {
     const bool row_ok = row < o.M;
     const int nchunks = bn >> 5;
     if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -198,22 +249,12 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             if (ch + 1 < nchunks) load_gu(col0 + 32, gn, un);
             uint32_t v[32];
             src.load(ch * 32, v);
-            if (row_ok) {
-                const long long off = row * o.ld + col0;
-                __nv_bfloat16* dgd = static_cast<__nv_bfloat16*>(o.out0) + off;
-                __nv_bfloat16* dud = static_cast<__nv_bfloat16*>(o.out1) + off;
-                __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(o.out2) + off;
+            uint4 dgq[4], duq[4], hq[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (col0 + 8 * q < o.N) {
-                        uint4 dgq, duq, hq;
-                        swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq, duq, hq);
-                        st_out(dgd + 8 * q, dgq);
-                        st_out(dud + 8 * q, duq);
-                        st_out(hd + 8 * q, hq);
-                    }
-                }
-            }
+            for (int q = 0; q < 4; ++q) swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq[q], duq[q], hq[q]);
+            emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, dgq, stg);
+            emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, duq, stg);
+            emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 gv[q] = gn[q];
@@ -221,71 +262,62 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             }
         }
     } else {
-    for (int ch = 0; ch < nchunks; ++ch) {
-        const int col0 = col_base + ch * 32;
-        if (col0 >= o.N) break;  // warp-uniform
-        if constexpr (EPI == EPI_BF16) {
-            uint32_t v[32];
-            src.load(ch * 32, v);
-            if (row_ok) {
-                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.out0) + row * o.ld + col0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (col0 + 8 * q < o.N) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                        w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                        w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                        w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                        st_out(dst + 8 * q, w);
-                    }
-                }
-            }
-        } else if constexpr (EPI == EPI_F32) {
-#pragma unroll
-            for (int acc = 0; acc < NACC; ++acc) {
+        for (int ch = 0; ch < nchunks; ++ch) {
+            const int col0 = col_base + ch * 32;
+            if (col0 >= o.N) break;  // warp-uniform
+            if constexpr (EPI == EPI_BF16) {
                 uint32_t v[32];
-                src.load(acc * bn + ch * 32, v);
-                if (row_ok) {
-                    float* dst = static_cast<float*>(acc == 0 ? o.out0 : o.out1) + o.split_off + row * o.ld + col0;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (col0 + 4 * q < o.N) {
-                            *reinterpret_cast<uint4*>(dst + 4 * q) =
-                                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                        }
-                    }
-                }
-            }
-        } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-            uint32_t vg[32], vu[32];
-            src.load2(ch * 32, vg, bn + ch * 32, vu);
-            if (row_ok) {
-                const long long off = row * o.ld + col0;
-                __nv_bfloat16* gd = static_cast<__nv_bfloat16*>(o.out0) + off;
-                __nv_bfloat16* ud = static_cast<__nv_bfloat16*>(o.out1) + off;
-                __nv_bfloat16* hd = static_cast<__nv_bfloat16*>(o.out2) + off;
+                src.load(ch * 32, v);
+                uint4 w[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    if (col0 + 8 * q < o.N) {
-                        uint32_t gw[4], uw[4], hw[4];
+                    w[q].x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                    w[q].y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                    w[q].z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                    w[q].w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                }
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, w, stg);
+            } else if constexpr (EPI == EPI_F32) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            gw[e] = pack_bf16(__uint_as_float(vg[8 * q + 2 * e]), __uint_as_float(vg[8 * q + 2 * e + 1]));
-                            uw[e] = pack_bf16(__uint_as_float(vu[8 * q + 2 * e]), __uint_as_float(vu[8 * q + 2 * e + 1]));
-                            const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
-                            const float h0 = g0 * sigmoid_f(g0) * bf16_lo(uw[e]);
-                            const float h1 = g1 * sigmoid_f(g1) * bf16_hi(uw[e]);
-                            hw[e] = pack_bf16(h0, h1);
+                for (int acc = 0; acc < NACC; ++acc) {
+                    uint32_t v[32];
+                    src.load(acc * bn + ch * 32, v);
+                    if (row_ok) {
+                        float* dst = static_cast<float*>(acc == 0 ? o.out0 : o.out1) + o.split_off + row * o.ld + col0;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (col0 + 4 * q < o.N) {
+                                *reinterpret_cast<uint4*>(dst + 4 * q) =
+                                    make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                            }
                         }
-                        st_out(gd + 8 * q, make_uint4(gw[0], gw[1], gw[2], gw[3]));
-                        st_out(ud + 8 * q, make_uint4(uw[0], uw[1], uw[2], uw[3]));
-                        st_out(hd + 8 * q, make_uint4(hw[0], hw[1], hw[2], hw[3]));
                     }
                 }
+            } else {  // EPI_SWIGLU_FWD
+                uint32_t vg[32], vu[32];
+                src.load2(ch * 32, vg, bn + ch * 32, vu);
+                uint4 gq[4], uq[4], hq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t gw[4], uw[4], hw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        gw[e] = pack_bf16(__uint_as_float(vg[8 * q + 2 * e]), __uint_as_float(vg[8 * q + 2 * e + 1]));
+                        uw[e] = pack_bf16(__uint_as_float(vu[8 * q + 2 * e]), __uint_as_float(vu[8 * q + 2 * e + 1]));
+                        const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
+                        const float h0 = g0 * sigmoid_f(g0) * bf16_lo(uw[e]);
+                        const float h1 = g1 * sigmoid_f(g1) * bf16_hi(uw[e]);
+                        hw[e] = pack_bf16(h0, h1);
+                    }
+                    gq[q] = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+                    uq[q] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+                    hq[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                }
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, gq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, uq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
             }
         }
-    }
     }
 }
 

@@ -373,11 +373,12 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_splits = 1;
     a.tail_part = tail_part;
     a.tail_ctr = tail_ctr;
-    const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
+    const uint32_t staging = 128 + 4 * kStageWarpBytes;  // epilogue store staging (4 warps)
+    const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kPairStageBytes);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
     a.stages = stages;
-    const size_t smem = 1024 + static_cast<size_t>(stages) * kPairStageBytes + gemm_ctl_bytes();
+    const size_t smem = 1024 + static_cast<size_t>(stages) * kPairStageBytes + gemm_ctl_bytes() + staging;
     auto kern = umma2_gemm_kernel<B_MN, EPI>;
     static int max_clusters[kMaxDevices] = {};
     int dev = 0;

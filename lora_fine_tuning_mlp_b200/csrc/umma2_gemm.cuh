@@ -35,7 +35,10 @@ constexpr int kPairBM = 256;
 constexpr int kPairHalfN = 128;
 constexpr uint32_t kPairBBytes = kPairHalfN * kBK * 2;                  // 16 KB per CTA
 constexpr uint32_t kPairStageBytes = kATileBytes + kPairBBytes;         // 32 KB per CTA
-constexpr int kPairMaxStages = 8;
+#ifndef LMLP_PAIR_STAGES
+#define LMLP_PAIR_STAGES 6  // 6 x 32 KB: as fast as 7 (measured), leaves room for the store staging
+#endif
+constexpr int kPairMaxStages = LMLP_PAIR_STAGES;
 constexpr uint32_t kPairTmemCols = 512;                                 // 2 buffers x 256 columns
 
 struct PairSeg {
@@ -225,6 +228,13 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     o.M = P.M;
     o.N = P.N;
     const int bn = 256 / NACC;
+    // This warp's staging area for coalesced stores, after the barrier block.
+    // Used by the SwiGLU epilogues (three outputs per chunk); the single bf16
+    // output stores directly (measured interleaved: staging helps the former
+    // by 1-2% and costs the latter about as much).
+    const uint32_t stg = EPI == EPI_BF16 ? 0u
+                                         : ((c.full + gemm_ctl_bytes() + 127u) & ~127u) +
+                                               static_cast<uint32_t>(warp - 2) * kStageWarpBytes;
     int abuf = 0;
     uint32_t aphase = 0;
     if (a.force_timeout) {
@@ -240,7 +250,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * 256u;
         float* part = nullptr;
         if (t.tail < 0) {
-            epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, TmemSrc{tacc});
+            epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, TmemSrc{tacc}, stg);
         } else {
             // this split's accumulator rows -> fp32 partial
             part = a.tail_part + ((static_cast<long long>(t.tail) * a.tail_splits + t.ks) * 2 + rank) * (kBM * 256ll) +
@@ -276,7 +286,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
                 __threadfence();
                 const long long split_stride = 2ll * kBM * 256;
                 PartialSrc src{part - static_cast<long long>(t.ks) * split_stride, split_stride, a.tail_splits};
-                epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, src);
+                epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, src, stg);
             }
         }
     }
