@@ -288,10 +288,11 @@ def b200_arm(args, cfg):
         step()
     torch.cuda.synchronize()
 
-    # ---- device-timed region: K steps, inputs resident in HBM
+    # ---- device-timed region: K steps, inputs resident in HBM.  No per-kernel
+    # events here: an event between two launches would stop the next kernel
+    # from starting under the previous one's tail (programmatic dependent
+    # launch), so `value` is taken without them.
     sampler = ClockSampler(dev.index)
-    _lib.timing_enable(True)
-    _lib.timing_collect()
     launches0 = _lib.launch_count()
     barrier()
     torch.cuda.synchronize()
@@ -306,9 +307,21 @@ def b200_arm(args, cfg):
     barrier()
     clocks = sampler.stop()
     launches = _lib.launch_count() - launches0
+    ms_max = replicas.max_over_ranks(t0.elapsed_time(t1), device=dev)
+
+    # ---- second timed region of the same work with the library's CUDA events
+    # around every launch (on the stream each kernel runs on): the per-kernel
+    # durations behind the roofline figures.
+    _lib.timing_enable(True)
+    _lib.timing_collect()
+    barrier()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    barrier()
     recs = _lib.timing_collect()
     _lib.timing_enable(False)
-    ms_max = replicas.max_over_ranks(t0.elapsed_time(t1), device=dev)
 
     # ---- end-to-end through the public API with host buffers: every step copies
     # its X and dOut from pinned host memory (overlapped with the previous
@@ -375,6 +388,7 @@ def b200_arm(args, cfg):
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
             "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(per.items(), key=lambda kv: -kv[1][0])},
+            "kernels_note": "per-launch CUDA events, second timed region of the same length (events stop launch overlap)",
         }
         if world == 1 and not args.no_cpu_baseline:
             tps, n, dt = time_oracle(cfg, args.cpu_budget)

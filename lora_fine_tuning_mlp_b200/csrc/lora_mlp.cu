@@ -297,10 +297,22 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     a.wait_limit = g_wait_limit.load();
     a.force_timeout = g_force_timeout.load();
     const int grid = b.units < sms ? b.units : sms;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = LMLP_PDL ? 1 : 0;
+    cudaError_t err;
     {
         LaunchScope scope(name, st);
-        kern<<<grid, kGemmThreads, smem, st>>>(a);
+        err = cudaLaunchKernelEx(&cfg, kern, a);
     }
+    if (err != cudaSuccess) return LORA_MLP_ERR_CUDA;
     return last_launch_error();
 }
 
@@ -384,11 +396,13 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -417,6 +431,7 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.force_timeout = g_force_timeout.load();
     int clusters = a.total_units < max_clusters[dev] ? a.total_units : max_clusters[dev];
     cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.numAttrs = LMLP_PDL ? 2 : 1;
     cudaError_t err;
     {
         LaunchScope scope(name, st);

@@ -330,6 +330,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(ctl_ptr + (c.tmem_slot - ctl));
+#if LMLP_PDL
+    // Everything above touched only this CTA's own resources; from here on
+    // the kernel reads what the previous launch wrote.
+    grid_dependency_wait();
+    grid_launch_dependents();
+#endif
 
     if (warp == 0) {
         if (lane == 0) pair_producer<B_MN>(args, base, rank, leader, c);

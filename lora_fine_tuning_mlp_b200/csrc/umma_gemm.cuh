@@ -26,6 +26,10 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#ifndef LMLP_PDL
+#define LMLP_PDL 1  // launch the GEMM kernels with programmatic stream serialisation
+#endif
+
 #include "epilogue.cuh"
 #include "ptx.cuh"
 
@@ -461,6 +465,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(ctl_ptr + (c.tmem_slot - ctl));
+#if LMLP_PDL
+    // Everything above touched only this CTA's own resources; from here on
+    // the kernel reads what the previous launch wrote.
+    grid_dependency_wait();
+    grid_launch_dependents();
+#endif
 
     if (warp == 0) {
         if (lane == 0) producer_loop<NACC>(args, base, stage_bytes, c);
