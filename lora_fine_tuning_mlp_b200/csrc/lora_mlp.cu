@@ -465,7 +465,10 @@ int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t
 // unit per SM and kUnitCost (in K blocks) stands for a unit's epilogue and
 // split-K bookkeeping.  Depends only on the shape (a fixed 148-CTA grid), so
 // workspace sizes do not depend on the device.
-constexpr int64_t kUnitCost = 6;
+#ifndef LMLP_UNIT_COST
+#define LMLP_UNIT_COST 6
+#endif
+constexpr int64_t kUnitCost = LMLP_UNIT_COST;
 
 struct SkinnySpec {
     int64_t M;      // output rows

@@ -150,7 +150,10 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
 // producer first waits until that many stages are free, then issues their
 // copies back to back, so the DRAM pages of each A row are requested
 // together rather than one 128-byte piece at a time.
-constexpr int kLoadBurst = 4;
+#ifndef LMLP_LOAD_BURST
+#define LMLP_LOAD_BURST 4
+#endif
+constexpr int kLoadBurst = LMLP_LOAD_BURST;
 
 template <int NACC>
 __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
