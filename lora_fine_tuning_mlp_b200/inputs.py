@@ -159,3 +159,57 @@ def zero_B(inputs: dict) -> dict:
     for k in ("Bg", "Bu", "Bd"):
         o[k] = np.zeros_like(inputs[k])
     return o
+
+
+# ----------------------------------------------------------------------------- LoRA linear
+
+
+@dataclasses.dataclass(frozen=True)
+class LinearConfig:
+    """One LoRA-adapted projection: X [N, in] -> Y [N, out]."""
+    name: str
+    N: int
+    d_in: int
+    d_out: int
+    r: int
+    alpha: float
+    int4: bool = False
+    index: int = 50
+
+    @property
+    def seed(self) -> int:
+        return 1234 + self.index
+
+    def flops(self) -> float:
+        """fwd + bwd: 2 dense products for fwd+dX, rank-r paths, no dW."""
+        return 4.0 * self.N * self.d_in * self.d_out + 8.0 * self.N * self.r * (self.d_in + self.d_out)
+
+
+LINEAR_CONFIGS = (
+    LinearConfig("linear_tiny", 300, 192, 320, 8, 16.0, index=50),
+    LinearConfig("llama3_8b_qproj", 4096, 4096, 4096, 16, 16.0, index=51),
+    LinearConfig("llama3_8b_kproj", 4096, 4096, 1024, 16, 16.0, index=52),
+)
+LINEAR_BY_NAME = {c.name: c for c in LINEAR_CONFIGS}
+
+
+def make_linear_inputs(cfg: LinearConfig) -> dict:
+    """X ~ N(0,1), W ~ N(0, 1/in), A ~ U(+-1/sqrt(in)), B ~ N(0, 0.02^2),
+    dY ~ N(0,1); drawn in this order in fp32 and rounded to bf16 (int4 W:
+    the block quantiser above)."""
+    rng = np.random.Generator(np.random.PCG64(cfg.seed))
+    N, di, do, r = cfg.N, cfg.d_in, cfg.d_out, cfg.r
+    f32 = {
+        "X": rng.standard_normal((N, di), dtype=np.float32),
+        "W": rng.standard_normal((do, di), dtype=np.float32) * np.float32(1.0 / np.sqrt(di)),
+        "A": rng.uniform(-1.0 / np.sqrt(di), 1.0 / np.sqrt(di), size=(r, di)).astype(np.float32),
+        "B": rng.standard_normal((do, r), dtype=np.float32) * np.float32(0.02),
+        "dY": rng.standard_normal((N, do), dtype=np.float32),
+    }
+    out = {}
+    for k, v in f32.items():
+        if cfg.int4 and k == "W":
+            out["W_q"], out["W_scale"] = quantize_int4(v)
+        else:
+            out[k] = f32_to_bf16_bits(v)
+    return out

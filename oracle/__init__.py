@@ -15,3 +15,4 @@ from .lora_mlp import (  # noqa: F401
     up_gate_feature_grads,
     weights_f64,
 )
+from . import lora_linear  # noqa: F401,E402
