@@ -2,6 +2,10 @@
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload NAME]
 
+The default workload is the MLP on the Llama-3-8B shapes.  --workload
+llama3_8b_qproj / llama3_8b_kproj instead times the single LoRA linear
+projection (forward + backward) with the same JSON contract.
+
 One step = forward + backward of the whole hot path over one batch of
 synthetic tokens (all kernels: rank-r projections, gate/up GEMM with SwiGLU
 epilogue, down GEMM, dH GEMM with SwiGLU-backward epilogue, dX GEMM, the
@@ -36,6 +40,7 @@ import numpy as np  # noqa: E402
 from lora_fine_tuning_mlp_b200 import inputs as synth  # noqa: E402
 
 METRIC = "fused LoRA-SwiGLU MLP fwd+bwd tokens/s and TFLOP/s vs bf16 dense peak"
+LINEAR_METRIC = "fused LoRA linear fwd+bwd tokens/s and TFLOP/s vs bf16 dense peak"
 DEFAULT_WORKLOAD = "llama3_8b_mlp"
 
 
@@ -60,8 +65,9 @@ def csrc_sha256() -> str:
             h.update(f.encode())
             with open(os.path.join(d, f), "rb") as fh:
                 h.update(fh.read())
-    with open(os.path.join(ROOT, "include", "lora_mlp.h"), "rb") as fh:
-        h.update(fh.read())
+    for hdr in ("lora_mlp.h", "lora_linear.h"):
+        with open(os.path.join(ROOT, "include", hdr), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()
 
 
@@ -401,18 +407,228 @@ def b200_arm(args, cfg):
     return 0
 
 
+# ----------------------------------------------------------------------------- LoRA linear legs
+
+
+def linear_flops(cfg) -> dict:
+    N, di, do, r = cfg.N, cfg.d_in, cfg.d_out, cfg.r
+    return {
+        "L0_lowrank_in": 2.0 * N * di * r,
+        "L1_linear_fwd": 2.0 * N * do * (di + r),
+        "L2_lowrank_out_dB": 2.0 * 2 * N * do * r,
+        "L3_linear_dX": 2.0 * N * di * (do + r),
+        "L4_dA": 2.0 * N * di * r,
+    }
+
+
+def linear_config_dict(cfg):
+    return {"workload": cfg.name, "N_tokens": cfg.N, "d_in": cfg.d_in, "d_out": cfg.d_out, "r": cfg.r,
+            "alpha": cfg.alpha, "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
+            "l2": "flushed: a 256 MB buffer is written between timed steps",
+            "parallelism": "replicas"}
+
+
+def time_linear_oracle(cfg, budget_s: float, inp):
+    from oracle import lora_linear as olin
+
+    p_full = olin.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dY")})
+
+    def run(idx):
+        p = dict(p_full)
+        p["X"] = olin.bf16_to_f64(inp["X"][idx])
+        dY = olin.bf16_to_f64(inp["dY"][idx])
+        t0 = time.perf_counter()
+        olin.backward(p, cfg.alpha, dY, olin.forward(p, cfg.alpha))
+        return time.perf_counter() - t0
+
+    rows = inp["X"].shape[0]
+    t_probe = run(np.arange(64))
+    n = max(64, min(rows, int(64 * budget_s / max(t_probe, 1e-3)) // 64 * 64))
+    return n, run
+
+
+def linear_reference_arm(args, cfg):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    inp = synth.make_linear_inputs(cfg)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    n, run = time_linear_oracle(cfg, per_step, inp)
+    times = []
+    for i in range(args.warmup + args.steps):
+        idx = (np.arange(n) + i * n) % cfg.N
+        dt = run(idx)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total
+    line = {
+        "impl": "reference", "metric": LINEAR_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": linear_config_dict(cfg),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
+                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def linear_arm(args, cfg):
+    """One step = LoRA linear forward + backward over N tokens.  The frozen
+    projection (32 MB for q) fits in L2, so a 256 MB buffer is written
+    between timed steps; the flush runs outside the per-step launches but
+    inside the timed region, and its own time is measured and subtracted."""
+    import torch
+    import torch.distributed as dist
+
+    from lora_fine_tuning_mlp_b200 import _lib, api, replicas
+
+    rank, local, world = replicas.world()
+    if world > 1:
+        torch.cuda.set_device(local)
+        replicas.init("nccl", device=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _lib.lib()
+    inp = synth.make_linear_inputs(cfg)
+    w = api.linear_weights_from_host(inp, cfg.alpha, dev)
+    X = api.to_device_bf16(inp["X"], dev)
+    dY = api.to_device_bf16(inp["dY"], dev)
+    N = cfg.N
+    Y = torch.empty((N, cfg.d_out), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((N, cfg.d_in), dtype=torch.bfloat16, device=dev)
+    dA, dB = torch.empty_like(w.A), torch.empty_like(w.B)
+    wsf, wsb = api.Workspace(), api.Workspace()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    barrier = replicas.barrier
+
+    def step(x=X, g=dY):
+        _, saved = api.linear_forward(x, w, Y=Y, workspace=wsf)
+        api.linear_backward(x, w, saved, g, dX=dX, dA=dA, dB=dB, workspace=wsb)
+
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return replicas.max_over_ranks(a.elapsed_time(b), device=dev)
+
+    def flushed_step():
+        flush.fill_(1)
+        step()
+
+    for _ in range(args.warmup):
+        flushed_step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = _lib.launch_count()
+    ms_total = timed(flushed_step, args.steps)
+    launches = _lib.launch_count() - launches0
+    clocks = sampler.stop()
+    ms_flush = timed(lambda: flush.fill_(1), args.steps)
+    ms_max = max(ms_total - ms_flush, 1e-6)
+
+    _lib.timing_enable(True)
+    _lib.timing_collect()
+    timed(flushed_step, args.steps)
+    recs = _lib.timing_collect()
+    _lib.timing_enable(False)
+
+    # end to end: pinned-host X and dY copied in, dA and dB copied out, every step
+    Xh = torch.from_numpy(inp["X"].view("int16")).view(torch.bfloat16).pin_memory()
+    dYh = torch.from_numpy(inp["dY"].view("int16")).view(torch.bfloat16).pin_memory()
+    dAh = torch.empty(dA.shape, dtype=dA.dtype, pin_memory=True)
+    dBh = torch.empty(dB.shape, dtype=dB.dtype, pin_memory=True)
+    Xd, dYd = torch.empty_like(X), torch.empty_like(dY)
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        dYd.copy_(dYh, non_blocking=True)
+        step(Xd, dYd)
+        dAh.copy_(dA, non_blocking=True)
+        dBh.copy_(dB, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    ems = timed(e2e_step, args.steps)
+    h2d = (X.numel() + dY.numel()) * 2
+    d2h = (dA.numel() + dB.numel()) * 2
+
+    per = {}
+    for name, kms in recs:
+        s_ = per.setdefault(name, [0.0, 0])
+        s_[0] += kms
+        s_[1] += 1
+    peaks = load_peaks()
+    fl = linear_flops(cfg)
+    dom = max(per.items(), key=lambda kv: kv[1][0])[0] if per else None
+    roof = None
+    if dom in fl:
+        avg_ms = per[dom][0] / per[dom][1]
+        achieved = fl[dom] / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": ncu_traffic(cfg.name, dom),
+                "peak_source": f"{peaks['source']} bf16_tflops (burst: short steps between L2 flushes)",
+                "flops_per_launch": fl[dom], "avg_launch_ms": avg_ms}
+    barrier()
+    if rank == 0:
+        tflops = world * cfg.flops() * args.steps / (ms_max * 1e-3) / 1e12
+        line = {
+            "metric": LINEAR_METRIC, "value": replicas.job_throughput(N, args.steps, ms_max, world),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": linear_config_dict(cfg), "tflops": tflops,
+            "frac_of_peak": {"measured_burst": tflops / world / peaks["bf16_tflops"]},
+            "roofline": roof,
+            "e2e": {"value": replicas.job_throughput(N, args.steps, ems, world), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "per step: H2D of X and dY from pinned host, forward+backward, D2H of dA and dB "
+                            "(no L2 flush)"},
+            "gpu_launches": launches,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(per.items(), key=lambda kv: -kv[1][0])},
+            "flush_ms_per_step": ms_flush / args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n, run = time_linear_oracle(cfg, args.cpu_budget, inp)
+            dt = run(np.arange(n))
+            line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
+                                    "sample": f"{n} tokens of the {cfg.name} shapes, numpy fp64 oracle, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=("b200", "reference"))
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.BY_NAME) + sorted(synth.LINEAR_BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload in synth.LINEAR_BY_NAME:
+        cfg = synth.LINEAR_BY_NAME[args.workload]
+        return linear_reference_arm(args, cfg) if args.impl == "reference" else linear_arm(args, cfg)
     cfg = synth.BY_NAME[args.workload]
     if args.impl == "reference":
         return reference_arm(args, cfg)

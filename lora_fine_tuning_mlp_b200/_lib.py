@@ -1,4 +1,4 @@
-"""ctypes binding of liblora_mlp.so (include/lora_mlp.h).
+"""ctypes binding of liblora_mlp.so (include/lora_mlp.h, include/lora_linear.h).
 
 Argument marshalling only: every step of the MLP runs in the library's CUDA
 kernels.  Loading fails loudly if the shared library has not been built.
@@ -27,7 +27,7 @@ WEIGHTS_INT4_B64 = 1
 WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Sg", "Su", "Sd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 
-# Every symbol include/lora_mlp.h declares.
+# Every symbol include/lora_mlp.h and include/lora_linear.h declare.
 SYMBOLS = (
     "lora_mlp_sizes",
     "lora_mlp_forward",
@@ -40,6 +40,9 @@ SYMBOLS = (
     "lora_mlp_launch_count",
     "lora_mlp_forward_noalloc",
     "lora_mlp_debug_force_timeout",
+    "lora_linear_sizes",
+    "lora_linear_forward",
+    "lora_linear_backward",
 )
 
 
@@ -54,6 +57,15 @@ class Weights(ctypes.Structure):
 
 class Grads(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in GRAD_FIELDS]
+
+
+class LinShape(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64),
+                ("r", ctypes.c_int64), ("alpha", ctypes.c_float), ("weight_format", ctypes.c_int32)]
+
+
+class LinWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W", "S", "A", "B")]
 
 
 class KernelTime(ctypes.Structure):
@@ -98,11 +110,18 @@ def lib() -> ctypes.CDLL:
                                                    vp, vp]
             L.lora_mlp_debug_force_timeout.argtypes = [ctypes.c_int, i64]
             L.lora_mlp_debug_force_timeout.restype = ctypes.c_int
+            L.lora_linear_sizes.argtypes = [ctypes.POINTER(LinShape), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                            ctypes.POINTER(sz)]
+            L.lora_linear_forward.argtypes = [ctypes.POINTER(LinShape), ctypes.POINTER(LinWeights), vp, vp, vp,
+                                              vp, sz, vp]
+            L.lora_linear_backward.argtypes = [ctypes.POINTER(LinShape), ctypes.POINTER(LinWeights), vp, vp, vp,
+                                               vp, vp, vp, vp, sz, vp]
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
                          "lora_mlp_dequant_int4",
-                         "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect"):
+                         "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect",
+                         "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -176,3 +195,25 @@ def debug_force_timeout(enable: bool, wait_cycles: int = 0) -> None:
 
 def launch_count() -> int:
     return int(lib().lora_mlp_launch_count())
+
+
+def make_lin_shape(N, d_in, d_out, r, alpha, weight_format=WEIGHTS_BF16) -> LinShape:
+    return LinShape(int(N), int(d_in), int(d_out), int(r), float(alpha), int(weight_format))
+
+
+def lin_sizes(shape: LinShape):
+    f, b, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().lora_linear_sizes(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b), ctypes.byref(s)),
+          "lora_linear_sizes")
+    return f.value, b.value, s.value
+
+
+def lin_forward(shape: LinShape, weights: LinWeights, X, Y, saved, workspace, workspace_bytes, stream) -> int:
+    return lib().lora_linear_forward(ctypes.byref(shape), ctypes.byref(weights), X, Y, saved, workspace,
+                                     workspace_bytes, stream)
+
+
+def lin_backward(shape: LinShape, weights: LinWeights, X, saved, dY, dX, dA, dB, workspace, workspace_bytes,
+                 stream) -> int:
+    return lib().lora_linear_backward(ctypes.byref(shape), ctypes.byref(weights), X, saved, dY, dX, dA, dB,
+                                      workspace, workspace_bytes, stream)

@@ -1,7 +1,7 @@
 """PyTorch-facing wrappers of the C ABI.
 
 PyTorch provides device memory and the current stream; every step of the
-LoRA SwiGLU MLP runs in the library's sm_100a kernels.  There is no fallback:
+LoRA SwiGLU MLP and of the LoRA linear runs in the library's sm_100a kernels.  There is no fallback:
 if the CUDA library is missing or the device is not a B200 the call raises.
 """
 from __future__ import annotations
@@ -287,3 +287,126 @@ class HostBatchTrainer:
         if next_Xh is None:
             self.primed = False
         return self.grads_host
+
+
+# ----------------------------------------------------------------------------- LoRA linear
+
+
+@dataclass
+class LinearWeights:
+    """One frozen projection with a LoRA adapter (nn.Linear layout).
+
+    bf16: W [d_out, d_in].  int4: W uint8 [d_out, d_in/2] and fp16 scales
+    S [d_out, d_in/64].  Adapter (bf16): A [r, d_in], B [d_out, r].
+    """
+    W: torch.Tensor
+    A: torch.Tensor
+    B: torch.Tensor
+    alpha: float
+    S: torch.Tensor | None = None
+
+    @property
+    def int4(self) -> bool:
+        return self.W.dtype == torch.uint8
+
+    @property
+    def r(self) -> int:
+        return int(self.A.shape[0])
+
+    @property
+    def d_in(self) -> int:
+        return int(self.A.shape[1])
+
+    @property
+    def d_out(self) -> int:
+        return int(self.B.shape[0])
+
+    def shape(self, N: int) -> _lib.LinShape:
+        fmt = _lib.WEIGHTS_INT4_B64 if self.int4 else _lib.WEIGHTS_BF16
+        return _lib.make_lin_shape(N, self.d_in, self.d_out, self.r, self.alpha, fmt)
+
+    def validate(self):
+        di, do, r = self.d_in, self.d_out, self.r
+        if self.int4:
+            _need(self.W, "W", torch.uint8, (do, di // 2))
+            _need(self.S, "S", torch.float16, (do, di // 64))
+        else:
+            _need(self.W, "W", BF16, (do, di))
+        _need(self.A, "A", BF16, (r, di))
+        _need(self.B, "B", BF16, (do, r))
+
+    def c_struct(self) -> _lib.LinWeights:
+        return _lib.LinWeights(self.W.data_ptr(), None if self.S is None else self.S.data_ptr(),
+                               self.A.data_ptr(), self.B.data_ptr())
+
+
+def linear_sizes(w: LinearWeights, N: int):
+    """(forward workspace, backward workspace, saved) byte counts."""
+    return _lib.lin_sizes(w.shape(N))
+
+
+def linear_forward(X: torch.Tensor, w: LinearWeights, *, Y=None, workspace: Workspace | None = None,
+                   stream=None):
+    """Y = X (W + s B A)^T.  Returns (Y, saved) where saved is the opaque
+    rank-r buffer backward needs."""
+    N = X.shape[0]
+    _need(X, "X", BF16, (N, w.d_in))
+    w.validate()
+    shape = w.shape(N)
+    fws, _, svs = _lib.lin_sizes(shape)
+    dev = X.device
+    Y = torch.empty((N, w.d_out), dtype=BF16, device=dev) if Y is None else _need(Y, "Y", BF16, (N, w.d_out))
+    saved = torch.empty(max(svs, 256), dtype=torch.uint8, device=dev)
+    ws = (workspace or Workspace()).get(fws, dev)
+    _lib.check(_lib.lin_forward(shape, w.c_struct(), _p(X), _p(Y), _p(saved), _p(ws), ws.numel(),
+                                _stream(stream)), "lora_linear_forward")
+    return Y, saved
+
+
+def linear_backward(X: torch.Tensor, w: LinearWeights, saved: torch.Tensor, dY: torch.Tensor, *, dX=None,
+                    dA=None, dB=None, workspace: Workspace | None = None, stream=None):
+    """Returns (dX, dA, dB)."""
+    N = X.shape[0]
+    _need(X, "X", BF16, (N, w.d_in))
+    _need(dY, "dY", BF16, (N, w.d_out))
+    w.validate()
+    shape = w.shape(N)
+    _, bws, _ = _lib.lin_sizes(shape)
+    dev = X.device
+    dX = torch.empty((N, w.d_in), dtype=BF16, device=dev) if dX is None else _need(dX, "dX", BF16, (N, w.d_in))
+    dA = torch.empty_like(w.A) if dA is None else _need(dA, "dA", BF16, tuple(w.A.shape))
+    dB = torch.empty_like(w.B) if dB is None else _need(dB, "dB", BF16, tuple(w.B.shape))
+    ws = (workspace or Workspace()).get(bws, dev)
+    _lib.check(_lib.lin_backward(shape, w.c_struct(), _p(X), _p(saved), _p(dY), _p(dX), _p(dA), _p(dB), _p(ws),
+                                 ws.numel(), _stream(stream)), "lora_linear_backward")
+    return dX, dA, dB
+
+
+class LoRALinearFunction(torch.autograd.Function):
+    """autograd wrapper: Y = X (W + s B A)^T.  Usage:
+    LoRALinearFunction.apply(X, w, A, B) where w is a LinearWeights whose A and
+    B are the same tensors."""
+
+    @staticmethod
+    def forward(ctx, X, w: LinearWeights, A, B):
+        Y, saved = linear_forward(X.contiguous(), w)
+        ctx.w = w
+        ctx.saved_lr = saved
+        ctx.save_for_backward(X)
+        return Y
+
+    @staticmethod
+    def backward(ctx, dY):
+        (X,) = ctx.saved_tensors
+        dX, dA, dB = linear_backward(X, ctx.w, ctx.saved_lr, dY.contiguous())
+        return dX, None, dA, dB
+
+
+def linear_weights_from_host(inp: dict, alpha: float, device="cuda") -> LinearWeights:
+    """Upload a host LoRA-linear input dict to the device."""
+    if "W_q" in inp:
+        return LinearWeights(W=torch.from_numpy(inp["W_q"]).to(device), A=to_device_bf16(inp["A"], device),
+                             B=to_device_bf16(inp["B"], device), alpha=float(alpha),
+                             S=torch.from_numpy(inp["W_scale"]).to(device))
+    return LinearWeights(W=to_device_bf16(inp["W"], device), A=to_device_bf16(inp["A"], device),
+                         B=to_device_bf16(inp["B"], device), alpha=float(alpha))

@@ -29,6 +29,7 @@
 #include <vector>
 
 #include "lora_mlp.h"
+#include "lora_linear.h"
 #include "aux_kernels.cuh"
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
@@ -1001,6 +1002,253 @@ int lora_mlp_debug_force_timeout(int enable, int64_t wait_cycles) {
     if (enable && wait_cycles < 1) return LORA_MLP_ERR_INVALID_ARG;
     g_wait_limit.store(enable ? static_cast<long long>(wait_cycles) : kWaitLimitCycles);
     g_force_timeout.store(enable ? 1 : 0);
+    return LORA_MLP_OK;
+}
+
+}  // extern "C"
+
+// ============================================================================= LoRA linear
+//
+// One LoRA-adapted projection (include/lora_linear.h), on the same engines:
+//   L0  R  = s X A^T   -> R [N, r] and saved R^T [r, ldN]      split-K, finalised in kernel
+//   L1  Y  = X W^T + R B^T                                     CTA pairs, K = d_in + r
+//   L2  T  = s dY B    -> T [N, r], T^T [r, ldN];  dB = dY^T R  split-K, two problems
+//   L3  dX = dY W + T A                                        CTA pairs, MN-major W and A
+//   L4  dA = T^T X     (written [r, d_in])                     split-K token reduction
+
+namespace {
+
+enum { LK_R, LK_TDB, LK_DA, LK_COUNT };
+constexpr int kLinProbs[LK_COUNT] = {1, 2, 1};
+
+struct LinPlan {
+    int64_t N, din, dout, r, ldN;
+    float s;
+    bool int4;
+    int bn_r, bn_r64;
+    SkinnySpec spec[LK_COUNT][kMaxProbs];
+    int splits[LK_COUNT][kMaxProbs];
+    size_t part_off[LK_COUNT][kMaxProbs];
+    size_t ctr_bytes;
+    size_t f_r, f_part, f_ctr, f_tail, f_w, f_total;
+    size_t b_t, b_tT, b_part, b_ctr, b_tail, b_w, b_total;
+    size_t s_rT, s_total;
+};
+
+LinPlan make_lin_plan(const lora_linear_shape& sh) {
+    LinPlan p{};
+    p.N = sh.N;
+    p.din = sh.d_in;
+    p.dout = sh.d_out;
+    p.r = sh.r;
+    p.ldN = round_up(sh.N, 8);
+    p.s = static_cast<float>(static_cast<double>(sh.alpha) / static_cast<double>(sh.r));
+    p.int4 = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64;
+    p.bn_r = static_cast<int>(round_up(sh.r, 32));
+    p.bn_r64 = static_cast<int>(round_up(sh.r, 64));
+    const int64_t N = p.N, di = p.din, dout = p.dout, r = p.r;
+    const int64_t kb_in = ceil_div(di, kBK), kb_out = ceil_div(dout, kBK), kb_n = ceil_div(N, kBK);
+    p.spec[LK_R][0] = {N, r, kb_in};
+    p.spec[LK_TDB][0] = {N, r, kb_out};
+    p.spec[LK_TDB][1] = {dout, r, kb_n};
+    p.spec[LK_DA][0] = {di, r, kb_n};
+    size_t part_f = 0, part_b = 0;
+    int64_t max_tiles = 0;
+    for (int l = 0; l < LK_COUNT; ++l) {
+        plan_splits(p.spec[l], kLinProbs[l], p.splits[l]);
+        size_t off = 0;
+        for (int i = 0; i < kLinProbs[l]; ++i) {
+            p.part_off[l][i] = off;
+            off += static_cast<size_t>(p.splits[l][i]) * p.spec[l][i].M * p.spec[l][i].ncols;
+        }
+        if (l == LK_R) part_f = off;
+        else part_b = std::max(part_b, off);
+        max_tiles = std::max(max_tiles, launch_tiles(p.spec[l], kLinProbs[l]));
+    }
+    p.ctr_bytes = static_cast<size_t>(std::max<int64_t>(max_tiles, 2 * kTailMaxUnits) + 8) * sizeof(int);
+    const size_t bf = 2, f32 = 4, rz = r, ldN = p.ldN;
+    const size_t wsz = static_cast<size_t>(dout) * di * bf;
+    Carver f;
+    p.f_r = f.take(static_cast<size_t>(N) * rz * bf);
+    p.f_part = f.take(part_f * f32);
+    p.f_ctr = f.take(p.ctr_bytes);
+    p.f_tail = f.take(kTailPartFloats * f32);
+    p.f_w = p.int4 ? f.take(wsz) : 0;
+    p.f_total = f.off;
+    Carver b;
+    p.b_t = b.take(static_cast<size_t>(N) * rz * bf);
+    p.b_tT = b.take(rz * ldN * bf);
+    p.b_part = b.take(part_b * f32);
+    p.b_ctr = b.take(p.ctr_bytes);
+    p.b_tail = b.take(kTailPartFloats * f32);
+    p.b_w = p.int4 ? b.take(wsz) : 0;
+    p.b_total = b.off;
+    Carver sv;
+    p.s_rT = sv.take(rz * ldN * bf);
+    p.s_total = sv.off;
+    return p;
+}
+
+int validate_lin_shape(const lora_linear_shape* sh) {
+    if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->N < 1 || sh->d_in < 1 || sh->d_out < 1 || sh->r < 1) return LORA_MLP_ERR_INVALID_ARG;
+    if (!std::isfinite(sh->alpha)) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->d_in % 8 || sh->d_out % 8 || sh->r % 8 || sh->r > 128) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64 && sh->d_in % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    const int64_t lim = (int64_t{1} << 31) - 1;
+    if (sh->N > lim || sh->d_in > lim || sh->d_out > lim) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    return LORA_MLP_OK;
+}
+
+int check_lin_weights(const lora_linear_shape* sh, const lora_linear_weights* w) {
+    if (w == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_ptrs({w->W, w->A, w->B}));
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_ptrs({w->S});
+    return LORA_MLP_OK;
+}
+
+// The bf16 frozen weight: the caller's, or int4 dequantised into the workspace.
+int lin_frozen_weight(const LinPlan& pl, const lora_linear_weights* w, uint8_t* ws, size_t off, int sms,
+                      cudaStream_t st, const void** out) {
+    if (!pl.int4) {
+        *out = w->W;
+        return LORA_MLP_OK;
+    }
+    LMLP_TRY(launch_dequant(w->W, w->S, pl.dout, pl.din, ws + off, sms, st));
+    *out = ws + off;
+    return LORA_MLP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lora_linear_sizes(const lora_linear_shape* shape, size_t* fwd_workspace_bytes, size_t* bwd_workspace_bytes,
+                      size_t* saved_bytes) {
+    LMLP_TRY(validate_lin_shape(shape));
+    const LinPlan pl = make_lin_plan(*shape);
+    if (fwd_workspace_bytes) *fwd_workspace_bytes = pl.f_total;
+    if (bwd_workspace_bytes) *bwd_workspace_bytes = pl.b_total;
+    if (saved_bytes) *saved_bytes = pl.s_total;
+    return LORA_MLP_OK;
+}
+
+int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weights* w, const void* X, void* Y,
+                        void* saved, void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_lin_shape(shape));
+    LMLP_TRY(check_lin_weights(shape, w));
+    LMLP_TRY(check_ptrs({X, Y, saved, workspace}));
+    const LinPlan pl = make_lin_plan(*shape);
+    if (workspace_bytes < pl.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* sv = static_cast<uint8_t*>(saved);
+    const int64_t N = pl.N, din = pl.din, dout = pl.dout, r = pl.r;
+    __nv_bfloat16* R = reinterpret_cast<__nv_bfloat16*>(ws + pl.f_r);
+    float* part = reinterpret_cast<float*>(ws + pl.f_part);
+    int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
+    float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
+    if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    {  // L0: R = s X A^T -> R [N, r], saved R^T [r, ldN]
+        GemmBuilder b(pl.bn_r);
+        const int ax = b.a_k(X, N, din, din);
+        const int ba = b.b_k(w->A, r, din, din);
+        Prob* p = b.prob(N, r, pl.splits[LK_R][0]);
+        b.seg(p, ax, ba, -1, din);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = N * r;
+        b.fin(p, pl.s, static_cast<int>(r), R, r, sv + pl.s_rT, nullptr, pl.ldN, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L0_lowrank_in", ctr)));
+    }
+    const void* W = nullptr;
+    LMLP_TRY(lin_frozen_weight(pl, w, ws, pl.f_w, di.sms, st, &W));
+    {  // L1: Y = X W^T + R B^T
+        PairBuilder b(N, dout, 256);
+        const int ax = b.a_k(X, N, din, din);
+        const int ar = b.a_k(R, N, r, r);
+        const int bw = b.b_k(W, dout, din, din);
+        const int bb = b.b_k(w->B, dout, r, r);
+        b.seg(ax, bw, bw, 0, kPairHalfN, 0, 0, din);
+        b.seg(ar, bb, bb, 0, kPairHalfN, 0, 0, r);
+        b.a.prob.out0 = Y;
+        b.a.prob.ld = dout;
+        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
+    }
+    return LORA_MLP_OK;
+}
+
+int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weights* w, const void* X,
+                         const void* saved, const void* dY, void* dX, void* dA, void* dB, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_lin_shape(shape));
+    LMLP_TRY(check_lin_weights(shape, w));
+    LMLP_TRY(check_ptrs({X, saved, dY, dX, dA, dB, workspace}));
+    const LinPlan pl = make_lin_plan(*shape);
+    if (workspace_bytes < pl.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    const int64_t N = pl.N, din = pl.din, dout = pl.dout, r = pl.r, ldN = pl.ldN;
+    __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_t);
+    __nv_bfloat16* TT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_tT);
+    float* part = reinterpret_cast<float*>(ws + pl.b_part);
+    int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
+    float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
+    if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    {  // L2: T = s dY B -> T [N, r], T^T [r, ldN];  dB = dY^T R (R from saved, already s-scaled)
+        const int* sp = pl.splits[LK_TDB];
+        GemmBuilder b(pl.bn_r64);
+        const int a0 = b.a_k(dY, N, dout, dout);
+        const int b0 = b.b_mn(w->B, dout, r, r);
+        const int a1 = b.a_mn(dY, N, dout, dout);
+        const int b1 = b.b_k(sv + pl.s_rT, r, N, ldN);
+        Prob* p0 = b.prob(N, r, sp[0], false, true);
+        b.seg(p0, a0, b0, -1, dout);
+        p0->out0 = part + pl.part_off[LK_TDB][0];
+        p0->ld = r;
+        p0->split_stride = N * r;
+        b.fin(p0, pl.s, static_cast<int>(r), T, r, TT, nullptr, ldN, static_cast<int>(r));
+        Prob* p1 = b.prob(dout, r, sp[1], true, false);
+        b.seg(p1, a1, b1, -1, N);
+        p1->out0 = part + pl.part_off[LK_TDB][1];
+        p1->ld = r;
+        p1->split_stride = dout * r;
+        b.fin(p1, 1.0f, static_cast<int>(r), dB, r, nullptr, nullptr, 0, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L2_lowrank_out_dB", ctr)));
+    }
+    const void* W = nullptr;
+    LMLP_TRY(lin_frozen_weight(pl, w, ws, pl.b_w, di.sms, st, &W));
+    {  // L3: dX = dY W + T A
+        PairBuilder b(N, din, 256);
+        const int ady = b.a_k(dY, N, dout, dout);
+        const int at = b.a_k(T, N, r, r);
+        const int bw = b.b_mn(W, dout, din, din);
+        const int ba = b.b_mn(w->A, r, din, din);
+        b.seg(ady, bw, bw, 0, kPairHalfN, 0, 0, dout);
+        b.seg(at, ba, ba, 0, kPairHalfN, 0, 0, r);
+        b.a.prob.out0 = dX;
+        b.a.prob.ld = din;
+        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
+    }
+    {  // L4: dA^T = X^T T  (written transposed: dA [r, d_in])
+        GemmBuilder b(pl.bn_r);
+        const int a = b.a_mn(X, N, din, din);
+        const int bt = b.b_k(TT, r, N, ldN);
+        Prob* p = b.prob(din, r, pl.splits[LK_DA][0], true, false);
+        b.seg(p, a, bt, -1, N);
+        p->out0 = part;
+        p->ld = r;
+        p->split_stride = din * r;
+        b.fin(p, 1.0f, static_cast<int>(r), nullptr, 0, dA, nullptr, din, static_cast<int>(r));
+        LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L4_dA", ctr)));
+    }
     return LORA_MLP_OK;
 }
 

@@ -11,7 +11,7 @@ from lora_fine_tuning_mlp_b200 import _lib
 from lora_fine_tuning_mlp_b200 import build as libbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "lora_mlp.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("lora_mlp.h", "lora_linear.h")]
 
 
 @pytest.fixture(scope="module")
@@ -21,9 +21,9 @@ def L():
 
 
 def header_symbols():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(lora_mlp_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(lora_(?:mlp|linear)_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_symbols():
@@ -141,3 +141,53 @@ def test_timing_toggle_without_gpu(L):
     _lib.timing_enable(False)
     assert _lib.timing_collect() == []
     assert _lib.launch_count() == 0
+
+
+# ----------------------------------------------------------------------------- LoRA linear
+
+
+def lshape(N=300, d_in=192, d_out=320, r=8, alpha=16.0, fmt=0):
+    return _lib.make_lin_shape(N, d_in, d_out, r, alpha, fmt)
+
+
+def test_linear_sizes(L):
+    f1, b1, s1 = _lib.lin_sizes(lshape(N=300))
+    f2, b2, s2 = _lib.lin_sizes(lshape(N=4096))
+    assert 0 < f1 < f2 and 0 < b1 < b2 and 0 < s1 < s2
+    assert s1 >= 8 * 304 * 2          # s X A^T kept as bf16 [r, N padded to 8]
+    f4, b4, _ = _lib.lin_sizes(lshape(d_in=256, fmt=1))
+    f0, b0, _ = _lib.lin_sizes(lshape(d_in=256, fmt=0))
+    assert f4 - f0 >= 320 * 256 * 2 and b4 - b0 >= 320 * 256 * 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), _lib.ERR_INVALID_ARG),
+    (dict(d_out=-8), _lib.ERR_INVALID_ARG),
+    (dict(alpha=float("nan")), _lib.ERR_INVALID_ARG),
+    (dict(fmt=3), _lib.ERR_INVALID_ARG),
+    (dict(d_in=196), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(d_out=324), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(r=4), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(r=136), _lib.ERR_UNSUPPORTED_SHAPE),
+    (dict(d_in=200, fmt=1), _lib.ERR_UNSUPPORTED_SHAPE),
+])
+def test_linear_shape_validation(L, kw, code):
+    f = ctypes.c_size_t()
+    assert L.lora_linear_sizes(ctypes.byref(lshape(**kw)), ctypes.byref(f), None, None) == code
+
+
+def test_linear_argument_errors(L):
+    sh = lshape()
+    fws, bws, _ = _lib.lin_sizes(sh)
+    w = _lib.LinWeights(FAKE, None, FAKE, FAKE)
+    assert _lib.lin_forward(sh, w, FAKE, FAKE, FAKE, FAKE, fws - 1, None) == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.lin_forward(sh, w, None, FAKE, FAKE, FAKE, fws, None) == _lib.ERR_INVALID_ARG
+    assert _lib.lin_forward(sh, _lib.LinWeights(FAKE, None, FAKE + 2, FAKE), FAKE, FAKE, FAKE, FAKE, fws,
+                            None) == _lib.ERR_MISALIGNED
+    assert _lib.lin_forward(lshape(d_in=256, fmt=1), w, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) \
+        == _lib.ERR_INVALID_ARG     # int4 needs the scales
+    assert _lib.lin_backward(sh, w, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, bws, None) == _lib.ERR_INVALID_ARG
+    assert _lib.lin_backward(sh, w, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, FAKE, bws, None) \
+        == _lib.ERR_MISALIGNED
+    assert _lib.lin_backward(sh, w, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bws - 1, None) \
+        == _lib.ERR_WORKSPACE_TOO_SMALL
