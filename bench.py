@@ -315,6 +315,25 @@ def b200_arm(args, cfg):
     launches = _lib.launch_count() - launches0
     ms_max = replicas.max_over_ranks(t0.elapsed_time(t1), device=dev)
 
+    # ---- forward alone and backward alone (same protocol, device-timed)
+    _, saved_fb = api.forward(X, w, out=out, workspace=wsf)
+
+    def timed_region(fn):
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return replicas.max_over_ranks(a.elapsed_time(b), device=dev) / args.steps
+
+    fwd_ms = timed_region(lambda: api.forward(X, w, out=out, workspace=wsf))
+    bwd_ms = timed_region(lambda: api.backward(X, w, saved_fb, dOut, dX=dX, grads=grads, workspace=wsb))
+    del saved_fb
+
     # ---- second timed region of the same work with the library's CUDA events
     # around every launch (on the stream each kernel runs on): the per-kernel
     # durations behind the roofline figures.
@@ -386,6 +405,9 @@ def b200_arm(args, cfg):
                 "measured_sustained": tflops / world / peaks["bf16_tflops_sustained"],
                 "nominal_2250": tflops / world / 2250.0},
             "roofline": roof,
+            "fwd_ms_per_step": fwd_ms, "bwd_ms_per_step": bwd_ms,
+            "fwd_tflops_per_gpu": cfg.flops_fwd() / (fwd_ms * 1e-3) / 1e12,
+            "bwd_tflops_per_gpu": cfg.flops_bwd() / (bwd_ms * 1e-3) / 1e12,
             "e2e": {"value": replicas.job_throughput(N, args.steps, ems, world), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "what": "api.HostBatchTrainer: per step H2D of X and dOut from pinned host (overlapped with "

@@ -17,42 +17,85 @@ __device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 v) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(v));
 }
 
-// One thread per 64-element block (one scale): the magnitudes for |q| = 0..8
-// are computed once with dequant_one, then every code is a lookup plus a sign
-// flip.  This equals dequant_one(q, scale) bit for bit, because q*scale is
-// exact and round-to-nearest-even is symmetric in sign: fl(-x) = -fl(x).
-// Packed rows are [rows, cols/2] bytes, scales [rows, cols/64], both row-major,
-// so block i's 32 code bytes start at byte 32*i and its outputs at element 64*i.
-__global__ void __launch_bounds__(256) dequant_int4_kernel(const uint4* __restrict__ packed,
-                                                           const __half* __restrict__ scales, long long rows,
-                                                           long long cols, __nv_bfloat16* __restrict__ w) {
-    const long long total = rows * (cols / 64);
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const float sc = __half2float(scales[i]);
-        uint32_t mag[9];
+// Warp-cooperative dequantisation.  Packed codes [rows, cols/2] bytes and
+// scales [rows, cols/64] are row-major, so flat block i (64 elements, one
+// scale) has its 32 code bytes at byte 32*i and its outputs at element 64*i.
+// A warp takes kDqPasses passes of 8 consecutive blocks (512 elements) per
+// iteration:
+//  1. every lane issues its loads first (the scale of block L/4 and two
+//     4-byte code words per pass), so their latencies overlap;
+//  2. lane L computes magnitudes L%4 and L%4+4 (and 8 when L%4 = 0) of block
+//     L/4 with dequant_one and writes them to that block's 16-entry table in
+//     shared memory at the code's two's-complement nibble, the negative code
+//     -m at nibble 16-m with the sign bit flipped.  This equals
+//     dequant_one(-m, scale) bit for bit: q*scale is exact and round to
+//     nearest even is symmetric in sign, fl(-x) = -fl(x);
+//  3. lane L converts the 8 codes of elements 8L .. 8L+7 and 256+8L ..
+//     256+8L+7 of each pass with table lookups: one 4-byte load and one
+//     16-byte store each, so a warp's loads and stores cover contiguous
+//     128 B and 512 B spans.
+constexpr int kDqWarps = 8;
+#ifndef LMLP_DQ_PASSES
+#define LMLP_DQ_PASSES 2
+#endif
+constexpr int kDqPasses = LMLP_DQ_PASSES;
+
+__global__ void __launch_bounds__(kDqWarps * 32) dequant_int4_kernel(const uint32_t* __restrict__ packed,
+                                                                     const __half* __restrict__ scales,
+                                                                     long long nblocks,
+                                                                     __nv_bfloat16* __restrict__ w) {
+    __shared__ uint32_t tab[kDqWarps][kDqPasses * 8 * 16];
+    const int lane = threadIdx.x & 31;
+    const int wid = threadIdx.x >> 5;
+    uint32_t* t = tab[wid];
+    const long long nchunks = (nblocks + 8 * kDqPasses - 1) / (8 * kDqPasses);
+    for (long long c = static_cast<long long>(blockIdx.x) * kDqWarps + wid; c < nchunks;
+         c += static_cast<long long>(gridDim.x) * kDqWarps) {
+        const long long cb = c * (8 * kDqPasses);  // first block of this iteration
+        float sc[kDqPasses];
+        uint32_t word[kDqPasses][2];
 #pragma unroll
-        for (int m = 0; m < 9; ++m) mag[m] = bf16_bits(dequant_one(m, sc));
-        const uint4 p0 = packed[2 * i], p1 = packed[2 * i + 1];
-        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint4* out = reinterpret_cast<uint4*>(w + i * 64);
+        for (int p = 0; p < kDqPasses; ++p) {
+            const long long b = cb + p * 8 + (lane >> 2);
+            sc[p] = b < nblocks ? __half2float(scales[b]) : 0.0f;
 #pragma unroll
-        for (int wd = 0; wd < 8; ++wd) {
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t half2[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int nib = static_cast<int>((words[wd] >> (8 * e + 4 * h)) & 0xFu);
-                    const int q = nib >= 8 ? nib - 16 : nib;
-                    const uint32_t m = mag[q < 0 ? -q : q];
-                    half2[h] = q < 0 ? (m ^ 0x8000u) : m;
-                }
-                o[e] = half2[0] | (half2[1] << 16);
+            for (int h = 0; h < 2; ++h) {
+                const int e0 = h * 256 + lane * 8;
+                const long long e = (cb + p * 8) * 64 + e0;
+                word[p][h] = (cb + p * 8 + (e0 >> 6)) < nblocks ? packed[e >> 3] : 0u;
             }
-            out[wd] = make_uint4(o[0], o[1], o[2], o[3]);
         }
+#pragma unroll
+        for (int p = 0; p < kDqPasses; ++p) {
+            uint32_t* tb = t + (p * 8 + (lane >> 2)) * 16;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int m = (lane & 3) + 4 * j;
+                const uint32_t v = bf16_bits(dequant_one(m, sc[p]));
+                tb[m] = v;
+                if (m != 0) tb[16 - m] = v ^ 0x8000u;
+            }
+            if ((lane & 3) == 0) tb[8] = bf16_bits(dequant_one(8, sc[p])) ^ 0x8000u;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < kDqPasses; ++p) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e0 = h * 256 + lane * 8;
+                const int lb = p * 8 + (e0 >> 6);
+                if (cb + lb < nblocks) {
+                    const uint32_t* tb = t + lb * 16;
+                    const uint32_t wd = word[p][h];
+                    uint32_t o[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        o[k] = tb[(wd >> (8 * k)) & 0xFu] | (tb[(wd >> (8 * k + 4)) & 0xFu] << 16);
+                    *reinterpret_cast<uint4*>(w + (cb + p * 8) * 64 + e0) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        __syncwarp();
     }
 }
 
