@@ -278,6 +278,7 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     b.finish(counters);
     if (!b.ok) return LORA_MLP_ERR_CUDA;
     GemmArgs& a = b.a;
+    a.nmaps = b.nmaps;
     a.b_bytes = static_cast<uint32_t>(a.bn * 128);  // K-major: bn rows x 128 B; MN-major: bn/64 chunks x 8 KB
     const uint32_t stage_bytes = kATileBytes + NACC * a.b_bytes;
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
@@ -380,6 +381,7 @@ template <bool B_MN, int EPI>
 int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, float* tail_part, int* tail_ctr) {
     if (!b.ok) return LORA_MLP_ERR_CUDA;
     PairArgs& a = b.a;
+    a.nmaps = b.nmaps;
     const int tiles = a.prob.tiles_m * a.prob.tiles_n;
     a.total_units = tiles;
     a.full_units = tiles;

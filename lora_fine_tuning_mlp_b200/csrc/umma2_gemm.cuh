@@ -82,6 +82,7 @@ struct alignas(64) PairArgs {
     int* tail_ctr;     // [tail tile][rank], zero before the launch
     long long wait_limit;  // SM cycles a barrier wait may spin before the kernel gives up
     int force_timeout;     // test hook: the epilogue waits on a barrier nothing signals
+    int nmaps;             // maps[0, nmaps) are encoded
 };
 
 struct PairUnit {
@@ -307,6 +308,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
 
+    // Tensor maps are launch parameters: prefetch them under the previous
+    // kernel's tail (programmatic dependent launch).
+    if (warp == 0 && lane < args.nmaps) tma_prefetch_desc(&args.maps[lane]);
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < args.stages; ++s) {
             mbar_init(c.full + 8u * s, 1);

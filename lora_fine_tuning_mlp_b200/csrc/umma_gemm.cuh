@@ -90,6 +90,7 @@ struct alignas(64) GemmArgs {
     uint32_t b_bytes;  // one B tile: bn rows (or bn/64 MN chunks) x 128 B
     long long wait_limit;  // SM cycles a barrier wait may spin before the kernel gives up
     int force_timeout;     // test hook: the epilogue waits on a barrier nothing signals
+    int nmaps;             // maps[0, nmaps) are encoded
 };
 
 struct Unit {
@@ -446,6 +447,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid
     const int lane = threadIdx.x & 31;
     const uint32_t tmem_cols = gemm_tmem_cols(NACC, args.bn);
 
+    // The tensor maps are launch parameters, not outputs of an earlier
+    // launch: fetching them now overlaps that latency with the previous
+    // kernel's tail (programmatic dependent launch).
+    if (warp == 0 && lane < args.nmaps) tma_prefetch_desc(&args.maps[lane]);
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < args.stages; ++s) {
             mbar_init(c.full + 8u * s, 1);
