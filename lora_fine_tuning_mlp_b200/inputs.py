@@ -213,3 +213,22 @@ def make_linear_inputs(cfg: LinearConfig) -> dict:
         else:
             out[k] = f32_to_bf16_bits(v)
     return out
+
+
+# ----------------------------------------------------------------------------- pre-norm block
+
+RMS_EPS = 1e-5
+
+
+def make_block_inputs(cfg: Config) -> dict:
+    """Inputs of the pre-norm block out = MLP(RMSNorm(X)): the MLP inputs of
+    `cfg` with every row of X rescaled by a log-uniform factor in [1/4, 4]
+    (so rows have different RMS, like a residual stream) and a frozen gain
+    gamma ~ U(0.5, 1.5) [d].  Both come from a second generator (seed + 7919),
+    so the MLP inputs themselves are unchanged; X is rounded to bf16 again."""
+    out = make_inputs(cfg)
+    rng = np.random.Generator(np.random.PCG64(cfg.seed + 7919))
+    scale = np.exp(rng.uniform(np.log(0.25), np.log(4.0), size=(cfg.N, 1))).astype(np.float32)
+    out["X"] = f32_to_bf16_bits(bf16_bits_to_f32(out["X"]) * scale)
+    out["gamma"] = f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=cfg.d).astype(np.float32))
+    return out

@@ -16,3 +16,4 @@ from .lora_mlp import (  # noqa: F401
     weights_f64,
 )
 from . import lora_linear  # noqa: F401,E402
+from . import rmsnorm  # noqa: F401,E402

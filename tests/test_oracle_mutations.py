@@ -133,3 +133,55 @@ def test_forward_mistakes_are_caught(kind):
 @pytest.mark.parametrize("kind", ["drop_curvature_term", "wrong_sign", "missing_lora_dx", "transposed_dB_operand"])
 def test_backward_mistakes_are_caught(kind):
     assert not fd_pin_holds(oracle.forward, mutated_backward(kind))
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+
+from oracle import rmsnorm as orn  # noqa: E402
+
+
+def rms_pins_hold(fwd, bwd):
+    """Library rms_norm (forward + autograd backward) and central differences."""
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((5, 12)) * rng.uniform(0.2, 4.0, (5, 1))
+    gamma = rng.uniform(0.5, 1.5, 12)
+    dy = rng.standard_normal((5, 12))
+    eps = 1e-3
+    y, rstd = fwd(x, gamma, eps)
+    tx = torch.from_numpy(x.copy()).requires_grad_(True)
+    ty = torch.nn.functional.rms_norm(tx, (12,), torch.from_numpy(gamma), eps=eps)
+    ty.backward(torch.from_numpy(dy))
+    if np.max(np.abs(y - ty.detach().numpy())) > 1e-12:
+        return False
+    dx = bwd(x, gamma, rstd, dy)
+    return bool(np.max(np.abs(dx - tx.grad.numpy())) <= 1e-10 * np.max(np.abs(dx)))
+
+
+def test_rmsnorm_pins_accept_the_oracle():
+    assert rms_pins_hold(orn.rmsnorm_forward, orn.rmsnorm_backward)
+
+
+RMS_MUTANTS = {
+    # variance about the mean instead of the mean square
+    "centred": (lambda x, g, e: (x * (1 / np.sqrt(np.var(x, axis=1) + e))[:, None] * g,
+                                 1 / np.sqrt(np.var(x, axis=1) + e)), orn.rmsnorm_backward),
+    # eps outside the square root
+    "eps_outside": (lambda x, g, e: (x * (1 / (np.sqrt(np.mean(x * x, axis=1)) + e))[:, None] * g,
+                                     1 / (np.sqrt(np.mean(x * x, axis=1)) + e)), orn.rmsnorm_backward),
+    # backward drops the projection term
+    "no_projection": (orn.rmsnorm_forward, lambda x, g, r, dy: r[:, None] * dy * g),
+    # backward forgets gamma inside the projection
+    "gamma_outside_mean": (orn.rmsnorm_forward,
+                           lambda x, g, r, dy: r[:, None] * (dy * g - (x * r[:, None]) * np.mean(
+                               dy * x * r[:, None], axis=1)[:, None])),
+    # backward uses sum instead of mean
+    "sum_not_mean": (orn.rmsnorm_forward,
+                     lambda x, g, r, dy: r[:, None] * (dy * g - (x * r[:, None]) * np.sum(
+                         dy * g * x * r[:, None], axis=1)[:, None])),
+}
+
+
+@pytest.mark.parametrize("name", sorted(RMS_MUTANTS))
+def test_rmsnorm_pins_reject_mutant(name):
+    fwd, bwd = RMS_MUTANTS[name]
+    assert not rms_pins_hold(fwd, bwd)
