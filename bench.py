@@ -166,23 +166,42 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 
-def time_oracle(cfg, budget_s: float, inp=None):
+def oracle_inputs(cfg, block=False):
+    c = synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4, seed_index=cfg.index)
+    return synth.make_block_inputs(c) if block else synth.make_inputs(c)
+
+
+def oracle_step(p, x, dOut, alpha, gamma=None):
+    """One fp64 oracle forward + backward (of the pre-norm block when gamma is given)."""
+    import oracle
+    from oracle import rmsnorm as orn
+
+    if gamma is None:
+        p["X"] = x
+        oracle.backward(p, alpha, dOut, oracle.forward(p, alpha))
+        return
+    xn, rstd = orn.rmsnorm_forward(x, gamma, synth.RMS_EPS)
+    p["X"] = xn
+    b = oracle.backward(p, alpha, dOut, oracle.forward(p, alpha))
+    orn.rmsnorm_backward(x, gamma, rstd, b["dX"])
+
+
+def time_oracle(cfg, budget_s: float, inp=None, block=False):
     """Time the fp64 oracle forward+backward on a token sample of `cfg` sized
-    to take about budget_s.  Returns (tokens/s, sample tokens, seconds, threads)."""
+    to take about budget_s.  Returns (tokens/s, sample tokens, seconds)."""
     import oracle
 
     if inp is None:
-        inp = synth.make_inputs(synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4,
-                                             seed_index=cfg.index))
-    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut")})
+        inp = oracle_inputs(cfg, block)
+    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut", "gamma")})
+    gamma = oracle.bf16_to_f64(inp["gamma"]) if block else None
 
     def run(n):
         p = dict(p_full)
-        p["X"] = oracle.bf16_to_f64(inp["X"][:n])
+        x = oracle.bf16_to_f64(inp["X"][:n])
         dOut = oracle.bf16_to_f64(inp["dOut"][:n])
         t0 = time.perf_counter()
-        f = oracle.forward(p, cfg.alpha)
-        oracle.backward(p, cfg.alpha, dOut, f)
+        oracle_step(p, x, dOut, cfg.alpha, gamma)
         return time.perf_counter() - t0
 
     t_probe = run(32)
@@ -214,20 +233,20 @@ def reference_arm(args, cfg):
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     import oracle
 
-    inp = synth.make_inputs(synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4,
-                                         seed_index=cfg.index))
-    _, n, _ = time_oracle(cfg, per_step, inp)
-    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut")})
+    block = getattr(args, "block", False)
+    inp = oracle_inputs(cfg, block)
+    _, n, _ = time_oracle(cfg, per_step, inp, block)
+    p_full = oracle.weights_f64({k: v for k, v in inp.items() if k not in ("X", "dOut", "gamma")})
+    gamma = oracle.bf16_to_f64(inp["gamma"]) if block else None
     times = []
     for i in range(args.warmup + args.steps):
         lo = (i * n) % inp["X"].shape[0]
         idx = np.arange(lo, lo + n) % inp["X"].shape[0]
         p = dict(p_full)
-        p["X"] = oracle.bf16_to_f64(inp["X"][idx])
+        x = oracle.bf16_to_f64(inp["X"][idx])
         dOut = oracle.bf16_to_f64(inp["dOut"][idx])
         t0 = time.perf_counter()
-        f = oracle.forward(p, cfg.alpha)
-        oracle.backward(p, cfg.alpha, dOut, f)
+        oracle_step(p, x, dOut, cfg.alpha, gamma)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
@@ -238,17 +257,23 @@ def reference_arm(args, cfg):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(cfg),
+        "config": config_dict(cfg, getattr(args, "block", False)),
         "tflops": cfg.flops() * (n / cfg.N) * len(times) / total / 1e12,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle)"},
+                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle"
+                                   + (", pre-norm block" if block else "") + ")"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_dict(cfg):
+def config_dict(cfg, block=False):
+    if block:
+        d = config_dict(cfg)
+        d["workload"] = "llama3_8b_block" if cfg.name == "llama3_8b_mlp" else cfg.name + "_block"
+        d["prenorm"] = f"RMSNorm (frozen gain), eps {synth.RMS_EPS}; out = MLP(RMSNorm(X))"
+        return d
     return {"workload": cfg.name, "N_tokens": cfg.N, "d": cfg.d, "d_ff": cfg.d_ff, "r": cfg.r, "alpha": cfg.alpha,
             "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
             "l2": "no flush: inputs larger than L2 (frozen weights %.0f MB > 126 MB)" % (
@@ -273,10 +298,13 @@ def b200_arm(args, cfg):
     dev = torch.device("cuda", torch.cuda.current_device())
     _lib.lib()
 
-    inp = synth.make_inputs(cfg)
+    block = args.block
+    inp = synth.make_block_inputs(cfg) if block else synth.make_inputs(cfg)
     w = api.weights_from_host(inp, cfg.alpha, dev)
     X = api.to_device_bf16(inp["X"], dev)
     dOut = api.to_device_bf16(inp["dOut"], dev)
+    gamma = api.to_device_bf16(inp["gamma"], dev) if block else None
+    eps = synth.RMS_EPS
     N, d, f = cfg.N, cfg.d, cfg.d_ff
     out = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
@@ -284,9 +312,19 @@ def b200_arm(args, cfg):
     wsf, wsb = api.Workspace(), api.Workspace()
     stream = torch.cuda.current_stream()
 
+    def fwd(x=X):
+        if block:
+            return api.block_forward(x, w, gamma, eps, out=out, workspace=wsf)
+        return api.forward(x, w, out=out, workspace=wsf)
+
+    def bwd(saved, x=X, g_out=dOut):
+        if block:
+            return api.block_backward(x, w, gamma, saved, g_out, dX=dX, grads=grads, workspace=wsb)
+        return api.backward(x, w, saved, g_out, dX=dX, grads=grads, workspace=wsb)
+
     def step(x=X, g_out=dOut):
-        o, saved = api.forward(x, w, out=out, workspace=wsf)
-        api.backward(x, w, saved, g_out, dX=dX, grads=grads, workspace=wsb)
+        o, saved = fwd(x)
+        bwd(saved, x, g_out)
 
     barrier = replicas.barrier
 
@@ -316,7 +354,7 @@ def b200_arm(args, cfg):
     ms_max = replicas.max_over_ranks(t0.elapsed_time(t1), device=dev)
 
     # ---- forward alone and backward alone (same protocol, device-timed)
-    _, saved_fb = api.forward(X, w, out=out, workspace=wsf)
+    _, saved_fb = fwd()
 
     def timed_region(fn):
         barrier()
@@ -330,8 +368,8 @@ def b200_arm(args, cfg):
         barrier()
         return replicas.max_over_ranks(a.elapsed_time(b), device=dev) / args.steps
 
-    fwd_ms = timed_region(lambda: api.forward(X, w, out=out, workspace=wsf))
-    bwd_ms = timed_region(lambda: api.backward(X, w, saved_fb, dOut, dX=dX, grads=grads, workspace=wsb))
+    fwd_ms = timed_region(fwd)
+    bwd_ms = timed_region(lambda: bwd(saved_fb))
     del saved_fb
 
     # ---- second timed region of the same work with the library's CUDA events
@@ -353,7 +391,7 @@ def b200_arm(args, cfg):
     # step's compute) and reads its six adapter gradients back to the host.
     Xh = [torch.from_numpy(inp["X"].view("int16")).view(torch.bfloat16).pin_memory() for _ in range(2)]
     dOh = [torch.from_numpy(inp["dOut"].view("int16")).view(torch.bfloat16).pin_memory() for _ in range(2)]
-    trainer = api.HostBatchTrainer(w, N, dev)
+    trainer = api.HostBatchTrainer(w, N, dev, gamma=gamma, eps=eps)
     h2d, d2h = trainer.h2d_bytes(), trainer.d2h_bytes()
 
     def run_e2e(n):
@@ -399,7 +437,7 @@ def b200_arm(args, cfg):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args.block),
             "tflops": tflops, "frac_of_peak": {
                 "measured_burst": tflops / world / peaks["bf16_tflops"],
                 "measured_sustained": tflops / world / peaks["bf16_tflops_sustained"],
@@ -419,7 +457,7 @@ def b200_arm(args, cfg):
             "kernels_note": "per-launch CUDA events, second timed region of the same length (events stop launch overlap)",
         }
         if world == 1 and not args.no_cpu_baseline:
-            tps, n, dt = time_oracle(cfg, args.cpu_budget)
+            tps, n, dt = time_oracle(cfg, args.cpu_budget, block=args.block)
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
                                     "sample": f"{n} tokens of the {cfg.name} shapes, numpy fp64 oracle, {dt:.1f} s"}
         print(json.dumps(line), flush=True)
@@ -489,7 +527,8 @@ def linear_reference_arm(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": linear_config_dict(cfg),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
-                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle)"},
+                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle"
+                                   + (", pre-norm block" if block else "") + ")"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -642,7 +681,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=("b200", "reference"))
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(synth.BY_NAME) + sorted(synth.LINEAR_BY_NAME))
+                    choices=sorted(synth.BY_NAME) + sorted(synth.LINEAR_BY_NAME) + sorted(synth.BLOCK_BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
@@ -651,7 +690,9 @@ def main():
     if args.workload in synth.LINEAR_BY_NAME:
         cfg = synth.LINEAR_BY_NAME[args.workload]
         return linear_reference_arm(args, cfg) if args.impl == "reference" else linear_arm(args, cfg)
-    cfg = synth.BY_NAME[args.workload]
+    block = args.workload in synth.BLOCK_BY_NAME
+    cfg = synth.BLOCK_BY_NAME[args.workload] if block else synth.BY_NAME[args.workload]
+    args.block = block
     if args.impl == "reference":
         return reference_arm(args, cfg)
     return b200_arm(args, cfg)

@@ -1,4 +1,4 @@
-"""ctypes binding of liblora_mlp.so (include/lora_mlp.h, include/lora_linear.h).
+"""ctypes binding of liblora_mlp.so (include/lora_mlp.h, lora_linear.h, lora_rmsnorm.h).
 
 Argument marshalling only: every step of the MLP runs in the library's CUDA
 kernels.  Loading fails loudly if the shared library has not been built.
@@ -27,7 +27,7 @@ WEIGHTS_INT4_B64 = 1
 WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Sg", "Su", "Sd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 
-# Every symbol include/lora_mlp.h and include/lora_linear.h declare.
+# Every symbol include/lora_mlp.h, lora_linear.h and lora_rmsnorm.h declare.
 SYMBOLS = (
     "lora_mlp_sizes",
     "lora_mlp_forward",
@@ -43,6 +43,11 @@ SYMBOLS = (
     "lora_linear_sizes",
     "lora_linear_forward",
     "lora_linear_backward",
+    "lora_rmsnorm_forward",
+    "lora_rmsnorm_backward",
+    "lora_mlp_block_sizes",
+    "lora_mlp_block_forward",
+    "lora_mlp_block_backward",
 )
 
 
@@ -116,12 +121,22 @@ def lib() -> ctypes.CDLL:
                                               vp, sz, vp]
             L.lora_linear_backward.argtypes = [ctypes.POINTER(LinShape), ctypes.POINTER(LinWeights), vp, vp, vp,
                                                vp, vp, vp, vp, sz, vp]
+            L.lora_rmsnorm_forward.argtypes = [i64, i64, ctypes.c_float, vp, vp, vp, vp, vp]
+            L.lora_rmsnorm_backward.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp]
+            L.lora_mlp_block_sizes.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                               ctypes.POINTER(sz)]
+            L.lora_mlp_block_forward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, ctypes.c_float,
+                                                 vp, vp, vp, vp, vp, vp, sz, vp]
+            L.lora_mlp_block_backward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
+                                                  vp, vp, vp, ctypes.POINTER(Grads), vp, sz, vp]
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
                          "lora_mlp_dequant_int4",
                          "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect",
-                         "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward"):
+                         "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward",
+                         "lora_rmsnorm_forward", "lora_rmsnorm_backward", "lora_mlp_block_sizes",
+                         "lora_mlp_block_forward", "lora_mlp_block_backward"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -217,3 +232,30 @@ def lin_backward(shape: LinShape, weights: LinWeights, X, saved, dY, dX, dA, dB,
                  stream) -> int:
     return lib().lora_linear_backward(ctypes.byref(shape), ctypes.byref(weights), X, saved, dY, dX, dA, dB,
                                       workspace, workspace_bytes, stream)
+
+
+def block_sizes(shape: Shape):
+    f, b, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().lora_mlp_block_sizes(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b), ctypes.byref(s)),
+          "lora_mlp_block_sizes")
+    return f.value, b.value, s.value
+
+
+def block_forward(shape: Shape, weights: Weights, gamma, eps, X, out, g, u, saved, workspace, workspace_bytes,
+                  stream) -> int:
+    return lib().lora_mlp_block_forward(ctypes.byref(shape), ctypes.byref(weights), gamma, float(eps), X, out, g, u,
+                                        saved, workspace, workspace_bytes, stream)
+
+
+def block_backward(shape: Shape, weights: Weights, gamma, X, g, u, saved, dOut, dX, grads: Grads, workspace,
+                   workspace_bytes, stream) -> int:
+    return lib().lora_mlp_block_backward(ctypes.byref(shape), ctypes.byref(weights), gamma, X, g, u, saved, dOut,
+                                         dX, ctypes.byref(grads), workspace, workspace_bytes, stream)
+
+
+def rmsnorm_forward(N, d, eps, x, gamma, y, rstd, stream) -> int:
+    return lib().lora_rmsnorm_forward(int(N), int(d), float(eps), x, gamma, y, rstd, stream)
+
+
+def rmsnorm_backward(N, d, x, gamma, rstd, dy, dx, stream) -> int:
+    return lib().lora_rmsnorm_backward(int(N), int(d), x, gamma, rstd, dy, dx, stream)

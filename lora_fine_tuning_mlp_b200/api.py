@@ -234,9 +234,11 @@ class HostBatchTrainer:
     overlap with compute is new.
     """
 
-    def __init__(self, w: MLPWeights, N: int, device=None):
+    def __init__(self, w: MLPWeights, N: int, device=None, gamma: torch.Tensor | None = None, eps: float = 1e-5):
+        """With `gamma`, each step runs the pre-norm block MLP(RMSNorm(X))."""
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.w, self.N, self.dev = w, N, dev
+        self.gamma, self.eps = gamma, eps
         d = w.d
         self.X = [torch.empty((N, d), dtype=BF16, device=dev) for _ in range(2)]
         self.dOut = [torch.empty((N, d), dtype=BF16, device=dev) for _ in range(2)]
@@ -278,8 +280,13 @@ class HostBatchTrainer:
             self._stage(nxt, next_Xh, next_dOh)
         stream = torch.cuda.current_stream(self.dev)
         stream.wait_event(self.ready[cur])
-        o, saved = forward(self.X[cur], self.w, out=self.out, workspace=self.wsf)
-        backward(self.X[cur], self.w, saved, self.dOut[cur], dX=self.dX, grads=self.grads, workspace=self.wsb)
+        if self.gamma is None:
+            o, saved = forward(self.X[cur], self.w, out=self.out, workspace=self.wsf)
+            backward(self.X[cur], self.w, saved, self.dOut[cur], dX=self.dX, grads=self.grads, workspace=self.wsb)
+        else:
+            o, saved = block_forward(self.X[cur], self.w, self.gamma, self.eps, out=self.out, workspace=self.wsf)
+            block_backward(self.X[cur], self.w, self.gamma, saved, self.dOut[cur], dX=self.dX, grads=self.grads,
+                           workspace=self.wsb)
         self.free[cur].record(stream)
         for k, v in self.grads.items():
             self.grads_host[k].copy_(v, non_blocking=True)
@@ -410,3 +417,92 @@ def linear_weights_from_host(inp: dict, alpha: float, device="cuda") -> LinearWe
                              S=torch.from_numpy(inp["W_scale"]).to(device))
     return LinearWeights(W=to_device_bf16(inp["W"], device), A=to_device_bf16(inp["A"], device),
                          B=to_device_bf16(inp["B"], device), alpha=float(alpha))
+
+
+# ----------------------------------------------------------------------------- RMSNorm and the pre-norm block
+
+
+def rmsnorm_forward(x: torch.Tensor, gamma: torch.Tensor, eps: float, *, stream=None):
+    """Returns (y, rstd): y = RMSNorm(x) * gamma (bf16), rstd fp32 [N]."""
+    N, d = x.shape
+    _need(x, "x", BF16)
+    _need(gamma, "gamma", BF16, (d,))
+    y = torch.empty_like(x)
+    rstd = torch.empty((N,), dtype=torch.float32, device=x.device)
+    _lib.check(_lib.rmsnorm_forward(N, d, eps, _p(x), _p(gamma), _p(y), _p(rstd), _stream(stream)),
+               "lora_rmsnorm_forward")
+    return y, rstd
+
+
+def rmsnorm_backward(x: torch.Tensor, gamma: torch.Tensor, rstd: torch.Tensor, dy: torch.Tensor, *, stream=None):
+    N, d = x.shape
+    _need(x, "x", BF16)
+    _need(gamma, "gamma", BF16, (d,))
+    _need(rstd, "rstd", torch.float32, (N,))
+    _need(dy, "dy", BF16, (N, d))
+    dx = torch.empty_like(x)
+    _lib.check(_lib.rmsnorm_backward(N, d, _p(x), _p(gamma), _p(rstd), _p(dy), _p(dx), _stream(stream)),
+               "lora_rmsnorm_backward")
+    return dx
+
+
+def block_forward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, eps: float, *, out=None,
+                  workspace: Workspace | None = None, stream=None):
+    """out = MLP(RMSNorm(X) * gamma).  Returns (out, Saved); Saved.lowrank
+    also holds the per-row rstd."""
+    N, d = X.shape
+    _need(X, "X", BF16, (N, w.d))
+    _need(gamma, "gamma", BF16, (w.d,))
+    w.validate()
+    shape = w.shape(N)
+    fws, _, svs = _lib.block_sizes(shape)
+    dev = X.device
+    out = torch.empty((N, d), dtype=BF16, device=dev) if out is None else _need(out, "out", BF16, (N, d))
+    g = torch.empty((N, w.d_ff), dtype=BF16, device=dev)
+    u = torch.empty((N, w.d_ff), dtype=BF16, device=dev)
+    saved = torch.empty(max(svs, 256), dtype=torch.uint8, device=dev)
+    ws = (workspace or Workspace()).get(fws, dev)
+    _lib.check(_lib.block_forward(shape, w.c_struct(), _p(gamma), eps, _p(X), _p(out), _p(g), _p(u), _p(saved),
+                                  _p(ws), ws.numel(), _stream(stream)), "lora_mlp_block_forward")
+    return out, Saved(g, u, saved)
+
+
+def block_backward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, saved: Saved, dOut: torch.Tensor, *,
+                   dX=None, grads=None, workspace: Workspace | None = None, stream=None):
+    """Returns (dX, {dAg, dBg, dAu, dBu, dAd, dBd}) for the block input X."""
+    N, d = X.shape
+    _need(X, "X", BF16, (N, w.d))
+    _need(gamma, "gamma", BF16, (w.d,))
+    _need(dOut, "dOut", BF16, (N, d))
+    w.validate()
+    shape = w.shape(N)
+    _, bws, _ = _lib.block_sizes(shape)
+    dev = X.device
+    dX = torch.empty((N, d), dtype=BF16, device=dev) if dX is None else _need(dX, "dX", BF16, (N, d))
+    if grads is None:
+        grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    gs = _lib.Grads(*[grads[k].data_ptr() for k in _lib.GRAD_FIELDS])
+    ws = (workspace or Workspace()).get(bws, dev)
+    _lib.check(_lib.block_backward(shape, w.c_struct(), _p(gamma), _p(X), _p(saved.g), _p(saved.u),
+                                   _p(saved.lowrank), _p(dOut), _p(dX), gs, _p(ws), ws.numel(), _stream(stream)),
+               "lora_mlp_block_backward")
+    return dX, grads
+
+
+class LoRAMLPBlockFunction(torch.autograd.Function):
+    """autograd wrapper of the pre-norm block: out = MLP(RMSNorm(X) * gamma).
+    Usage: LoRAMLPBlockFunction.apply(X, w, gamma, eps, Ag, Bg, Au, Bu, Ad, Bd)
+    (gamma frozen: no gradient)."""
+
+    @staticmethod
+    def forward(ctx, X, w: MLPWeights, gamma, eps, Ag, Bg, Au, Bu, Ad, Bd):
+        out, saved = block_forward(X.contiguous(), w, gamma, eps)
+        ctx.w, ctx.gamma, ctx.saved_lr = w, gamma, saved
+        ctx.save_for_backward(X)
+        return out
+
+    @staticmethod
+    def backward(ctx, dOut):
+        (X,) = ctx.saved_tensors
+        dX, g = block_backward(X, ctx.w, ctx.gamma, ctx.saved_lr, dOut.contiguous())
+        return dX, None, None, None, g["dAg"], g["dBg"], g["dAu"], g["dBu"], g["dAd"], g["dBd"]

@@ -30,7 +30,9 @@
 
 #include "lora_mlp.h"
 #include "lora_linear.h"
+#include "lora_rmsnorm.h"
 #include "aux_kernels.cuh"
+#include "rmsnorm.cuh"
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
 #include "umma2_gemm.cuh"
@@ -1253,6 +1255,181 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L4_dA", ctr)));
     }
     return LORA_MLP_OK;
+}
+
+}  // extern "C"
+
+// ============================================================================= pre-norm block
+//
+// out = MLP(RMSNorm(X)): one norm launch, then the MLP's launches on the
+// normalised rows.  Backward: the normalised rows are recomputed from X and
+// the saved rstd (the same kernel and arithmetic as the forward, so the same
+// bits), the MLP backward runs on them, and one launch maps its dX through
+// the norm's backward.
+
+namespace {
+
+// Rows of up to 16384 (forward) / 8192 (backward) elements run one row per
+// 128-thread CTA with the row in registers; wider rows fall back to the
+// warp-per-row loop kernels.
+int launch_rmsnorm_fwd(int64_t N, int64_t d, float eps, const void* x, const void* gamma, const float* rstd_in,
+                       float* rstd_out, void* y, int sms, cudaStream_t st) {
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* gb = static_cast<const __nv_bfloat16*>(gamma);
+    auto* yb = static_cast<__nv_bfloat16*>(y);
+    const int di = static_cast<int>(d);
+    const int64_t nch = (d / 8 + kRowThreads - 1) / kRowThreads;  // 8-element chunks per thread
+    const long long cap = static_cast<long long>(sms) * 16;
+    const dim3 rgrid(static_cast<unsigned>(N < cap ? N : cap)), rblock(kRowThreads);
+    long long wblocks = (N + kRmsWarps - 1) / kRmsWarps;
+    if (wblocks > static_cast<long long>(sms) * 8) wblocks = static_cast<long long>(sms) * 8;
+    {
+        LaunchScope scope("rmsnorm_fwd", st);
+        if (nch <= 2) rmsnorm_fwd_row_kernel<2><<<rgrid, rblock, 0, st>>>(xb, gb, N, di, eps, rstd_in, rstd_out, yb);
+        else if (nch <= 4)
+            rmsnorm_fwd_row_kernel<4><<<rgrid, rblock, 0, st>>>(xb, gb, N, di, eps, rstd_in, rstd_out, yb);
+        else if (nch <= 8)
+            rmsnorm_fwd_row_kernel<8><<<rgrid, rblock, 0, st>>>(xb, gb, N, di, eps, rstd_in, rstd_out, yb);
+        else if (nch <= 16)
+            rmsnorm_fwd_row_kernel<16><<<rgrid, rblock, 0, st>>>(xb, gb, N, di, eps, rstd_in, rstd_out, yb);
+        else
+            rmsnorm_fwd_kernel<<<static_cast<unsigned>(wblocks), kRmsWarps * 32, 0, st>>>(xb, gb, N, di, eps,
+                                                                                        rstd_in, rstd_out, yb);
+    }
+    return last_launch_error();
+}
+
+int launch_rmsnorm_bwd(int64_t N, int64_t d, const void* x, const void* gamma, const float* rstd, const void* dy,
+                       void* dx, int sms, cudaStream_t st) {
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* gb = static_cast<const __nv_bfloat16*>(gamma);
+    const auto* db = static_cast<const __nv_bfloat16*>(dy);
+    auto* ob = static_cast<__nv_bfloat16*>(dx);
+    const int di = static_cast<int>(d);
+    const int64_t nch = (d / 8 + kRowThreads - 1) / kRowThreads;
+    const long long cap = static_cast<long long>(sms) * 16;
+    const dim3 rgrid(static_cast<unsigned>(N < cap ? N : cap)), rblock(kRowThreads);
+    long long wblocks = (N + kRmsWarps - 1) / kRmsWarps;
+    if (wblocks > static_cast<long long>(sms) * 8) wblocks = static_cast<long long>(sms) * 8;
+    {
+        LaunchScope scope("rmsnorm_bwd", st);
+        if (nch <= 2) rmsnorm_bwd_row_kernel<2><<<rgrid, rblock, 0, st>>>(xb, gb, rstd, db, N, di, ob);
+        else if (nch <= 4) rmsnorm_bwd_row_kernel<4><<<rgrid, rblock, 0, st>>>(xb, gb, rstd, db, N, di, ob);
+        else if (nch <= 8) rmsnorm_bwd_row_kernel<8><<<rgrid, rblock, 0, st>>>(xb, gb, rstd, db, N, di, ob);
+        else
+            rmsnorm_bwd_kernel<<<static_cast<unsigned>(wblocks), kRmsWarps * 32, 0, st>>>(xb, gb, rstd, db, N, di,
+                                                                                        ob);
+    }
+    return last_launch_error();
+}
+
+int validate_norm(int64_t N, int64_t d) {
+    if (N < 1 || d < 1) return LORA_MLP_ERR_INVALID_ARG;
+    if (d % 8) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    const int64_t lim = (int64_t{1} << 31) - 1;
+    if (N > lim || d > lim) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    return LORA_MLP_OK;
+}
+
+// Workspace / saved layout of the block (offsets in bytes).
+struct BlockPlan {
+    size_t xn, dxn, mlp_f, mlp_b, f_total, b_total;
+    size_t s_mlp, s_rstd, s_total;
+};
+
+BlockPlan make_block_plan(const lora_mlp_shape& sh) {
+    const Plan pl = make_plan(sh);
+    BlockPlan b{};
+    const size_t xbytes = static_cast<size_t>(sh.N) * static_cast<size_t>(sh.d) * 2;
+    Carver f;
+    b.xn = f.take(xbytes);
+    b.mlp_f = f.take(pl.f_total);
+    b.f_total = f.off;
+    Carver k;
+    k.take(xbytes);  // xn at offset 0 in both workspaces
+    b.dxn = k.take(xbytes);
+    b.mlp_b = k.take(pl.b_total);
+    b.b_total = k.off;
+    Carver sv;
+    b.s_mlp = sv.take(pl.s_total);
+    b.s_rstd = sv.take(static_cast<size_t>(sh.N) * sizeof(float));
+    b.s_total = sv.off;
+    return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lora_rmsnorm_forward(int64_t N, int64_t d, float eps, const void* x, const void* gamma, void* y, void* rstd,
+                         void* stream) {
+    LMLP_TRY(validate_norm(N, d));
+    if (!std::isfinite(eps) || eps < 0.0f) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_ptrs({x, gamma, y, rstd}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return launch_rmsnorm_fwd(N, d, eps, x, gamma, nullptr, static_cast<float*>(rstd), y, di.sms,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int lora_rmsnorm_backward(int64_t N, int64_t d, const void* x, const void* gamma, const void* rstd, const void* dy,
+                          void* dx, void* stream) {
+    LMLP_TRY(validate_norm(N, d));
+    LMLP_TRY(check_ptrs({x, gamma, rstd, dy, dx}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return launch_rmsnorm_bwd(N, d, x, gamma, static_cast<const float*>(rstd), dy, dx, di.sms,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int lora_mlp_block_sizes(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes, size_t* bwd_workspace_bytes,
+                         size_t* saved_bytes) {
+    LMLP_TRY(validate_shape(shape));
+    const BlockPlan b = make_block_plan(*shape);
+    if (fwd_workspace_bytes) *fwd_workspace_bytes = b.f_total;
+    if (bwd_workspace_bytes) *bwd_workspace_bytes = b.b_total;
+    if (saved_bytes) *saved_bytes = b.s_total;
+    return LORA_MLP_OK;
+}
+
+int lora_mlp_block_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* gamma, float eps,
+                           const void* X, void* out, void* g, void* u, void* saved, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    LMLP_TRY(check_weights(shape, w));
+    if (!std::isfinite(eps) || eps < 0.0f) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_ptrs({gamma, X, out, g, u, saved, workspace}));
+    const BlockPlan b = make_block_plan(*shape);
+    if (workspace_bytes < b.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* sv = static_cast<uint8_t*>(saved);
+    LMLP_TRY(launch_rmsnorm_fwd(shape->N, shape->d, eps, X, gamma, nullptr, reinterpret_cast<float*>(sv + b.s_rstd),
+                                ws + b.xn, di.sms, st));
+    return lora_mlp_forward(shape, w, ws + b.xn, out, g, u, sv + b.s_mlp, ws + b.mlp_f, b.f_total - b.mlp_f,
+                            stream);
+}
+
+int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* gamma, const void* X,
+                            const void* g, const void* u, const void* saved, const void* dOut, void* dX,
+                            const lora_mlp_grads* grads, void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    LMLP_TRY(check_weights(shape, w));
+    LMLP_TRY(check_ptrs({gamma, X, g, u, saved, dOut, dX, workspace}));
+    const BlockPlan b = make_block_plan(*shape);
+    if (workspace_bytes < b.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    const float* rstd = reinterpret_cast<const float*>(sv + b.s_rstd);
+    LMLP_TRY(launch_rmsnorm_fwd(shape->N, shape->d, 0.0f, X, gamma, rstd, nullptr, ws + b.xn, di.sms, st));
+    LMLP_TRY(lora_mlp_backward(shape, w, ws + b.xn, g, u, sv + b.s_mlp, dOut, ws + b.dxn, grads, ws + b.mlp_b,
+                               b.b_total - b.mlp_b, stream));
+    return launch_rmsnorm_bwd(shape->N, shape->d, X, gamma, rstd, ws + b.dxn, dX, di.sms, st);
 }
 
 }  // extern "C"

@@ -232,3 +232,7 @@ def make_block_inputs(cfg: Config) -> dict:
     out["X"] = f32_to_bf16_bits(bf16_bits_to_f32(out["X"]) * scale)
     out["gamma"] = f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=cfg.d).astype(np.float32))
     return out
+
+
+# The block workloads: a name for the pre-norm block on an MLP workload's shapes.
+BLOCK_BY_NAME = {"llama3_8b_block": BY_NAME["llama3_8b_mlp"]}

@@ -11,7 +11,7 @@ from lora_fine_tuning_mlp_b200 import _lib
 from lora_fine_tuning_mlp_b200 import build as libbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADERS = [os.path.join(ROOT, "include", h) for h in ("lora_mlp.h", "lora_linear.h")]
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("lora_mlp.h", "lora_linear.h", "lora_rmsnorm.h")]
 
 
 @pytest.fixture(scope="module")
@@ -23,7 +23,7 @@ def L():
 def header_symbols():
     text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(lora_(?:mlp|linear)_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(lora_(?:mlp|linear|rmsnorm)_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_symbols():
@@ -191,3 +191,35 @@ def test_linear_argument_errors(L):
         == _lib.ERR_MISALIGNED
     assert _lib.lin_backward(sh, w, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bws - 1, None) \
         == _lib.ERR_WORKSPACE_TOO_SMALL
+
+
+# ----------------------------------------------------------------------------- RMSNorm and the block
+
+
+def test_block_sizes_add_the_norm_buffers(L):
+    sh = shape()
+    f, b, s = _lib.sizes(sh)
+    bf, bb, bs = _lib.block_sizes(sh)
+    assert bf >= f + 512 * 256 * 2          # the normalised rows
+    assert bb >= b + 2 * 512 * 256 * 2      # normalised rows and their gradient
+    assert bs >= s + 512 * 4                # rstd
+
+
+def test_norm_and_block_argument_errors(L):
+    assert _lib.rmsnorm_forward(0, 64, 1e-5, FAKE, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.rmsnorm_forward(4, 60, 1e-5, FAKE, FAKE, FAKE, FAKE, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _lib.rmsnorm_forward(4, 64, -1.0, FAKE, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.rmsnorm_forward(4, 64, float("nan"), FAKE, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.rmsnorm_forward(4, 64, 1e-5, FAKE, None, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.rmsnorm_backward(4, 64, FAKE, FAKE, FAKE + 4, FAKE, FAKE, None) == _lib.ERR_MISALIGNED
+    sh = shape()
+    bf, bb, _ = _lib.block_sizes(sh)
+    assert _lib.block_forward(sh, weights(), FAKE, 1e-5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bf - 1, None) \
+        == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.block_forward(sh, weights(), None, 1e-5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bf, None) \
+        == _lib.ERR_INVALID_ARG
+    g = _lib.Grads(*([FAKE] * 6))
+    assert _lib.block_backward(sh, weights(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, g, FAKE, bb - 1, None) \
+        == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.block_backward(sh, weights(), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, g, FAKE, bb, None) \
+        == _lib.ERR_INVALID_ARG
