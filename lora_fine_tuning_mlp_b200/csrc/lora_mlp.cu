@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -255,6 +256,32 @@ struct GemmBuilder {
         p->ld_tr = ld_tr;
         p->tr_split = tr_split;
         p->counters = reinterpret_cast<int*>(1);  // placeholder: assigned in finish()
+    }
+    // Processing order by feature band: unit u of problem p gets the key
+    // feat_of(p, tile, kb0, kb1) (the feature coordinate of the data it reads);
+    // units are taken in increasing key order (ties: launch order).  Called
+    // after finish().  Only for launches whose problems all have tiles_n == 1.
+    template <class KeyFn>
+    void order_units(KeyFn feat_of) {
+        if (units > kMaxPerm || units > 65535) return;
+        std::vector<std::pair<long long, int>> key(static_cast<size_t>(units));
+        for (int i = 0; i < a.nprobs; ++i) {
+            const Prob& p = a.prob[i];
+            if (p.tiles_n != 1) return;
+            const int n = p.tiles_m * p.splits;
+            for (int lu = 0; lu < n; ++lu) {
+                const int tile = lu / p.splits, ks = lu - tile * p.splits;
+                const int kb0 = static_cast<int>((static_cast<long long>(ks) * p.nkb) / p.splits);
+                const int kb1 = static_cast<int>((static_cast<long long>(ks + 1) * p.nkb) / p.splits);
+                key[static_cast<size_t>(p.unit0 + lu)] = {feat_of(i, tile, kb0, kb1), p.unit0 + lu};
+            }
+        }
+        std::stable_sort(key.begin(), key.end(),
+                         [](const std::pair<long long, int>& x, const std::pair<long long, int>& y) {
+                             return x.first < y.first;
+                         });
+        for (int i = 0; i < units; ++i) a.perm[i] = static_cast<uint16_t>(key[static_cast<size_t>(i)].second);
+        a.nperm = units;
     }
     void finish(int* counters) {
         int u = 0, c = 0;
@@ -899,6 +926,15 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         pbu->ld = r;
         pbu->split_stride = dff * r;
         b.fin(pbu, 1.0f, static_cast<int>(r), grads->dBu, r, nullptr, nullptr, 0, static_cast<int>(r));
+        // dg and du are read twice here (K-major for T, MN-major for dB) and
+        // are larger than L2 together.  Taking the units in order of the
+        // hidden features they read puts both reads of each feature band in
+        // the same round, so the second one is served from L2.
+        b.finish(ctr);
+        b.order_units([](int prob, int tile, int kb0, int kb1) -> long long {
+            return prob < 2 ? static_cast<long long>(kb0 + kb1) * (kBK / 2)    // T: K runs over features
+                            : static_cast<long long>(tile) * kBM + kBM / 2;   // dAd, dB: M runs over features
+        });
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B_mid_lowrank_grads", ctr)));
     }
     LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 0, di.sms, st, &W[0]));

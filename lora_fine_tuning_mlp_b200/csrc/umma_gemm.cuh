@@ -43,6 +43,7 @@ constexpr int kMaxSegs = 4;
 constexpr int kMaxProbs = 5;
 constexpr int kMaxStages = 12;
 constexpr int kGemmThreads = 192;
+constexpr int kMaxPerm = 2048;  // units a launch can reorder (see GemmArgs::perm)
 
 struct Seg {
     int a_map;
@@ -91,6 +92,11 @@ struct alignas(64) GemmArgs {
     long long wait_limit;  // SM cycles a barrier wait may spin before the kernel gives up
     int force_timeout;     // test hook: the epilogue waits on a barrier nothing signals
     int nmaps;             // maps[0, nmaps) are encoded
+    // Optional processing order: with nperm == total_units, the i-th unit
+    // taken by the persistent grid is perm[i].  Lets a launch group the units
+    // that read the same data into the same round, so the second read hits L2.
+    int nperm;
+    uint16_t perm[kMaxPerm];
 };
 
 struct Unit {
@@ -98,6 +104,7 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+    if (a.nperm > 0) u = a.perm[u];
     Unit r;
     r.p = 0;
     for (int i = 1; i < a.nprobs; ++i)
