@@ -56,17 +56,30 @@ def load_peaks():
 
 
 def csrc_sha256() -> str:
-    """Hash of the CUDA sources, to tell whether a stored ncu figure still applies."""
+    """Hash of the translation unit the GEMM kernels are built from (lora_mlp.cu
+    and every local file it includes, transitively), to tell whether a stored
+    ncu figure still applies to the kernels this build runs."""
     import hashlib
-    d = os.path.join(ROOT, "lora_fine_tuning_mlp_b200", "csrc")
+    import re as _re
+    csrc = os.path.join(ROOT, "lora_fine_tuning_mlp_b200", "csrc")
+    inc = os.path.join(ROOT, "include")
+    seen, todo = [], ["lora_mlp.cu"]
+    while todo:
+        f = todo.pop(0)
+        if f in seen:
+            continue
+        path = next((os.path.join(dd, f) for dd in (csrc, inc) if os.path.exists(os.path.join(dd, f))), None)
+        if path is None:
+            continue
+        seen.append(f)
+        with open(path, "rb") as fh:
+            text = fh.read()
+        todo += [m.decode() for m in _re.findall(rb'#include\s+"([^"]+)"', text)]
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
-    for hdr in ("lora_mlp.h", "lora_linear.h"):
-        with open(os.path.join(ROOT, "include", hdr), "rb") as fh:
+    for f in sorted(seen):
+        path = next(os.path.join(dd, f) for dd in (csrc, inc) if os.path.exists(os.path.join(dd, f)))
+        h.update(f.encode())
+        with open(path, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
@@ -527,8 +540,7 @@ def linear_reference_arm(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": linear_config_dict(cfg),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
-                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle"
-                                   + (", pre-norm block" if block else "") + ")"},
+                         "sample": f"{n} tokens of the {cfg.name} shapes per step (numpy fp64 oracle)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "lora_mlp.cu"), os.path.join(CSRC, "noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "epilogue.cuh", "umma_gemm.cuh", "umma2_gemm.cuh", "aux_kernels.cuh")] + [
-    os.path.join(ROOT, "include", "lora_mlp.h")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cuh")] + [
+    os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include"))) if f.endswith(".h")]
 OUT = os.path.join(HERE, "liblora_mlp.so")
 
 

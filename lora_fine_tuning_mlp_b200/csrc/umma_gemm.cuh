@@ -228,6 +228,11 @@ __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_b
     }
 }
 
+// The MMA issuer (one thread).  The rank-r products are tall and skinny: a
+// K block's UMMAs take the tensor core only 16-64 cycles, so this loop, not
+// the tensor core, sets how fast a CTA can consume its stages.  It is kept
+// short: segments are walked directly (only a segment's last block can be
+// partial) and each stage's descriptors are those of stage 0 plus an offset.
 template <int NACC>
 __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
                                          uint32_t tmem_base, const SmemCtl& c) {
@@ -236,6 +241,9 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
     int abuf = 0;
     uint32_t aphase = 0;
     const uint32_t acc_cols = NACC * a.bn;
+    // bytes >> 4 per stage in the descriptors' 14-bit address field (shared
+    // memory is < 256 KB, so adding offsets never carries out of the field)
+    const uint32_t sstep = stage_bytes >> 4;
     for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
         const Unit t = decode_unit(a, u);
         const Prob& P = a.prob[t.p];
@@ -246,57 +254,55 @@ __device__ __forceinline__ void mma_loop(const GemmArgs& a, uint32_t smem_base, 
         // (A is read from smem once instead of twice).
         const bool pair_ok = NACC == 2 && !b_mn && 2 * a.bn <= 256;
         const uint32_t idesc_pair = idesc_bf16(static_cast<uint32_t>(2 * a.bn), a_mn, b_mn);
+        // Stage-0 descriptors; the next 16-wide K slice is 32 B further along
+        // a K-major tile and 2048 B (16 rows of 128 B) along an MN-major one.
+        const uint64_t a0 = a_mn ? sw128_desc(smem_base, 8192u, 1024u) : sw128_desc(smem_base, 16u, 1024u);
+        const uint32_t astep = a_mn ? (2048u >> 4) : (32u >> 4);
+        const uint32_t bstep = b_mn ? (2048u >> 4) : (32u >> 4);
+        uint64_t b0[NACC];
+#pragma unroll
+        for (int acc = 0; acc < NACC; ++acc) {
+            const uint32_t sB = smem_base + kATileBytes + acc * a.b_bytes;
+            b0[acc] = b_mn ? sw128_desc(sB, 8192u, 1024u) : sw128_desc(sB, 16u, 1024u);
+        }
         if (!wait_or_abort(c.acce + 8u * abuf, aphase ^ 1u, c)) return;
         tc_fence_after();
         uint32_t started = 0;
-        int seg = 0, seg_kb0 = 0;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
-                seg_kb0 += P.seg[seg].kblocks;
-                ++seg;
-            }
-            const Seg& S = P.seg[seg];
-            const int k0 = (kb - seg_kb0) * kBK;
-            const int kvalid = min(kBK, S.k_len - k0);
-            const int nk = (kvalid + 15) >> 4;
-            if (!wait_or_abort(c.full + 8u * stage, phase, c)) return;
-            tc_fence_after();
-            const uint32_t sA = smem_base + stage * stage_bytes;
-            if (pair_ok && S.b_map[0] >= 0 && S.b_map[1] >= 0 && (started == 0u || started == 3u)) {
-                const uint32_t sB = sA + kATileBytes;
-                const uint32_t d = tmem_base + abuf * acc_cols;
-                for (int k = 0; k < nk; ++k) {
-                    const uint64_t ad = a_mn ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
-                                             : sw128_desc(sA + 32u * k, 16u, 1024u);
-                    const uint64_t bd = sw128_desc(sB + 32u * k, 16u, 1024u);
-                    umma_bf16(d, ad, bd, idesc_pair, (started & 1u) | (k > 0 ? 1u : 0u));
+        int seg_kb0 = 0;
+        for (int sg = 0; sg < P.nsegs; ++sg) {
+            const Seg& S = P.seg[sg];
+            const int nkb = S.kblocks;
+            const int lo = max(t.kb0 - seg_kb0, 0), hi = min(t.kb1 - seg_kb0, nkb);
+            seg_kb0 += nkb;
+            for (int kb = lo; kb < hi; ++kb) {
+                const int nk = kb == nkb - 1 ? ((S.k_len - kb * kBK + 15) >> 4) : 4;
+                if (!wait_or_abort(c.full + 8u * stage, phase, c)) return;
+                tc_fence_after();
+                const uint32_t so = stage * sstep;
+                const uint64_t ad = a0 + so;
+                if (pair_ok && S.b_map[0] >= 0 && S.b_map[1] >= 0 && (started == 0u || started == 3u)) {
+                    const uint64_t bd = b0[0] + so;
+                    const uint32_t d = tmem_base + abuf * acc_cols;
+                    for (int k = 0; k < nk; ++k)
+                        umma_bf16(d, ad + k * astep, bd + k * bstep, idesc_pair, (started & 1u) | (k > 0 ? 1u : 0u));
+                    started = 3u;
+                } else {
+#pragma unroll
+                    for (int acc = 0; acc < NACC; ++acc) {
+                        if (S.b_map[acc] < 0) continue;
+                        const uint64_t bd = b0[acc] + so;
+                        const uint32_t d = tmem_base + abuf * acc_cols + acc * a.bn;
+                        for (int k = 0; k < nk; ++k)
+                            umma_bf16(d, ad + k * astep, bd + k * bstep, idesc,
+                                      ((started >> acc) & 1u) | (k > 0 ? 1u : 0u));
+                        started |= 1u << acc;
+                    }
                 }
-                started = 3u;
                 umma_commit(c.empty + 8u * stage);
                 if (++stage == a.stages) {
                     stage = 0;
                     phase ^= 1u;
                 }
-                continue;
-            }
-#pragma unroll
-            for (int acc = 0; acc < NACC; ++acc) {
-                if (S.b_map[acc] < 0) continue;
-                const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
-                const uint32_t d = tmem_base + abuf * acc_cols + acc * a.bn;
-                for (int k = 0; k < nk; ++k) {
-                    const uint64_t ad = a_mn ? sw128_desc(sA + 2048u * k, 8192u, 1024u)
-                                             : sw128_desc(sA + 32u * k, 16u, 1024u);
-                    const uint64_t bd = b_mn ? sw128_desc(sB + 2048u * k, 8192u, 1024u)
-                                             : sw128_desc(sB + 32u * k, 16u, 1024u);
-                    umma_bf16(d, ad, bd, idesc, ((started >> acc) & 1u) | (k > 0 ? 1u : 0u));
-                }
-                started |= 1u << acc;
-            }
-            umma_commit(c.empty + 8u * stage);
-            if (++stage == a.stages) {
-                stage = 0;
-                phase ^= 1u;
             }
         }
         umma_commit(c.accf + 8u * abuf);
