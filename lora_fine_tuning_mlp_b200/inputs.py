@@ -16,6 +16,9 @@ order, each drawn in float32 and rounded to bf16 with round-to-nearest-even):
   A ~ U(-1/sqrt(fan_in), +1/sqrt(fan_in)), fan_in = d for Ag, Au and d_ff for Ad
   B ~ N(0, 0.02^2)  (std 0.02, non-zero so that every adapter gradient is exercised)
   dOut ~ N(0, 1)
+
+The LoRA linear, pre-norm block and cross-entropy workloads further down
+state their own recipes.
 """
 from __future__ import annotations
 
@@ -236,3 +239,77 @@ def make_block_inputs(cfg: Config) -> dict:
 
 # The block workloads: a name for the pre-norm block on an MLP workload's shapes.
 BLOCK_BY_NAME = {"llama3_8b_block": BY_NAME["llama3_8b_mlp"]}
+
+
+# ----------------------------------------------------------------------------- cross-entropy
+
+CE_IGNORE_INDEX = -100
+
+
+@dataclasses.dataclass(frozen=True)
+class CEConfig:
+    """Cross-entropy over a vocabulary of V logits per token.
+
+    logit_scale multiplies the logits (Cohere's logit scaling); softcap > 0
+    applies c * tanh(t / c) after it (Gemma 2's final-logit softcapping).
+    The raw logits are drawn with std `z_std`."""
+    name: str
+    N: int
+    V: int
+    logit_scale: float = 1.0
+    softcap: float = 0.0
+    z_std: float = 2.0
+    ignore_frac: float = 0.03
+    index: int = 70
+
+    @property
+    def seed(self) -> int:
+        return 1234 + self.index
+
+    def bytes_fwd(self) -> int:
+        """Algorithmic HBM bytes of the forward: the logits read once."""
+        return 2 * self.N * self.V
+
+    def bytes_bwd(self) -> int:
+        """Backward: the logits read once, their gradient written once."""
+        return 4 * self.N * self.V
+
+
+CE_CONFIGS = (
+    CEConfig("ce_tiny", 37, 1003, 1.0, 0.0, index=70),
+    CEConfig("ce_tiny_softcap", 45, 2051, 1.0, 30.0, z_std=10.0, index=71),
+    CEConfig("ce_tiny_scale", 29, 777, 0.0625, 0.0, z_std=32.0, index=72),
+    CEConfig("gemma2_256k_ce", 4096, 256000, 1.0, 30.0, z_std=10.0, index=73),
+    CEConfig("cohere_256k_ce", 4096, 256000, 0.0625, 0.0, z_std=32.0, index=74),
+    CEConfig("llama3_128k_ce", 4096, 128256, 1.0, 0.0, index=75),
+)
+CE_BY_NAME = {c.name: c for c in CE_CONFIGS}
+
+
+def custom_ce(N, V, logit_scale=1.0, softcap=0.0, z_std=2.0, ignore_frac=0.03, seed_index=80,
+              name="custom_ce") -> CEConfig:
+    return CEConfig(name, N, V, logit_scale, softcap, z_std, ignore_frac, seed_index)
+
+
+def make_ce_inputs(cfg: CEConfig) -> dict:
+    """logits [N, V] bf16 bits ~ N(0, z_std^2) rounded to bf16; labels [N]
+    int64 uniform in [0, V), a fraction ignore_frac of them replaced by
+    CE_IGNORE_INDEX; dloss [N] float32 ~ U(0.5, 1.5) / N (a per-row upstream
+    gradient that is not uniform, so a row mix-up shows).  One PCG64
+    generator, seed 1234 + index, drawn in this order; the logits are drawn
+    and rounded in blocks of rows so the float32 copy of a 256K vocabulary
+    never exists whole."""
+    rng = np.random.Generator(np.random.PCG64(cfg.seed))
+    N, V = cfg.N, cfg.V
+    z = np.empty((N, V), dtype=np.uint16)
+    step = max(1, (1 << 24) // V)
+    for r0 in range(0, N, step):
+        r1 = min(N, r0 + step)
+        blk = rng.standard_normal((r1 - r0, V), dtype=np.float32)
+        blk *= np.float32(cfg.z_std)
+        z[r0:r1] = f32_to_bf16_bits(blk)
+    labels = rng.integers(0, V, size=N, dtype=np.int64)
+    ignore = rng.random(N) < cfg.ignore_frac
+    labels[ignore] = CE_IGNORE_INDEX
+    dloss = (rng.uniform(0.5, 1.5, size=N) / N).astype(np.float32)
+    return {"logits": z, "labels": labels, "dloss": dloss}

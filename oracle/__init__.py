@@ -17,3 +17,4 @@ from .lora_mlp import (  # noqa: F401
 )
 from . import lora_linear  # noqa: F401,E402
 from . import rmsnorm  # noqa: F401,E402
+from . import cross_entropy  # noqa: F401,E402
