@@ -41,6 +41,7 @@ from lora_fine_tuning_mlp_b200 import inputs as synth  # noqa: E402
 
 METRIC = "fused LoRA-SwiGLU MLP fwd+bwd tokens/s and TFLOP/s vs bf16 dense peak"
 LINEAR_METRIC = "fused LoRA linear fwd+bwd tokens/s and TFLOP/s vs bf16 dense peak"
+CE_METRIC = "chunked cross-entropy fwd+bwd tokens/s and GB/s vs HBM bandwidth"
 DEFAULT_WORKLOAD = "llama3_8b_mlp"
 SUSTAINED_MS = 2000.0  # timed regions at least this long are held to the sustained (power-capped) peak
 
@@ -706,6 +707,192 @@ def linear_arm(args, cfg):
     return 0
 
 
+# ----------------------------------------------------------------------------- cross-entropy legs
+
+
+def ce_config_dict(cfg):
+    return {"workload": cfg.name, "N_tokens": cfg.N, "V": cfg.V, "logit_scale": cfg.logit_scale,
+            "softcap": cfg.softcap, "ignore_index": synth.CE_IGNORE_INDEX, "ignore_frac": cfg.ignore_frac,
+            "l2": "no flush: logits %.1f GB > 126 MB L2" % (2 * cfg.N * cfg.V / 1e9), "parallelism": "replicas"}
+
+
+def time_ce_oracle(cfg, budget_s: float, inp):
+    """Rows of the workload the fp64 oracle handles in about budget_s (forward
+    + backward).  Returns (rows, run(idx) -> seconds)."""
+    from oracle import cross_entropy as oce
+
+    def run(idx):
+        t0 = time.perf_counter()
+        z = oce.bf16_to_f64(inp["logits"][idx])
+        lab = inp["labels"][idx]
+        _, lse = oce.forward(z, lab, cfg.logit_scale, cfg.softcap, synth.CE_IGNORE_INDEX)
+        oce.backward(z, lab, lse, inp["dloss"][idx], cfg.logit_scale, cfg.softcap, synth.CE_IGNORE_INDEX)
+        return time.perf_counter() - t0
+
+    t_probe = run(np.arange(2))
+    n = max(2, min(cfg.N, int(2 * budget_s / max(t_probe, 1e-3))))
+    return n, run
+
+
+def ce_reference_arm(args, cfg):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    inp = synth.make_ce_inputs(cfg)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    n, run = time_ce_oracle(cfg, per_step, inp)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = run((np.arange(n) + i * n) % cfg.N)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total
+    line = {
+        "impl": "reference", "metric": CE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": ce_config_dict(cfg),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
+                         "sample": f"{n} rows of the {cfg.name} logits per step (numpy fp64 oracle)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ce_arm(args, cfg):
+    """One step = cross-entropy forward (chunk partials + row combine) and
+    backward over N rows of V logits, the gradient written to its own buffer
+    so that every step sees the same logits.  The logits (2 GB on the 256K
+    workloads) are far larger than L2."""
+    import torch
+    import torch.distributed as dist
+
+    from lora_fine_tuning_mlp_b200 import _lib, api, replicas
+
+    rank, local, world = replicas.world()
+    if world > 1:
+        torch.cuda.set_device(local)
+        replicas.init("nccl", device=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _lib.lib()
+    inp = synth.make_ce_inputs(cfg)
+    N, V = cfg.N, cfg.V
+    ld = (V + 7) // 8 * 8
+    host = torch.zeros((N, ld), dtype=torch.int16)
+    host[:, :V] = torch.from_numpy(inp["logits"].view(np.int16))
+    zfull = host.view(torch.bfloat16).to(dev)
+    z = zfull[:, :V]
+    lab = torch.from_numpy(inp["labels"]).to(dev)
+    dl = torch.from_numpy(inp["dloss"]).to(dev)
+    dz = torch.empty_strided(z.size(), z.stride(), dtype=torch.bfloat16, device=dev)
+    ws = api.Workspace()
+    kw = dict(logit_scale=cfg.logit_scale, softcap=cfg.softcap, ignore_index=synth.CE_IGNORE_INDEX)
+    stream = torch.cuda.current_stream()
+    barrier = replicas.barrier
+
+    def step(x=z):
+        _, lse = api.ce_forward(x, lab, workspace=ws, **kw)
+        api.ce_backward(x, lab, lse, dl, out=dz, **kw)
+
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return replicas.max_over_ranks(a.elapsed_time(b), device=dev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = _lib.launch_count()
+    w0 = time.monotonic()
+    ms_max = timed(step, args.steps)
+    w1 = time.monotonic()
+    launches = _lib.launch_count() - launches0
+    clocks = sampler.stop((w0, w1))
+
+    _lib.timing_enable(True)
+    _lib.timing_collect()
+    timed(step, args.steps)
+    recs = _lib.timing_collect()
+    _lib.timing_enable(False)
+
+    # end to end through the public API: the logits copied in from pinned host
+    # memory and the per-row losses copied back, every step
+    zh = host.view(torch.bfloat16).pin_memory()
+    lossh = torch.empty((N,), dtype=torch.float32, pin_memory=True)
+    zd = torch.empty_like(zfull)
+
+    def e2e_step():
+        zd.copy_(zh, non_blocking=True)
+        loss, lse = api.ce_forward(zd[:, :V], lab, workspace=ws, **kw)
+        api.ce_backward(zd[:, :V], lab, lse, dl, out=dz, **kw)
+        lossh.copy_(loss, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    ems = timed(e2e_step, e2e_steps)
+
+    per = {}
+    for name, kms in recs:
+        s_ = per.setdefault(name, [0.0, 0])
+        s_[0] += kms
+        s_[1] += 1
+    peaks = load_peaks()
+    algo = {"CE_fwd_chunks": cfg.bytes_fwd(), "CE_bwd": cfg.bytes_bwd()}
+    dom = max((k for k in per if k in algo), key=lambda k: per[k][0], default=None)
+    roof = None
+    if dom is not None:
+        avg_ms = per[dom][0] / per[dom][1]
+        achieved = algo[dom] / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks['source']} hbm_gbs (copy bandwidth)",
+                "bytes_per_launch": algo[dom], "avg_launch_ms": avg_ms}
+    barrier()
+    if rank == 0:
+        per_step = ms_max / args.steps
+        line = {
+            "metric": CE_METRIC, "value": replicas.job_throughput(N, args.steps, ms_max, world), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": ce_config_dict(cfg),
+            "gb_per_s": (cfg.bytes_fwd() + cfg.bytes_bwd()) / (per_step * 1e-3) / 1e9,
+            "roofline": roof,
+            "kernels_gb_per_s": {k: algo[k] / (v[0] / v[1] * 1e-3) / 1e9 for k, v in per.items() if k in algo},
+            "e2e": {"value": replicas.job_throughput(N, e2e_steps, ems, world), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(zfull.numel() * 2), "d2h_bytes_per_step": int(N * 4),
+                    "what": "per step: H2D of the logits from pinned host, forward + backward, D2H of the per-row "
+                            "losses"},
+            "gpu_launches": launches,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(per.items(), key=lambda kv: -kv[1][0])},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n, run = time_ce_oracle(cfg, args.cpu_budget, inp)
+            dt = run(np.arange(n))
+            line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": threads_used(), "kind": "oracle",
+                                    "sample": f"{n} rows of the {cfg.name} logits, numpy fp64 oracle, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -713,12 +900,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=("b200", "reference"))
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(synth.BY_NAME) + sorted(synth.LINEAR_BY_NAME) + sorted(synth.BLOCK_BY_NAME))
+                    choices=sorted(synth.BY_NAME) + sorted(synth.LINEAR_BY_NAME) + sorted(synth.BLOCK_BY_NAME)
+                    + sorted(synth.CE_BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload in synth.CE_BY_NAME:
+        cfg = synth.CE_BY_NAME[args.workload]
+        return ce_reference_arm(args, cfg) if args.impl == "reference" else ce_arm(args, cfg)
     if args.workload in synth.LINEAR_BY_NAME:
         cfg = synth.LINEAR_BY_NAME[args.workload]
         return linear_reference_arm(args, cfg) if args.impl == "reference" else linear_arm(args, cfg)

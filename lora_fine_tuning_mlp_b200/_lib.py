@@ -1,4 +1,4 @@
-"""ctypes binding of liblora_mlp.so (include/lora_mlp.h, lora_linear.h, lora_rmsnorm.h).
+"""ctypes binding of liblora_mlp.so (include/lora_mlp.h, lora_linear.h, lora_rmsnorm.h, lora_ce.h).
 
 Argument marshalling only: every step of the MLP runs in the library's CUDA
 kernels.  Loading fails loudly if the shared library has not been built.
@@ -27,7 +27,7 @@ WEIGHTS_INT4_B64 = 1
 WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Sg", "Su", "Sd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 
-# Every symbol include/lora_mlp.h, lora_linear.h and lora_rmsnorm.h declare.
+# Every symbol include/lora_mlp.h, lora_linear.h, lora_rmsnorm.h and lora_ce.h declare.
 SYMBOLS = (
     "lora_mlp_sizes",
     "lora_mlp_forward",
@@ -48,6 +48,10 @@ SYMBOLS = (
     "lora_mlp_block_sizes",
     "lora_mlp_block_forward",
     "lora_mlp_block_backward",
+    "lora_ce_sizes",
+    "lora_ce_forward",
+    "lora_ce_backward",
+    "lora_ce_device_status",
 )
 
 
@@ -71,6 +75,11 @@ class LinShape(ctypes.Structure):
 
 class LinWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W", "S", "A", "B")]
+
+
+class CEShape(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("V", ctypes.c_int64), ("ld", ctypes.c_int64),
+                ("logit_scale", ctypes.c_float), ("softcap", ctypes.c_float), ("ignore_index", ctypes.c_int64)]
 
 
 class KernelTime(ctypes.Structure):
@@ -129,6 +138,10 @@ def lib() -> ctypes.CDLL:
                                                  vp, vp, vp, vp, vp, vp, sz, vp]
             L.lora_mlp_block_backward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
                                                   vp, vp, vp, ctypes.POINTER(Grads), vp, sz, vp]
+            L.lora_ce_sizes.argtypes = [ctypes.POINTER(CEShape), ctypes.POINTER(sz)]
+            L.lora_ce_forward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, sz, vp]
+            L.lora_ce_backward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, vp]
+            L.lora_ce_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
@@ -136,7 +149,8 @@ def lib() -> ctypes.CDLL:
                          "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect",
                          "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward",
                          "lora_rmsnorm_forward", "lora_rmsnorm_backward", "lora_mlp_block_sizes",
-                         "lora_mlp_block_forward", "lora_mlp_block_backward"):
+                         "lora_mlp_block_forward", "lora_mlp_block_backward", "lora_ce_sizes",
+                         "lora_ce_forward", "lora_ce_backward", "lora_ce_device_status"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -259,3 +273,28 @@ def rmsnorm_forward(N, d, eps, x, gamma, y, rstd, stream) -> int:
 
 def rmsnorm_backward(N, d, x, gamma, rstd, dy, dx, stream) -> int:
     return lib().lora_rmsnorm_backward(int(N), int(d), x, gamma, rstd, dy, dx, stream)
+
+
+def make_ce_shape(N, V, ld=None, logit_scale=1.0, softcap=0.0, ignore_index=-100) -> CEShape:
+    return CEShape(int(N), int(V), int(V if ld is None else ld), float(logit_scale), float(softcap),
+                   int(ignore_index))
+
+
+def ce_sizes(shape: CEShape) -> int:
+    ws = ctypes.c_size_t()
+    check(lib().lora_ce_sizes(ctypes.byref(shape), ctypes.byref(ws)), "lora_ce_sizes")
+    return ws.value
+
+
+def ce_forward(shape: CEShape, logits, labels, loss, lse, workspace, workspace_bytes, stream) -> int:
+    return lib().lora_ce_forward(ctypes.byref(shape), logits, labels, loss, lse, workspace, workspace_bytes, stream)
+
+
+def ce_backward(shape: CEShape, logits, labels, lse, dloss, dlogits, stream) -> int:
+    return lib().lora_ce_backward(ctypes.byref(shape), logits, labels, lse, dloss, dlogits, stream)
+
+
+def ce_device_status(stream) -> int:
+    st = ctypes.c_int(0)
+    check(lib().lora_ce_device_status(stream, ctypes.byref(st)), "lora_ce_device_status")
+    return st.value

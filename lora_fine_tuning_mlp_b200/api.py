@@ -506,3 +506,81 @@ class LoRAMLPBlockFunction(torch.autograd.Function):
         (X,) = ctx.saved_tensors
         dX, g = block_backward(X, ctx.w, ctx.gamma, ctx.saved_lr, dOut.contiguous())
         return dX, None, None, None, g["dAg"], g["dBg"], g["dAu"], g["dBu"], g["dAd"], g["dBd"]
+
+
+# ----------------------------------------------------------------------------- chunked cross-entropy
+
+
+def _ce_shape(logits: torch.Tensor, logit_scale: float, softcap: float, ignore_index: int):
+    if logits.dim() != 2:
+        raise ValueError("logits must be [N, V]")
+    if logits.dtype != BF16 or not logits.is_cuda:
+        raise TypeError("logits must be a bf16 CUDA tensor")
+    if logits.stride(1) != 1:
+        raise ValueError("logits rows must be contiguous")
+    N, V = logits.shape
+    return _lib.make_ce_shape(N, V, logits.stride(0), logit_scale, softcap, ignore_index)
+
+
+def ce_forward(logits: torch.Tensor, labels: torch.Tensor, *, logit_scale: float = 1.0, softcap: float = 0.0,
+               ignore_index: int = -100, workspace: Workspace | None = None, stream=None):
+    """Per-row cross-entropy of bf16 logits [N, V] (row stride a multiple of
+    8) against int64 labels [N]: returns (loss [N] fp32, lse [N] fp32), loss 0
+    for rows labelled ignore_index."""
+    shape = _ce_shape(logits, logit_scale, softcap, ignore_index)
+    N = shape.N
+    _need(labels, "labels", torch.int64, (N,))
+    dev = logits.device
+    loss = torch.empty((N,), dtype=torch.float32, device=dev)
+    lse = torch.empty((N,), dtype=torch.float32, device=dev)
+    ws = (workspace or Workspace()).get(_lib.ce_sizes(shape), dev)
+    _lib.check(_lib.ce_forward(shape, _p(logits), _p(labels), _p(loss), _p(lse), _p(ws), ws.numel(),
+                               _stream(stream)), "lora_ce_forward")
+    return loss, lse
+
+
+def ce_backward(logits: torch.Tensor, labels: torch.Tensor, lse: torch.Tensor, dloss: torch.Tensor, *,
+                logit_scale: float = 1.0, softcap: float = 0.0, ignore_index: int = -100, out=None,
+                inplace: bool = False, stream=None):
+    """dlogits [N, V] bf16 for the per-row upstream gradient dloss [N] (fp32).
+    inplace=True writes the gradient over the logits."""
+    shape = _ce_shape(logits, logit_scale, softcap, ignore_index)
+    N = shape.N
+    _need(labels, "labels", torch.int64, (N,))
+    _need(lse, "lse", torch.float32, (N,))
+    _need(dloss, "dloss", torch.float32, (N,))
+    # The kernel writes the gradient with the logits' row stride, so the
+    # output keeps the logits' strides (empty_like would not for a padded view).
+    if inplace:
+        out = logits
+    elif out is None:
+        out = torch.empty_strided(logits.size(), logits.stride(), dtype=BF16, device=logits.device)
+    elif (out.shape != logits.shape or out.stride() != logits.stride() or out.dtype != BF16 or not out.is_cuda):
+        raise ValueError("out must have the logits' shape, strides and dtype")
+    _lib.check(_lib.ce_backward(shape, _p(logits), _p(labels), _p(lse), _p(dloss), _p(out), _stream(stream)),
+               "lora_ce_backward")
+    return out
+
+
+class CrossEntropyFunction(torch.autograd.Function):
+    """Mean cross-entropy over the rows whose label is not ignore_index, with
+    the library's chunked kernels.  Usage:
+    CrossEntropyFunction.apply(logits, labels, logit_scale, softcap, ignore_index).
+    The backward writes the logits' gradient over the logits (they are not
+    needed afterwards), as the pages' kernel does to save memory."""
+
+    @staticmethod
+    def forward(ctx, logits, labels, logit_scale=1.0, softcap=0.0, ignore_index=-100):
+        loss, lse = ce_forward(logits, labels, logit_scale=logit_scale, softcap=softcap, ignore_index=ignore_index)
+        n = (labels != ignore_index).sum().clamp_min(1).to(torch.float32)
+        ctx.save_for_backward(logits, labels, lse, n)
+        ctx.cfg = (logit_scale, softcap, ignore_index)
+        return loss.sum() / n
+
+    @staticmethod
+    def backward(ctx, g):
+        logits, labels, lse, n = ctx.saved_tensors
+        s, c, ign = ctx.cfg
+        dloss = (g.to(torch.float32) / n).expand(labels.shape[0]).contiguous()
+        dz = ce_backward(logits, labels, lse, dloss, logit_scale=s, softcap=c, ignore_index=ign, inplace=True)
+        return dz, None, None, None, None

@@ -32,7 +32,9 @@
 #include "lora_mlp.h"
 #include "lora_linear.h"
 #include "lora_rmsnorm.h"
+#include "lora_ce.h"
 #include "aux_kernels.cuh"
+#include "cross_entropy.cuh"
 #include "rmsnorm.cuh"
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
@@ -1466,6 +1468,138 @@ int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights*
     LMLP_TRY(lora_mlp_backward(shape, w, ws + b.xn, g, u, sv + b.s_mlp, dOut, ws + b.dxn, grads, ws + b.mlp_b,
                                b.b_total - b.mlp_b, stream));
     return launch_rmsnorm_bwd(shape->N, shape->d, X, gamma, rstd, ws + b.dxn, dX, di.sms, st);
+}
+
+}  // extern "C"
+
+// ============================================================================= cross-entropy
+//
+// Chunked cross-entropy (include/lora_ce.h): the forward reduces every
+// (row, vocabulary chunk) to its (max, sum of exp) in one launch and combines
+// each row's chunks in chunk order in a second; the backward is one
+// streaming launch over the same (row, chunk) grid.
+
+namespace {
+
+int validate_ce(const lora_ce_shape* sh) {
+    if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->N < 1 || sh->V < 1 || sh->ld < sh->V) return LORA_MLP_ERR_INVALID_ARG;
+    if (!std::isfinite(sh->logit_scale) || sh->logit_scale == 0.0f) return LORA_MLP_ERR_INVALID_ARG;
+    if (!std::isfinite(sh->softcap) || sh->softcap < 0.0f) return LORA_MLP_ERR_INVALID_ARG;
+    if (sh->ld % kCeVec != 0) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    const long long nchunk = (sh->V + kCeChunk - 1) / kCeChunk;
+    if (sh->N > (static_cast<long long>(INT32_MAX) / nchunk)) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    return LORA_MLP_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+CeArgs ce_args(const lora_ce_shape* sh, const void* logits, const int64_t* labels) {
+    CeArgs a;
+    a.z = static_cast<const __nv_bfloat16*>(logits);
+    a.ld = sh->ld;
+    a.V = sh->V;
+    a.N = sh->N;
+    a.nchunk = static_cast<int>((sh->V + kCeChunk - 1) / kCeChunk);
+    a.labels = reinterpret_cast<const long long*>(labels);
+    a.ignore = sh->ignore_index;
+    a.scale = sh->logit_scale;
+    a.cap = sh->softcap;
+    const bool cap = sh->softcap > 0.0f;
+    a.k2 = cap ? 2.0f * sh->logit_scale / sh->softcap * kLog2e : 0.0f;
+    a.inv_cap = cap ? 1.0f / sh->softcap : 0.0f;
+    return a;
+}
+
+struct CePlan {
+    size_t part, ty, total;
+};
+
+CePlan make_ce_plan(const lora_ce_shape& sh) {
+    const size_t nchunk = static_cast<size_t>((sh.V + kCeChunk - 1) / kCeChunk);
+    Carver c;
+    CePlan p;
+    p.part = c.take(static_cast<size_t>(sh.N) * nchunk * sizeof(float2));
+    p.ty = c.take(static_cast<size_t>(sh.N) * sizeof(float));
+    p.total = c.off;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lora_ce_sizes(const lora_ce_shape* shape, size_t* workspace_bytes) {
+    LMLP_TRY(validate_ce(shape));
+    if (workspace_bytes) *workspace_bytes = make_ce_plan(*shape).total;
+    return LORA_MLP_OK;
+}
+
+int lora_ce_forward(const lora_ce_shape* shape, const void* logits, const int64_t* labels, float* loss, float* lse,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_ce(shape));
+    if (logits == nullptr || labels == nullptr || loss == nullptr || lse == nullptr || workspace == nullptr)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (!aligned(logits, 16) || !aligned(labels, 8) || !aligned(loss, 4) || !aligned(lse, 4) ||
+        !aligned(workspace, 16))
+        return LORA_MLP_ERR_MISALIGNED;
+    const CePlan pl = make_ce_plan(*shape);
+    if (workspace_bytes < pl.total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CeArgs a = ce_args(shape, logits, labels);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float2* part = reinterpret_cast<float2*>(ws + pl.part);
+    float* ty = reinterpret_cast<float*>(ws + pl.ty);
+    {
+        LaunchScope scope("CE_fwd_chunks", st);
+        ce_fwd_partial_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(a, part, ty);
+    }
+    LMLP_TRY(last_launch_error());
+    {
+        LaunchScope scope("CE_fwd_combine", st);
+        ce_fwd_combine_kernel<<<static_cast<unsigned>((shape->N + 255) / 256), 256, 0, st>>>(a, part, ty, loss,
+                                                                                            lse);
+    }
+    return last_launch_error();
+}
+
+int lora_ce_backward(const lora_ce_shape* shape, const void* logits, const int64_t* labels, const float* lse,
+                     const float* dloss, void* dlogits, void* stream) {
+    LMLP_TRY(validate_ce(shape));
+    if (logits == nullptr || labels == nullptr || lse == nullptr || dloss == nullptr || dlogits == nullptr)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (!aligned(logits, 16) || !aligned(dlogits, 16) || !aligned(labels, 8) || !aligned(lse, 4) ||
+        !aligned(dloss, 4))
+        return LORA_MLP_ERR_MISALIGNED;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CeArgs a = ce_args(shape, logits, labels);
+    {
+        LaunchScope scope("CE_bwd", st);
+        ce_bwd_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(
+            a, lse, dloss, static_cast<__nv_bfloat16*>(dlogits), shape->ld);
+    }
+    return last_launch_error();
+}
+
+int lora_ce_device_status(void* stream, int* status) {
+    if (status == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_ce_status) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyAsync(&v, addr, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(addr, &zero, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return LORA_MLP_ERR_CUDA;
+    *status = v;
+    return LORA_MLP_OK;
 }
 
 }  // extern "C"

@@ -11,7 +11,7 @@ from lora_fine_tuning_mlp_b200 import _lib
 from lora_fine_tuning_mlp_b200 import build as libbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADERS = [os.path.join(ROOT, "include", h) for h in ("lora_mlp.h", "lora_linear.h", "lora_rmsnorm.h")]
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("lora_mlp.h", "lora_linear.h", "lora_rmsnorm.h", "lora_ce.h")]
 
 
 @pytest.fixture(scope="module")
@@ -23,7 +23,7 @@ def L():
 def header_symbols():
     text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(lora_(?:mlp|linear|rmsnorm)_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(lora_(?:mlp|linear|rmsnorm|ce)_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_symbols():
@@ -223,3 +223,45 @@ def test_norm_and_block_argument_errors(L):
         == _lib.ERR_WORKSPACE_TOO_SMALL
     assert _lib.block_backward(sh, weights(), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, g, FAKE, bb, None) \
         == _lib.ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- cross-entropy
+
+
+def test_ce_sizes(L):
+    ws = _lib.ce_sizes(_lib.make_ce_shape(4096, 256000))
+    # one (max, sum) float2 per (row, 65536-logit chunk) and one float per row
+    assert ws >= 4096 * 4 * 8 + 4096 * 4
+    assert _lib.ce_sizes(_lib.make_ce_shape(1, 1, 8)) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), _lib.ERR_INVALID_ARG),
+    (dict(V=0), _lib.ERR_INVALID_ARG),
+    (dict(ld=999), _lib.ERR_INVALID_ARG),            # ld < V
+    (dict(ld=1004), _lib.ERR_UNSUPPORTED_SHAPE),     # not a multiple of 8
+    (dict(logit_scale=0.0), _lib.ERR_INVALID_ARG),
+    (dict(logit_scale=float("nan")), _lib.ERR_INVALID_ARG),
+    (dict(softcap=-1.0), _lib.ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), _lib.ERR_INVALID_ARG),
+])
+def test_ce_shape_validation(L, kw, code):
+    args = dict(N=37, V=1000, ld=1000, logit_scale=1.0, softcap=0.0)
+    args.update(kw)
+    sh = _lib.make_ce_shape(**args)
+    ws = ctypes.c_size_t()
+    assert L.lora_ce_sizes(ctypes.byref(sh), ctypes.byref(ws)) == code
+
+
+def test_ce_argument_errors(L):
+    sh = _lib.make_ce_shape(37, 1000, 1008, 1.0, 30.0)
+    ws = _lib.ce_sizes(sh)
+    assert _lib.ce_forward(sh, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 1, None) == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.ce_forward(sh, None, FAKE, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert _lib.ce_forward(sh, FAKE + 8, FAKE, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_MISALIGNED
+    assert _lib.ce_forward(sh, FAKE, FAKE + 4, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_MISALIGNED
+    assert _lib.ce_backward(sh, FAKE, FAKE, FAKE, FAKE, None, None) == _lib.ERR_INVALID_ARG
+    assert _lib.ce_backward(sh, FAKE, FAKE, FAKE, FAKE, FAKE + 2, None) == _lib.ERR_MISALIGNED
+    assert _lib.ce_backward(sh, FAKE, FAKE, FAKE + 1, FAKE, FAKE, None) == _lib.ERR_MISALIGNED
+    assert L.lora_ce_forward(None, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert L.lora_ce_device_status(None, None) == _lib.ERR_INVALID_ARG
