@@ -227,25 +227,47 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
     const int nchunks = bn >> 5;
     if constexpr (EPI == EPI_SWIGLU_BWD) {
         // g and u of the next 32 columns are loaded while this chunk computes.
-        const __nv_bfloat16* g_row = static_cast<const __nv_bfloat16*>(o.in0) + row * o.ld;
-        const __nv_bfloat16* u_row = static_cast<const __nv_bfloat16*>(o.in1) + row * o.ld;
+        // With a staging area the warp loads its 32 rows x 64 B block
+        // coalesced (four lanes per 64-byte row segment, every load filling
+        // whole sectors) and transposes it through shared memory into one
+        // row per lane; without one, each lane loads its own row.
+        const __nv_bfloat16* gbase = static_cast<const __nv_bfloat16*>(o.in0);
+        const __nv_bfloat16* ubase = static_cast<const __nv_bfloat16*>(o.in1);
+        const int lane = threadIdx.x & 31;
+        const int row0 = row - lane;
         uint4 gv[4], uv[4], gn[4], un[4];
         auto load_gu = [&](int c0, uint4(&gq)[4], uint4(&uq)[4]) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                if (row_ok && c0 + 8 * q < o.N) {
-                    gq[q] = ld_in(g_row + c0 + 8 * q);
-                    uq[q] = ld_in(u_row + c0 + 8 * q);
+                // coalesced: slot q holds row 8q + lane/4, columns c0 + 8 (lane%4) ..
+                // per lane:  slot q holds this lane's row, columns c0 + 8q ..
+                const int r = stg != 0 ? row0 + 8 * q + (lane >> 2) : row;
+                const int c = stg != 0 ? c0 + 8 * (lane & 3) : c0 + 8 * q;
+                if (r < o.M && c < o.N) {
+                    gq[q] = ld_in(gbase + static_cast<long long>(r) * o.ld + c);
+                    uq[q] = ld_in(ubase + static_cast<long long>(r) * o.ld + c);
                 } else {
                     gq[q] = make_uint4(0, 0, 0, 0);
                     uq[q] = make_uint4(0, 0, 0, 0);
                 }
             }
         };
+        // coalesced layout -> one row per lane, through the warp's staging area
+        auto to_rows = [&](uint4(&x)[4]) {
+            if (stg == 0) return;
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sts128(stg + (8 * q + (lane >> 2)) * kStageRowBytes + (lane & 3) * 16, x[q]);
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) x[q] = lds128(stg + lane * kStageRowBytes + q * 16);
+        };
         load_gu(col_base, gv, uv);
         for (int ch = 0; ch < nchunks; ++ch) {
             const int col0 = col_base + ch * 32;
             if (col0 >= o.N) break;  // warp-uniform
+            to_rows(gv);
+            to_rows(uv);
             if (ch + 1 < nchunks) load_gu(col0 + 32, gn, un);
             uint32_t v[32];
             src.load(ch * 32, v);
