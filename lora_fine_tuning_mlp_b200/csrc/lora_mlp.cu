@@ -312,8 +312,18 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     a.nmaps = b.nmaps;
     a.b_bytes = static_cast<uint32_t>(a.bn * 128);  // K-major: bn rows x 128 B; MN-major: bn/64 chunks x 8 KB
     const uint32_t stage_bytes = kATileBytes + NACC * a.b_bytes;
-    const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes();
-    int stages = static_cast<int>(budget / stage_bytes);
+    // A launch with more units than SMs runs two CTAs per SM, each with half
+    // the shared memory: a CTA's single TMA-issuing thread, not the stage
+    // count, limits how fast these HBM-bound products stream (measured on the
+    // adapter-gradient launch of the Llama-3-8B shapes: 164 -> 107 us).
+    // Launches with at most one unit per SM keep one CTA and the deeper
+    // pipeline, which measured faster for them.
+    // Two CTAs also need their accumulators to fit the SM's 512 TMEM columns
+    // together and at least three stages each.
+    const uint32_t budget1 = kSmemLimit - 1024 - gemm_ctl_bytes();
+    const uint32_t budget2 = kSmemLimit / 2 - 2048 - gemm_ctl_bytes();
+    const int cps = (b.units > sms && gemm_tmem_cols(NACC, a.bn) <= 256 && budget2 / stage_bytes >= 3) ? 2 : 1;
+    int stages = static_cast<int>((cps == 2 ? budget2 : budget1) / stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
@@ -329,7 +339,8 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     }
     a.wait_limit = g_wait_limit.load();
     a.force_timeout = g_force_timeout.load();
-    const int grid = b.units < sms ? b.units : sms;
+    const int ctas = sms * cps;
+    const int grid = b.units < ctas ? b.units : ctas;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

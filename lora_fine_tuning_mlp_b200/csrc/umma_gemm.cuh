@@ -446,7 +446,9 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int nacc, int bn) {
 }
 
 template <int NACC, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
+// Up to two CTAs share an SM (launches with more units than SMs), so the
+// register budget is that of two resident CTAs.
+__global__ void __launch_bounds__(kGemmThreads, 2) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
