@@ -45,7 +45,7 @@ using namespace lmlp;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a layout constant
+constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a layout constant  // split-K sizing target (B200 SM count); a layout constant
 constexpr int kMaxSplits = 32;
 constexpr size_t kAlign = 256;
 constexpr uint32_t kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
@@ -522,7 +522,7 @@ struct SkinnySpec {
     int64_t nkb;    // K blocks
 };
 
-void plan_splits(const SkinnySpec* sp, int n, int* out) {
+void plan_splits(const SkinnySpec* sp, int n, int* out, int slots = kTargetCtas) {
     int64_t max_kb = 1;
     for (int i = 0; i < n; ++i) max_kb = std::max(max_kb, sp[i].nkb);
     double best = 1e300;
@@ -534,7 +534,7 @@ void plan_splits(const SkinnySpec* sp, int n, int* out) {
             units += ceil_div(sp[i].M, kBM) * s;
             longest = std::max(longest, (sp[i].nkb + s - 1) / s);
         }
-        const int64_t rounds = (units + kTargetCtas - 1) / kTargetCtas;
+        const int64_t rounds = (units + slots - 1) / slots;
         const double cost = static_cast<double>(rounds) * static_cast<double>(longest + kUnitCost);
         if (cost < best - 1e-9) {
             best = cost;
@@ -556,6 +556,12 @@ int64_t launch_tiles(const SkinnySpec* sp, int n) {
 // The skinny launches of one forward + backward, in launch order.
 enum { SK_F0, SK_F2, SK_B0, SK_BMID, SK_B5, SK_COUNT };
 constexpr int kSkinnyProbs[SK_COUNT] = {1, 1, 2, 5, 1};
+// Units per round that plan_splits sizes each launch for: one per SM, or two
+// for the row projections that then run two CTAs per SM (launch_gemm), which
+// measured faster for them on the Llama-3-8B shapes (F2 50 -> 44 us, B0
+// 37 -> 29 us) and slower for F0 and B5, whose finalising CTAs write the
+// transposed tiles.
+constexpr int kSkinnySlots[SK_COUNT] = {kTargetCtas, 2 * kTargetCtas, 2 * kTargetCtas, kTargetCtas, kTargetCtas};
 
 struct Plan {
     int64_t N, d, d_ff, r, ldN;
@@ -614,7 +620,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     size_t part_f = 0, part_b = 0;
     int64_t max_tiles = 0;
     for (int l = 0; l < SK_COUNT; ++l) {
-        plan_splits(p.spec[l], kSkinnyProbs[l], p.splits[l]);
+        plan_splits(p.spec[l], kSkinnyProbs[l], p.splits[l], kSkinnySlots[l]);
         size_t off = 0;
         for (int i = 0; i < kSkinnyProbs[l]; ++i) {
             p.part_off[l][i] = off;
