@@ -163,60 +163,71 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
 #endif
 constexpr int kLoadBurst = LMLP_LOAD_BURST;
 
+// The producer (one thread).  On the HBM-bound rank-r launches this loop
+// bounds the stream, so it is kept as short as the MMA issuer's: segments
+// are walked directly, and the per-segment tensor maps and byte count are
+// looked up once per segment, not per K block.  A separate wait cursor runs
+// up to one burst ahead of the issue cursor.
 template <int NACC>
 __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
                                               const SmemCtl& c) {
     int stage = 0;
     uint32_t phase = 0;
+    int wst = 0;  // next stage whose release to wait for
+    uint32_t wph = 0;
+    int credits = 0;  // stages known free ahead of `stage`
     const int burst = a.stages >= 2 * kLoadBurst ? kLoadBurst : 1;
     for (int u = blockIdx.x; u < a.total_units; u += gridDim.x) {
         const Unit t = decode_unit(a, u);
         const Prob& P = a.prob[t.p];
-        int seg = 0, seg_kb0 = 0;
-        for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += burst) {
-            const int cnt = min(burst, t.kb1 - kb0);
-            {
-                int st = stage;
-                uint32_t ph = phase;
-                for (int i = 0; i < cnt; ++i) {
-                    if (!wait_or_abort(c.empty + 8u * st, ph ^ 1u, c)) return;
-                    if (++st == a.stages) {
-                        st = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
-            for (int kb = kb0; kb < kb0 + cnt; ++kb) {
-                while (kb >= seg_kb0 + P.seg[seg].kblocks) {
-                    seg_kb0 += P.seg[seg].kblocks;
-                    ++seg;
-                }
-                const Seg& S = P.seg[seg];
-                const int k0 = (kb - seg_kb0) * kBK;
-                uint32_t bytes = kATileBytes;
+        const bool a_mn = P.a_mn != 0, b_mn = P.b_mn != 0;
+        const int m0 = t.mb * kBM;
+        const int n0 = t.nb * a.bn;
+        const int nbj = b_mn ? a.bn / 64 : 1;
+        int seg_kb0 = 0;
+        for (int sg = 0; sg < P.nsegs; ++sg) {
+            const Seg& S = P.seg[sg];
+            const int lo = max(t.kb0 - seg_kb0, 0), hi = min(t.kb1 - seg_kb0, S.kblocks);
+            seg_kb0 += S.kblocks;
+            if (lo >= hi) continue;
+            const CUtensorMap* am = &a.maps[S.a_map];
+            const CUtensorMap* bm[NACC];
+            uint32_t bytes = kATileBytes;
 #pragma unroll
-                for (int acc = 0; acc < NACC; ++acc)
-                    if (S.b_map[acc] >= 0) bytes += a.b_bytes;
+            for (int acc = 0; acc < NACC; ++acc) {
+                bm[acc] = S.b_map[acc] >= 0 ? &a.maps[S.b_map[acc]] : nullptr;
+                if (bm[acc] != nullptr) bytes += a.b_bytes;
+            }
+            for (int kb = lo; kb < hi; ++kb) {
+                if (credits == 0) {
+                    for (int i = 0; i < burst; ++i) {
+                        if (!wait_or_abort(c.empty + 8u * wst, wph ^ 1u, c)) return;
+                        if (++wst == a.stages) {
+                            wst = 0;
+                            wph ^= 1u;
+                        }
+                    }
+                    credits = burst;
+                }
+                --credits;
+                const int k0 = kb * kBK;
                 const uint32_t fb = c.full + 8u * stage;
                 mbar_arrive_expect_tx(fb, bytes);
                 const uint32_t sA = smem_base + stage * stage_bytes;
-                const CUtensorMap* am = &a.maps[S.a_map];
-                if (P.a_mn) {
-                    tma_load_2d(sA, am, fb, t.mb * kBM, k0);
-                    tma_load_2d(sA + 8192u, am, fb, t.mb * kBM + 64, k0);
+                if (a_mn) {
+                    tma_load_2d(sA, am, fb, m0, k0);
+                    tma_load_2d(sA + 8192u, am, fb, m0 + 64, k0);
                 } else {
-                    tma_load_2d(sA, am, fb, k0, t.mb * kBM);
+                    tma_load_2d(sA, am, fb, k0, m0);
                 }
 #pragma unroll
                 for (int acc = 0; acc < NACC; ++acc) {
-                    if (S.b_map[acc] < 0) continue;
+                    if (bm[acc] == nullptr) continue;
                     const uint32_t sB = sA + kATileBytes + acc * a.b_bytes;
-                    const CUtensorMap* bm = &a.maps[S.b_map[acc]];
-                    if (P.b_mn) {
-                        for (int j = 0; j < a.bn / 64; ++j)
-                            tma_load_2d(sB + 8192u * j, bm, fb, t.nb * a.bn + 64 * j, k0);
+                    if (b_mn) {
+                        for (int j = 0; j < nbj; ++j) tma_load_2d(sB + 8192u * j, bm[acc], fb, n0 + 64 * j, k0);
                     } else {
-                        tma_load_2d(sB, bm, fb, k0, t.nb * a.bn);
+                        tma_load_2d(sB, bm[acc], fb, k0, n0);
                     }
                 }
                 if (++stage == a.stages) {
