@@ -321,9 +321,10 @@ int launch_gemm(GemmBuilder& b, int sms, cudaStream_t st, const char* name, int*
     // Two CTAs also need their accumulators to fit the SM's 512 TMEM columns
     // together and at least three stages each.
     const uint32_t budget1 = kSmemLimit - 1024 - gemm_ctl_bytes();
-    const uint32_t budget2 = kSmemLimit / 2 - 2048 - gemm_ctl_bytes();
-    const int cps = (b.units > sms && gemm_tmem_cols(NACC, a.bn) <= 256 && budget2 / stage_bytes >= 3) ? 2 : 1;
-    int stages = static_cast<int>((cps == 2 ? budget2 : budget1) / stage_bytes);
+    const uint32_t budgetN = kSmemLimit / LMLP_MAX_CPS - 2048 - gemm_ctl_bytes();
+    const int cps = (b.units > sms && gemm_tmem_cols(NACC, a.bn) <= 512 / LMLP_MAX_CPS &&
+                     budgetN / stage_bytes >= 3) ? LMLP_MAX_CPS : 1;
+    int stages = static_cast<int>((cps > 1 ? budgetN : budget1) / stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;

@@ -158,6 +158,12 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
 // producer first waits until that many stages are free, then issues their
 // copies back to back, so the DRAM pages of each A row are requested
 // together rather than one 128-byte piece at a time.
+#ifndef LMLP_FIN_BATCH
+#define LMLP_FIN_BATCH 8  // split-K partials whose loads the finalising CTA issues together
+#endif
+#ifndef LMLP_MAX_CPS
+#define LMLP_MAX_CPS 2  // most CTAs of this kernel that share an SM
+#endif
 #ifndef LMLP_LOAD_BURST
 #define LMLP_LOAD_BURST 4
 #endif
@@ -352,10 +358,10 @@ __device__ __forceinline__ void splitk_finalize(const Prob& P, const Unit& t, in
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
         // Loads of up to 8 splits are issued before their (in-order) adds, so a
         // tile with many splits costs a few L2 round trips, not one per split.
-        for (int sp0 = 0; sp0 < P.splits; sp0 += 8) {
-            float4 v[8][2];
+        for (int sp0 = 0; sp0 < P.splits; sp0 += LMLP_FIN_BATCH) {
+            float4 v[LMLP_FIN_BATCH][2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < LMLP_FIN_BATCH; ++q) {
                 if (sp0 + q < P.splits) {
                     const float4* src4 = reinterpret_cast<const float4*>(src + (sp0 + q) * P.split_stride + j);
                     v[q][0] = __ldcg(src4);
@@ -363,7 +369,7 @@ __device__ __forceinline__ void splitk_finalize(const Prob& P, const Unit& t, in
                 }
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < LMLP_FIN_BATCH; ++q) {
                 if (sp0 + q < P.splits) {
                     acc[0] += v[q][0].x; acc[1] += v[q][0].y; acc[2] += v[q][0].z; acc[3] += v[q][0].w;
                     acc[4] += v[q][1].x; acc[5] += v[q][1].y; acc[6] += v[q][1].z; acc[7] += v[q][1].w;
@@ -459,7 +465,7 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int nacc, int bn) {
 template <int NACC, int EPI>
 // Up to two CTAs share an SM (launches with more units than SMs), so the
 // register budget is that of two resident CTAs.
-__global__ void __launch_bounds__(kGemmThreads, 2) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
+__global__ void __launch_bounds__(kGemmThreads, LMLP_MAX_CPS) umma_gemm_kernel(const __grid_constant__ GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
