@@ -282,6 +282,7 @@ CE_CONFIGS = (
     CEConfig("gemma2_256k_ce", 4096, 256000, 1.0, 30.0, z_std=10.0, index=73),
     CEConfig("cohere_256k_ce", 4096, 256000, 0.0625, 0.0, z_std=32.0, index=74),
     CEConfig("llama3_128k_ce", 4096, 128256, 1.0, 0.0, index=75),
+    CEConfig("gemma2_256k_ce_1k", 1024, 256000, 1.0, 30.0, z_std=10.0, index=76),  # 1024 tokens: profiling size
 )
 CE_BY_NAME = {c.name: c for c in CE_CONFIGS}
 
