@@ -6,96 +6,121 @@
 
 namespace lmlp {
 
-// Block-int4 weight element -> bf16: (fp32(q) * fp32(scale)) / 7 in IEEE fp32
-// (the product is exact; the divide is correctly rounded), then round to
-// nearest-even bf16.
-__device__ __forceinline__ __nv_bfloat16 dequant_one(int q, float scale) {
-    return __float2bfloat16_rn(__fdiv_rn(__fmul_rn(static_cast<float>(q), scale), 7.0f));
+// Packed two-lane fp32 arithmetic (sm_100 f32x2 instructions; each lane is
+// rounded exactly as the scalar instruction would round it).
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_packf(float lo, float hi) {
+    return f2_pack(__float_as_uint(lo), __float_as_uint(hi));
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
 }
 
-__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 v) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(v));
+// x / 7 correctly rounded in fp32 for x = fp32(q) * fp32(scale), q an int4
+// code and scale an fp16 (so x has at most 14 significant bits): the product
+// y = x * fl(1/7), then one correction by the exact residual e = x - 7y,
+// y + e * fl(1/7) rounded once by the FMA.  Checked exhaustively with exact
+// rational arithmetic against the correctly rounded quotient for every code
+// 1..8 and every positive finite fp16 scale (253,944 cases); negative x
+// follow from the sign symmetry of round-to-nearest-even.  It is evaluated
+// from -x (y = (-x)(-1/7), e' = 7y + (-x) = -e, result = e'(-1/7) + y): the
+// same values, and a zero x keeps its sign (a residual sum of +0 and -0
+// would otherwise turn -0 into +0).  Two lanes at a time; neg_x = -x.
+__device__ __forceinline__ uint64_t div7_rn_neg2(uint64_t neg_x) {
+    const uint64_t nr = f2_packf(-1.0f / 7.0f, -1.0f / 7.0f);  // -fl(1/7)
+    const uint64_t seven = f2_packf(7.0f, 7.0f);
+    const uint64_t y = f2_mul(neg_x, nr);
+    const uint64_t e = f2_fma(y, seven, neg_x);
+    return f2_fma(e, nr, y);
 }
 
-// Warp-cooperative dequantisation.  Packed codes [rows, cols/2] bytes and
-// scales [rows, cols/64] are row-major, so flat block i (64 elements, one
-// scale) has its 32 code bytes at byte 32*i and its outputs at element 64*i.
-// A warp takes kDqPasses passes of 8 consecutive blocks (512 elements) per
-// iteration:
-//  1. every lane issues its loads first (the scale of block L/4 and two
-//     4-byte code words per pass), so their latencies overlap;
-//  2. lane L computes magnitudes L%4 and L%4+4 (and 8 when L%4 = 0) of block
-//     L/4 with dequant_one and writes them to that block's 16-entry table in
-//     shared memory at the code's two's-complement nibble, the negative code
-//     -m at nibble 16-m with the sign bit flipped.  This equals
-//     dequant_one(-m, scale) bit for bit: q*scale is exact and round to
-//     nearest even is symmetric in sign, fl(-x) = -fl(x);
-//  3. lane L converts the 8 codes of elements 8L .. 8L+7 and 256+8L ..
-//     256+8L+7 of each pass with table lookups: one 4-byte load and one
-//     16-byte store each, so a warp's loads and stores cover contiguous
-//     128 B and 512 B spans.
-constexpr int kDqWarps = 8;
-#ifndef LMLP_DQ_PASSES
-#define LMLP_DQ_PASSES 2
-#endif
-constexpr int kDqPasses = LMLP_DQ_PASSES;
+// fp32 bits of 2^23 + (q + 8) for the two's-complement nibble n (0..15) of
+// code q: q + 8 = n ^ 8, and 2^23 + m is exact in fp32 for m < 2^23.
+__device__ __forceinline__ uint32_t nibble_bits(uint32_t n) { return 0x4B000000u | (n ^ 8u); }
 
-__global__ void __launch_bounds__(kDqWarps * 32) dequant_int4_kernel(const uint32_t* __restrict__ packed,
-                                                                     const __half* __restrict__ scales,
-                                                                     long long nblocks,
-                                                                     __nv_bfloat16* __restrict__ w) {
-    __shared__ uint32_t tab[kDqWarps][kDqPasses * 8 * 16];
-    const int lane = threadIdx.x & 31;
-    const int wid = threadIdx.x >> 5;
-    uint32_t* t = tab[wid];
-    const long long nchunks = (nblocks + 8 * kDqPasses - 1) / (8 * kDqPasses);
-    for (long long c = static_cast<long long>(blockIdx.x) * kDqWarps + wid; c < nchunks;
-         c += static_cast<long long>(gridDim.x) * kDqWarps) {
-        const long long cb = c * (8 * kDqPasses);  // first block of this iteration
-        float sc[kDqPasses];
-        uint32_t word[kDqPasses][2];
+// Eight codes (one 4-byte word, element 2k in the low nibble of byte k) ->
+// eight bf16 values (fp32(q) * fp32(scale)) / 7, rounded to nearest-even
+// bf16.  The product is exact and the quotient correctly rounded (div7_rn);
+// a non-finite scale takes IEEE's own divide (inf / 7 = inf, NaN stays NaN).
+template <bool kFinite>
+__device__ __forceinline__ uint4 dequant_word(uint32_t word, float scale) {
+    uint32_t o[4];
+    const uint64_t c8 = f2_packf(8388616.0f, 8388616.0f);  // 2^23 + 8
+    const uint64_t ns2 = f2_packf(-scale, -scale);
 #pragma unroll
-        for (int p = 0; p < kDqPasses; ++p) {
-            const long long b = cb + p * 8 + (lane >> 2);
-            sc[p] = b < nblocks ? __half2float(scales[b]) : 0.0f;
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t bl = nibble_bits((word >> (8 * j)) & 0xFu);
+        const uint32_t bh = nibble_bits((word >> (8 * j + 4)) & 0xFu);
+        // (2^23 + q + 8) - (2^23 + 8) = q exactly (+0 for code 0); q * (-scale)
+        // is -(q * scale) exactly, the sign of a zero included
+        const uint64_t neg_x = f2_mul(f2_sub(f2_pack(bl, bh), c8), ns2);
+        float lo, hi;
+        if (kFinite) {
+            f2_unpack(div7_rn_neg2(neg_x), lo, hi);
+        } else {
+            f2_unpack(neg_x, lo, hi);
+            lo = __fdiv_rn(lo, -7.0f);
+            hi = __fdiv_rn(hi, -7.0f);
+        }
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        o[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One thread per 8-code group per step: packed codes [rows, cols/2] bytes
+// and scales [rows, cols/64] are row-major, so group g (elements 8g .. 8g+7)
+// is the 4-byte code word g, its scale is scale g/8 and its output the 16
+// bytes at element 8g.  A CTA takes kDqUnroll x 256 consecutive groups and
+// issues all their loads before converting, so a warp's loads and stores
+// cover contiguous 128-byte and 512-byte spans and several are in flight.
+// Everything runs on the FMA and integer pipes, two lanes per fp32
+// instruction.
+constexpr int kDqThreads = 256;
+constexpr int kDqUnroll = 4;
+
+__global__ void __launch_bounds__(kDqThreads) dequant_int4_kernel(const uint32_t* __restrict__ packed,
+                                                                  const __half* __restrict__ scales,
+                                                                  long long ngroups,
+                                                                  __nv_bfloat16* __restrict__ w) {
+    const long long span = static_cast<long long>(kDqThreads) * kDqUnroll;
+    for (long long g0 = static_cast<long long>(blockIdx.x) * span + threadIdx.x; g0 < ngroups;
+         g0 += static_cast<long long>(gridDim.x) * span) {
+        uint32_t word[kDqUnroll];
+        float sc[kDqUnroll];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int e0 = h * 256 + lane * 8;
-                const long long e = (cb + p * 8) * 64 + e0;
-                word[p][h] = (cb + p * 8 + (e0 >> 6)) < nblocks ? packed[e >> 3] : 0u;
-            }
+        for (int k = 0; k < kDqUnroll; ++k) {
+            const long long g = g0 + k * kDqThreads;
+            word[k] = g < ngroups ? __ldcs(packed + g) : 0u;
+            sc[k] = g < ngroups ? __half2float(scales[g >> 3]) : 0.0f;
         }
 #pragma unroll
-        for (int p = 0; p < kDqPasses; ++p) {
-            uint32_t* tb = t + (p * 8 + (lane >> 2)) * 16;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int m = (lane & 3) + 4 * j;
-                const uint32_t v = bf16_bits(dequant_one(m, sc[p]));
-                tb[m] = v;
-                if (m != 0) tb[16 - m] = v ^ 0x8000u;
-            }
-            if ((lane & 3) == 0) tb[8] = bf16_bits(dequant_one(8, sc[p])) ^ 0x8000u;
+        for (int k = 0; k < kDqUnroll; ++k) {
+            const long long g = g0 + k * kDqThreads;
+            if (g >= ngroups) break;
+            const uint4 v = fabsf(sc[k]) <= 65504.0f ? dequant_word<true>(word[k], sc[k])  // finite scale
+                                                     : dequant_word<false>(word[k], sc[k]);
+            __stcs(reinterpret_cast<uint4*>(w) + g, v);
         }
-        __syncwarp();
-#pragma unroll
-        for (int p = 0; p < kDqPasses; ++p) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int e0 = h * 256 + lane * 8;
-                const int lb = p * 8 + (e0 >> 6);
-                if (cb + lb < nblocks) {
-                    const uint32_t* tb = t + lb * 16;
-                    const uint32_t wd = word[p][h];
-                    uint32_t o[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        o[k] = tb[(wd >> (8 * k)) & 0xFu] | (tb[(wd >> (8 * k + 4)) & 0xFu] << 16);
-                    *reinterpret_cast<uint4*>(w + (cb + p * 8) * 64 + e0) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
-        }
-        __syncwarp();
     }
 }
 

@@ -489,16 +489,16 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
 
 int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
                    cudaStream_t st) {
-    const long long nblk = rows * cols / 64;
-    const long long nchunks = (nblk + 8 * kDqPasses - 1) / (8 * kDqPasses);
-    long long blocks = (nchunks + kDqWarps - 1) / kDqWarps;
-    const long long cap = static_cast<long long>(sms) * 8;  // 8 CTAs of 8 warps: 64 warps per SM
+    const long long ngroups = rows * cols / 8;  // 8 codes per 4-byte word
+    const long long span = static_cast<long long>(kDqThreads) * kDqUnroll;
+    long long blocks = (ngroups + span - 1) / span;
+    const long long cap = static_cast<long long>(sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     {
         LaunchScope scope("dequant_int4", st);
-        dequant_int4_kernel<<<static_cast<int>(blocks), kDqWarps * 32, 0, st>>>(
-            static_cast<const uint32_t*>(packed), static_cast<const __half*>(scales), nblk,
+        dequant_int4_kernel<<<static_cast<int>(blocks), kDqThreads, 0, st>>>(
+            static_cast<const uint32_t*>(packed), static_cast<const __half*>(scales), ngroups,
             static_cast<__nv_bfloat16*>(w));
     }
     return last_launch_error();
