@@ -446,6 +446,24 @@ def rmsnorm_backward(x: torch.Tensor, gamma: torch.Tensor, rstd: torch.Tensor, d
     return dx
 
 
+class RMSNormFunction(torch.autograd.Function):
+    """autograd wrapper of the library's RMSNorm: y = x * rstd * gamma per row,
+    with the frozen gain gamma (no gradient for it) and the forward's rstd
+    reused by the backward.  Usage: RMSNormFunction.apply(x, gamma, eps)."""
+
+    @staticmethod
+    def forward(ctx, x, gamma, eps=1e-5):
+        x = x.contiguous()
+        y, rstd = rmsnorm_forward(x, gamma, eps)
+        ctx.save_for_backward(x, gamma, rstd)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, gamma, rstd = ctx.saved_tensors
+        return rmsnorm_backward(x, gamma, rstd, dy.contiguous()), None, None
+
+
 def block_forward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, eps: float, *, out=None,
                   workspace: Workspace | None = None, stream=None):
     """out = MLP(RMSNorm(X) * gamma).  Returns (out, Saved); Saved.lowrank

@@ -18,6 +18,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "f32x2.cuh"
+
 namespace lmlp {
 
 constexpr int kCeThreads = 256;
@@ -63,15 +65,50 @@ __device__ __forceinline__ float ce_exp2(float x) {
 // e^x = 2^(x log2(e)), for the (non-positive) differences t - max.
 __device__ __forceinline__ float ce_exp(float x) { return ce_exp2(x * kLog2e); }
 
+__device__ __forceinline__ float ce_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Transformed logit t.  With softcapping,
-// c tanh(w) = c (1 - 2 / (1 + e^(2w))), w = s z / c; the exponent is clamped
-// where tanh is already +-1 in fp32, so 1 + 2^x stays finite.
+// c tanh(w) = c - 2c / (1 + e^(2w)), w = s z / c.  Where tanh is +-1 in fp32
+// the exponential saturates to inf (reciprocal 0: t = c) or 0 (t = -c).
 __device__ __forceinline__ float ce_t(const CeArgs& a, float z) {
-    if (a.cap > 0.0f) {
-        const float x = fminf(fmaxf(a.k2 * z, -120.0f), 120.0f);
-        return a.cap * (1.0f - __fdividef(2.0f, 1.0f + ce_exp2(x)));
-    }
+    if (a.cap > 0.0f) return fmaf(ce_rcp(1.0f + ce_exp2(a.k2 * z)), -2.0f * a.cap, a.cap);
     return a.scale * z;
+}
+
+// The same for the four bf16 pairs of a 16-byte vector, as packed fp32
+// pairs {t[2k], t[2k+1]}: the fp32 arithmetic two lanes per instruction,
+// each lane rounded as ce_t rounds it.
+__device__ __forceinline__ void ce_t8(const CeArgs& a, const uint4& v, uint64_t (&t2)[4]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t z2 = f2_pack(w[k] << 16, w[k] & 0xFFFF0000u);
+        if (a.cap > 0.0f) {
+            float lo, hi;
+            f2_unpack(f2_mul(z2, f2_packf(a.k2, a.k2)), lo, hi);
+            f2_unpack(f2_add(f2_packf(ce_exp2(lo), ce_exp2(hi)), f2_packf(1.0f, 1.0f)), lo, hi);
+            t2[k] = f2_fma(f2_packf(ce_rcp(lo), ce_rcp(hi)), f2_packf(-2.0f * a.cap, -2.0f * a.cap),
+                           f2_packf(a.cap, a.cap));
+        } else {
+            t2[k] = f2_mul(z2, f2_packf(a.scale, a.scale));
+        }
+    }
+}
+
+// e^(t - m) for four packed pairs: subtract and scale two lanes at a time,
+// the exponentials one by one.
+__device__ __forceinline__ void ce_exp8(const uint64_t (&t2)[4], float m, uint64_t (&p2)[4]) {
+    const uint64_t m2 = f2_packf(m, m), l2e = f2_packf(kLog2e, kLog2e);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        f2_unpack(f2_mul(f2_sub(t2[k], m2), l2e), lo, hi);
+        p2[k] = f2_packf(ce_exp2(lo), ce_exp2(hi));
+    }
 }
 
 // (m, s) := (max, sum of e^(t - max)) of the union of two sets.
@@ -106,17 +143,19 @@ __device__ __forceinline__ void ce_load_tile(const __nv_bfloat16* zc, int tb, in
     }
 }
 
-// The transformed logits of the 8-wide vector at offset j < n; past n: -inf.
+// The transformed logits of the 8-wide vector at offset j < n, as packed
+// pairs; past n: -inf.
 __device__ __forceinline__ void ce_vector(const CeArgs& a, const __nv_bfloat16* zc, int j, int n, const uint4& v,
-                                          float (&t)[8]) {
+                                          uint64_t (&t2)[4]) {
     if (j + kCeVec <= n) {
-        ce_unpack(v, t);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = ce_t(a, t[e]);
+        ce_t8(a, v, t2);
     } else {
+        float t[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             t[e] = j + e < n ? ce_t(a, __bfloat162float(zc[j + e])) : __int_as_float(0xff800000u);  // -inf
+#pragma unroll
+        for (int k = 0; k < 4; ++k) t2[k] = f2_packf(t[2 * k], t[2 * k + 1]);
     }
 }
 
@@ -131,8 +170,11 @@ __device__ __forceinline__ void ce_fwd_tile(const CeArgs& a, const __nv_bfloat16
     for (int it = 0; it < kCeItems; ++it) {
         const int j = tb + (it * kCeThreads + static_cast<int>(threadIdx.x)) * kCeVec;
         if (j >= n) break;  // later vectors of this thread lie further right
+        uint64_t t2[4];
+        ce_vector(a, zc, j, n, v[it], t2);
         float t[8];
-        ce_vector(a, zc, j, n, v[it], t);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f2_unpack(t2[k], t[2 * k], t[2 * k + 1]);
         if (static_cast<unsigned>(yr - j) < static_cast<unsigned>(kCeVec)) {  // the label's vector
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -144,10 +186,11 @@ __device__ __forceinline__ void ce_fwd_tile(const CeArgs& a, const __nv_bfloat16
             r.s *= ce_exp(r.m - m8);
             r.m = m8;
         }
-        float s8 = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s8 += ce_exp(t[e] - r.m);
-        r.s += s8;
+        uint64_t p2[4];
+        ce_exp8(t2, r.m, p2);
+        float lo, hi;
+        f2_unpack(f2_add(f2_add(p2[0], p2[1]), f2_add(p2[2], p2[3])), lo, hi);
+        r.s += lo + hi;
     }
 }
 
@@ -229,44 +272,45 @@ __device__ __forceinline__ void ce_bwd_tile(const CeArgs& a, const __nv_bfloat16
     for (int it = 0; it < kCeItems; ++it) {
         const int j = tb + (it * kCeThreads + static_cast<int>(threadIdx.x)) * kCeVec;
         if (j >= n) break;
-        float d[8];
-        if (ignored) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) d[e] = 0.0f;
-        } else {
-            float t[8];
-            ce_vector(a, zc, j, n, v[it], t);
-            float p[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = ce_exp(t[e] - L);
+        uint32_t o[4] = {0u, 0u, 0u, 0u};
+        if (!ignored) {
+            uint64_t t2[4], p2[4];
+            ce_vector(a, zc, j, n, v[it], t2);
+            ce_exp8(t2, L, p2);
             if (static_cast<unsigned>(yr - j) < static_cast<unsigned>(kCeVec)) {  // the label's vector
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (e == yr - j) p[e] -= 1.0f;
-            }
-            if (a.cap > 0.0f) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float q = t[e] * a.inv_cap;  // t / c
-                    d[e] = g * p[e] * (1.0f - q * q);
+                for (int k = 0; k < 4; ++k) {
+                    float lo, hi;
+                    f2_unpack(p2[k], lo, hi);
+                    if (2 * k == yr - j) lo -= 1.0f;
+                    if (2 * k + 1 == yr - j) hi -= 1.0f;
+                    p2[k] = f2_packf(lo, hi);
                 }
-            } else {
+            }
+            const uint64_t g2 = f2_packf(g, g);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) d[e] = g * p[e];
+            for (int k = 0; k < 4; ++k) {
+                uint64_t d2 = f2_mul(p2[k], g2);
+                if (a.cap > 0.0f) {  // times 1 - (t/c)^2
+                    const uint64_t q2 = f2_mul(t2[k], f2_packf(a.inv_cap, a.inv_cap));
+                    const uint64_t nq2 = f2_mul(t2[k], f2_packf(-a.inv_cap, -a.inv_cap));
+                    d2 = f2_mul(d2, f2_fma(q2, nq2, f2_packf(1.0f, 1.0f)));
+                }
+                float lo, hi;
+                f2_unpack(d2, lo, hi);
+                __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+                o[k] = *reinterpret_cast<uint32_t*>(&h);
             }
         }
         if (j + kCeVec <= n) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(d[2 * e], d[2 * e + 1]);
-                w[e] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            __stcs(reinterpret_cast<uint4*>(dc + j), make_uint4(w[0], w[1], w[2], w[3]));
+            __stcs(reinterpret_cast<uint4*>(dc + j), make_uint4(o[0], o[1], o[2], o[3]));
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                if (j + e < n) dc[j + e] = __float2bfloat16_rn(d[e]);
+                if (j + e < n) {
+                    const uint32_t word = o[e >> 1];
+                    dc[j + e] = __ushort_as_bfloat16(static_cast<unsigned short>(e & 1 ? word >> 16 : word & 0xFFFFu));
+                }
         }
     }
 }

@@ -116,6 +116,27 @@ def test_block_equals_its_parts_bitwise():
         assert torch.equal(grads[k], grads2[k]), k
 
 
+def test_rmsnorm_autograd_function_matches_oracle():
+    """RMSNormFunction: forward y and backward dx (the gain is frozen) against
+    the fp64 oracle."""
+    rng = np.random.default_rng(61)
+    N, d = 300, 1024
+    x = (rng.standard_normal((N, d)) * rng.uniform(0.25, 4.0, (N, 1))).astype(np.float32)
+    gamma = rng.uniform(0.5, 1.5, d).astype(np.float32)
+    dy = rng.standard_normal((N, d)).astype(np.float32)
+    xb, gb, dyb = (synth.f32_to_bf16_bits(a) for a in (x, gamma, dy))
+    dev = torch.device("cuda:0")
+    tx = api.to_device_bf16(xb, dev).requires_grad_(True)
+    tg = api.to_device_bf16(gb, dev)
+    y = api.RMSNormFunction.apply(tx, tg, EPS)
+    y.backward(api.to_device_bf16(dyb, dev))
+    x64, g64, dy64 = (synth.bf16_bits_to_f32(a).astype(np.float64) for a in (xb, gb, dyb))
+    ry, rstd = orn.rmsnorm_forward(x64, g64, EPS)
+    rdx = orn.rmsnorm_backward(x64, g64, rstd, dy64)
+    assert relerr(np64(y.detach()), ry) <= TOL
+    assert relerr(np64(tx.grad), rdx) <= TOL
+
+
 def test_block_autograd_function():
     cfg = synth.custom(200, 128, 256, 8, 16.0, seed_index=85)
     inp = synth.make_block_inputs(cfg)
