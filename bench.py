@@ -299,8 +299,9 @@ def config_dict(cfg, block=False):
         return d
     return {"workload": cfg.name, "N_tokens": cfg.N, "d": cfg.d, "d_ff": cfg.d_ff, "r": cfg.r, "alpha": cfg.alpha,
             "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
-            "l2": "no flush: inputs larger than L2 (frozen weights %.0f MB > 126 MB)" % (
-                3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6),
+            "l2": "no flush: a step's operands exceed the 126 MB L2 (frozen weights %.0f MB, X %.0f MB, "
+                  "g/u/h %.0f MB each)" % (3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6,
+                                            2 * cfg.N * cfg.d / 1e6, 2 * cfg.N * cfg.d_ff / 1e6),
             "parallelism": "replicas"}
 
 
