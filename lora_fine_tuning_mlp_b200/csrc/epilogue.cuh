@@ -219,10 +219,14 @@ __device__ __forceinline__ void emit_chunk(__nv_bfloat16* base, long long ld, in
 
 // One output tile row per thread: `row` (may be >= M: stores are skipped),
 // columns [col_base, col_base + bn); accumulator a's column c is read from
-// `src` at a*bn + c.  `stg`: this warp's staging area (0 = store directly).
-template <int NACC, int EPI, class Src>
+// `src` at a*acc_stride + c.  `stg`: this warp's staging area (0 = store
+// directly).
+template <int NACC, int EPI, class Src, bool kPrefetchGU = true>
 __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src,
-                                              uint32_t stg = 0) {
+                                              uint32_t stg = 0, int acc_stride = -1) {
+    // acc_stride: distance in src columns between the two accumulators
+    // (default: bn, when a call covers all of a tile's columns)
+    if (acc_stride < 0) acc_stride = bn;
     const bool row_ok = row < o.M;
     const int nchunks = bn >> 5;
     if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -262,13 +266,16 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
 #pragma unroll
             for (int q = 0; q < 4; ++q) x[q] = lds128(stg + lane * kStageRowBytes + q * 16);
         };
-        load_gu(col_base, gv, uv);
+        if constexpr (kPrefetchGU) load_gu(col_base, gv, uv);
         for (int ch = 0; ch < nchunks; ++ch) {
             const int col0 = col_base + ch * 32;
             if (col0 >= o.N) break;  // warp-uniform
+            if constexpr (!kPrefetchGU) load_gu(col0, gv, uv);
             to_rows(gv);
             to_rows(uv);
-            if (ch + 1 < nchunks) load_gu(col0 + 32, gn, un);
+            if constexpr (kPrefetchGU) {
+                if (ch + 1 < nchunks) load_gu(col0 + 32, gn, un);
+            }
             uint32_t v[32];
             src.load(ch * 32, v);
             uint4 dgq[4], duq[4], hq[4];
@@ -277,10 +284,12 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, dgq, stg);
             emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, duq, stg);
             emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
+            if constexpr (kPrefetchGU) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                gv[q] = gn[q];
-                uv[q] = un[q];
+                for (int q = 0; q < 4; ++q) {
+                    gv[q] = gn[q];
+                    uv[q] = un[q];
+                }
             }
         }
     } else {
@@ -303,7 +312,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
 #pragma unroll
                 for (int acc = 0; acc < NACC; ++acc) {
                     uint32_t v[32];
-                    src.load(acc * bn + ch * 32, v);
+                    src.load(acc * acc_stride + ch * 32, v);
                     if (row_ok) {
                         float* dst = static_cast<float*>(acc == 0 ? o.out0 : o.out1) + o.split_off + row * o.ld + col0;
 #pragma unroll
@@ -317,7 +326,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                 }
             } else {  // EPI_SWIGLU_FWD
                 uint32_t vg[32], vu[32];
-                src.load2(ch * 32, vg, bn + ch * 32, vu);
+                src.load2(ch * 32, vg, acc_stride + ch * 32, vu);
                 uint4 gq[4], uq[4], hq[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {

@@ -431,7 +431,7 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_splits = 1;
     a.tail_part = tail_part;
     a.tail_ctr = tail_ctr;
-    const uint32_t staging = 128 + 4 * kStageWarpBytes;  // epilogue store staging (4 warps)
+    const uint32_t staging = 128 + pair_epi_warps<EPI>() * kStageWarpBytes;  // epilogue store staging, per warp
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kPairStageBytes);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
@@ -449,7 +449,7 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.blockDim = dim3(pair_threads<EPI>(), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;

@@ -41,6 +41,41 @@ constexpr uint32_t kPairStageBytes = kATileBytes + kPairBBytes;         // 32 KB
 constexpr int kPairMaxStages = LMLP_PAIR_STAGES;
 constexpr uint32_t kPairTmemCols = 512;                                 // 2 buffers x 256 columns
 
+// Epilogue warps of a CTA-pair launch, by epilogue kind: 4 (one per TMEM
+// lane quarter) or 8 (two per quarter, each taking half of the tile's
+// columns, for twice the epilogue's memory parallelism).  Ten warps leave
+// 168 registers a thread (three warps on two of the SM's four
+// sub-partitions), which the SwiGLU-backward epilogue fits once it stops
+// loading g and u a chunk ahead; the forward one does not (356 B of spills),
+// so only the former uses 8.  Measured on the dH GEMM: TinyLlama-1.1B shapes
+// 1061 -> 1036 us, Llama-3-8B shapes 491 -> 485 us (medians, interleaved).
+#ifndef LMLP_PAIR_EPI_WARPS_BF16
+#define LMLP_PAIR_EPI_WARPS_BF16 4
+#endif
+#ifndef LMLP_PAIR_EPI_WARPS_FWD
+#define LMLP_PAIR_EPI_WARPS_FWD 4
+#endif
+#ifndef LMLP_PAIR_EPI_WARPS_BWD
+#define LMLP_PAIR_EPI_WARPS_BWD 8
+#endif
+static_assert(LMLP_PAIR_EPI_WARPS_BF16 % 4 == 0 && LMLP_PAIR_EPI_WARPS_BF16 <= 8, "4 or 8 epilogue warps");
+static_assert(LMLP_PAIR_EPI_WARPS_FWD % 4 == 0 && LMLP_PAIR_EPI_WARPS_FWD <= 8, "4 or 8 epilogue warps");
+static_assert(LMLP_PAIR_EPI_WARPS_BWD % 4 == 0 && LMLP_PAIR_EPI_WARPS_BWD <= 8, "4 or 8 epilogue warps");
+template <int EPI>
+__host__ __device__ constexpr int pair_epi_warps() {
+    return EPI == EPI_SWIGLU_BWD ? LMLP_PAIR_EPI_WARPS_BWD
+                                 : (EPI == EPI_SWIGLU_FWD ? LMLP_PAIR_EPI_WARPS_FWD : LMLP_PAIR_EPI_WARPS_BF16);
+}
+template <int EPI>
+__host__ __device__ constexpr int pair_threads() {
+    return (2 + pair_epi_warps<EPI>()) * 32;
+}
+// Named barrier 1 over the epilogue warps.
+template <int EPI>
+__device__ __forceinline__ void pair_epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(pair_epi_warps<EPI>() * 32) : "memory");
+}
+
 struct PairSeg {
     int a_map;
     int b_map[2];  // B half 0 / half 1
@@ -238,6 +273,12 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int quarter = warp & 3;
+    // With 8 epilogue warps, warps 2-5 and 6-9 take the two column halves.
+    constexpr int kGroups = pair_epi_warps<EPI>() / 4;
+    // Two groups hold half the registers per thread: they load g and u chunk
+    // by chunk instead of one chunk ahead.
+    constexpr bool kPrefetch = kGroups == 1;
+    const int group = (warp - 2) >> 2;
     EpiOut o;
     o.out0 = P.out0;
     o.out1 = P.out1;
@@ -248,7 +289,9 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     o.split_off = 0;
     o.M = P.M;
     o.N = P.N;
-    const int bn = 256 / NACC;
+    const int bn = 256 / NACC;               // columns of each accumulator
+    const int gcols = bn / kGroups;          // of which this warp's group takes
+    const int gcol0 = group * gcols;
     // This warp's staging area for coalesced stores, after the barrier block.
     // Used by the SwiGLU epilogues (three outputs per chunk); the single bf16
     // output stores directly (measured interleaved: staging helps the former
@@ -271,12 +314,13 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * 256u;
         float* part = nullptr;
         if (t.tail < 0) {
-            epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, TmemSrc{tacc}, stg);
+            epilogue_tile<NACC, EPI, TmemSrc, kPrefetch>(o, row, t.nb * P.tile_n + gcol0, gcols,
+                                                         TmemSrc{tacc + static_cast<uint32_t>(gcol0)}, stg, bn);
         } else {
-            // this split's accumulator rows -> fp32 partial
+            // this split's accumulator rows (this group's columns) -> fp32 partial
             part = a.tail_part + ((static_cast<long long>(t.tail) * a.tail_splits + t.ks) * 2 + rank) * (kBM * 256ll) +
                    lrow * 256ll;
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int ch = group * (8 / kGroups); ch < (group + 1) * (8 / kGroups); ++ch) {
                 uint32_t v[32];
                 tmem_ld32(tacc + ch * 32, v);
                 tmem_ld_wait();
@@ -294,7 +338,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
         }
         if (t.tail >= 0) {
             __threadfence();
-            epi_bar();
+            pair_epi_bar<EPI>();
             if (threadIdx.x == 64) {
                 int* ctr = a.tail_ctr + t.tail * 2 + rank;
                 const int old = atomicAdd(ctr, 1);
@@ -302,19 +346,20 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
                 if (last) *ctr = 0;
                 *c.fin_flag = last;
             }
-            epi_bar();
+            pair_epi_bar<EPI>();
             if (*c.fin_flag) {
                 __threadfence();
                 const long long split_stride = 2ll * kBM * 256;
-                PartialSrc src{part - static_cast<long long>(t.ks) * split_stride, split_stride, a.tail_splits};
-                epilogue_tile<NACC, EPI>(o, row, t.nb * P.tile_n, bn, src, stg);
+                PartialSrc src{part - static_cast<long long>(t.ks) * split_stride + gcol0, split_stride,
+                               a.tail_splits};
+                epilogue_tile<NACC, EPI, PartialSrc, kPrefetch>(o, row, t.nb * P.tile_n + gcol0, gcols, src, stg, bn);
             }
         }
     }
 }
 
 template <bool B_MN, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
+__global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -338,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) umma2_gemm_kernel(const __gri
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(c.accf + 8u * b, 1);
-            mbar_init(c.acce + 8u * b, 8);  // 4 epilogue warps in each CTA of the pair
+            mbar_init(c.acce + 8u * b, 2 * pair_epi_warps<EPI>());  // every epilogue warp of both CTAs
         }
         mbar_init(c.drain, 1);
         mbar_init(c.never, 1);
