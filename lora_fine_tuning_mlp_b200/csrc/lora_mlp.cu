@@ -431,7 +431,8 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_splits = 1;
     a.tail_part = tail_part;
     a.tail_ctr = tail_ctr;
-    const uint32_t staging = 128 + pair_epi_warps<EPI>() * kStageWarpBytes;  // epilogue store staging, per warp
+    // epilogue store staging per warp, then the dH epilogue's g/u rings
+    const uint32_t staging = 128 + pair_epi_warps<EPI>() * kStageWarpBytes + pair_ring_bytes<EPI>();
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kPairStageBytes);
     if (stages > kPairMaxStages) stages = kPairMaxStages;

@@ -43,12 +43,10 @@ constexpr uint32_t kPairTmemCols = 512;                                 // 2 buf
 
 // Epilogue warps of a CTA-pair launch, by epilogue kind: 4 (one per TMEM
 // lane quarter) or 8 (two per quarter, each taking half of the tile's
-// columns, for twice the epilogue's memory parallelism).  Ten warps leave
-// 168 registers a thread (three warps on two of the SM's four
-// sub-partitions), which the SwiGLU-backward epilogue fits once it stops
-// loading g and u a chunk ahead; the forward one does not (356 B of spills),
-// so only the former uses 8.  Measured on the dH GEMM: TinyLlama-1.1B shapes
-// 1061 -> 1036 us, Llama-3-8B shapes 491 -> 485 us (medians, interleaved).
+// columns).  Ten warps leave 168 registers a thread (three warps on two of
+// the SM's four sub-partitions).  With g and u loaded into registers, 8 warps
+// made the dH GEMM 1-2 % faster than 4; with the cp.async ring below, 4 warps
+// are faster, since 8 rings leave room for only three operand stages.
 #ifndef LMLP_PAIR_EPI_WARPS_BF16
 #define LMLP_PAIR_EPI_WARPS_BF16 4
 #endif
@@ -56,7 +54,7 @@ constexpr uint32_t kPairTmemCols = 512;                                 // 2 buf
 #define LMLP_PAIR_EPI_WARPS_FWD 4
 #endif
 #ifndef LMLP_PAIR_EPI_WARPS_BWD
-#define LMLP_PAIR_EPI_WARPS_BWD 8
+#define LMLP_PAIR_EPI_WARPS_BWD 4
 #endif
 static_assert(LMLP_PAIR_EPI_WARPS_BF16 % 4 == 0 && LMLP_PAIR_EPI_WARPS_BF16 <= 8, "4 or 8 epilogue warps");
 static_assert(LMLP_PAIR_EPI_WARPS_FWD % 4 == 0 && LMLP_PAIR_EPI_WARPS_FWD <= 8, "4 or 8 epilogue warps");
@@ -69,6 +67,24 @@ __host__ __device__ constexpr int pair_epi_warps() {
 template <int EPI>
 __host__ __device__ constexpr int pair_threads() {
     return (2 + pair_epi_warps<EPI>()) * 32;
+}
+// The dH epilogue's g and u stream through a per-warp ring of shared-memory
+// slots filled by cp.async, LMLP_BWD_GU_RING chunks deep: the next chunk (at
+// a tile's end, the next tile's first) is in flight while one computes, no
+// registers hold it, and it lands row-major with no transpose.  0 loads g and
+// u into registers instead.  Measured interleaved on the dH GEMM against the
+// register path: TinyLlama-1.1B shapes 1027 -> 812 us, Qwen2-7B 1047 -> 1010
+// us, Llama-3-8B within noise (476 -> 468 us).  Deeper rings (3, 4 chunks)
+// cost an operand stage and measured slower on two of the three shapes.
+#ifndef LMLP_BWD_GU_RING
+#define LMLP_BWD_GU_RING 2
+#endif
+constexpr int kGuRing = LMLP_BWD_GU_RING;
+static_assert(kGuRing == 0 || kGuRing >= 2, "a ring holds at least two chunks");
+constexpr uint32_t kGuSlotBytes = 2 * kStageWarpBytes;  // g then u of one 32 x 32 chunk, 80-byte rows
+template <int EPI>
+__host__ __device__ constexpr uint32_t pair_ring_bytes() {
+    return (EPI == EPI_SWIGLU_BWD && kGuRing > 0) ? pair_epi_warps<EPI>() * kGuRing * kGuSlotBytes : 0u;
 }
 // Named barrier 1 over the epilogue warps.
 template <int EPI>
@@ -264,9 +280,131 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     }
 }
 
+// The dH + SwiGLU-backward epilogue with g and u streamed through the
+// warp's cp.async ring.  The warp walks the same (unit, chunk) sequence twice:
+// an issue cursor kGuRing - 1 chunks ahead fills ring slots (zeros outside
+// the matrix), and the consumer reads its row of each chunk back from shared
+// memory.  Each chunk is one cp.async group, so waiting until kGuRing - 1
+// groups remain in flight means the oldest chunk has landed.
+template <int EPI>
+__device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32_t tmem_base, uint32_t rank,
+                                                       const SmemCtl& c) {
+    const PairProb& P = a.prob;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int quarter = warp & 3;
+    constexpr int kGroups = pair_epi_warps<EPI>() / 4;
+    const int group = (warp - 2) >> 2;
+    const int gcols = 256 / kGroups;
+    const int gcol0 = group * gcols;
+    const int nch = gcols >> 5;
+    const uint32_t area = (c.full + gemm_ctl_bytes() + 127u) & ~127u;
+    const uint32_t stg = area + static_cast<uint32_t>(warp - 2) * kStageWarpBytes;
+    const uint32_t ring = area + pair_epi_warps<EPI>() * kStageWarpBytes +
+                          static_cast<uint32_t>(warp - 2) * (kGuRing * kGuSlotBytes);
+    const __nv_bfloat16* gbase = static_cast<const __nv_bfloat16*>(P.in0);
+    const __nv_bfloat16* ubase = static_cast<const __nv_bfloat16*>(P.in1);
+    if (a.force_timeout) {
+        wait_or_abort(c.never, 0, c);
+        return;
+    }
+    // issue cursor: unit iu, chunk ich, its first row and column, next slot
+    int iu = cid, ich = 0, irow0 = 0, icol0 = 0;
+    uint32_t islot = 0;
+    auto set_unit = [&]() {
+        if (iu < a.total_units) {
+            const PairUnit ti = pair_decode(a, iu);
+            irow0 = ti.mb * kPairBM + static_cast<int>(rank) * kBM + quarter * 32;
+            icol0 = ti.nb * P.tile_n + gcol0;
+        }
+    };
+    // 16-byte piece (row 8q + lane/4, columns 8 (lane%4) ..) of a chunk, as in
+    // a coalesced load: four lanes cover one row's 64 bytes.
+    const int prow = lane >> 2, pcol = 8 * (lane & 3);
+    const uint32_t poff = static_cast<uint32_t>(prow) * kStageRowBytes + static_cast<uint32_t>(lane & 3) * 16u;
+    auto issue = [&]() {
+        if (iu < a.total_units) {
+            const uint32_t sb = ring + islot * kGuSlotBytes + poff;
+            const int cc = icol0 + ich * 32 + pcol;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = irow0 + 8 * q + prow;
+                const bool ok = r < P.M && cc < P.N;
+                const long long off = ok ? static_cast<long long>(r) * P.ld + cc : 0;
+                cp_async16(sb + q * 8 * kStageRowBytes, gbase + off, ok ? 16u : 0u);
+                cp_async16(sb + kStageWarpBytes + q * 8 * kStageRowBytes, ubase + off, ok ? 16u : 0u);
+            }
+            if (++ich == nch) {
+                ich = 0;
+                iu += ncl;
+                set_unit();
+            }
+        }
+        cp_async_commit();
+        if (++islot == static_cast<uint32_t>(kGuRing)) islot = 0;
+    };
+    set_unit();
+#pragma unroll 1
+    for (int k = 0; k < kGuRing - 1; ++k) issue();
+
+    int abuf = 0;
+    uint32_t aphase = 0;
+    uint32_t cslot = 0;
+    for (int u = cid; u < a.total_units; u += ncl) {
+        const PairUnit t = pair_decode(a, u);
+        if (!wait_or_abort(c.accf + 8u * abuf, aphase, c)) {
+            cp_async_wait_all();
+            return;
+        }
+        tc_fence_after();
+        const int row = t.mb * kPairBM + static_cast<int>(rank) * kBM + quarter * 32 + lane;
+        const uint32_t tacc =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * 256u + static_cast<uint32_t>(gcol0);
+        for (int ch = 0; ch < nch; ++ch) {
+            issue();
+            cp_async_wait<(kGuRing > 0 ? kGuRing - 1 : 0)>();
+            __syncwarp();
+            const int col0 = t.nb * P.tile_n + gcol0 + ch * 32;
+            if (col0 < P.N) {  // warp-uniform
+                uint32_t v[32];
+                tmem_ld32(tacc + ch * 32, v);
+                const uint32_t rb = ring + cslot * kGuSlotBytes + static_cast<uint32_t>(lane) * kStageRowBytes;
+                uint4 gv[4], uv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    gv[q] = lds128(rb + q * 16);
+                    uv[q] = lds128(rb + kStageWarpBytes + q * 16);
+                }
+                tmem_ld_wait();
+                uint4 dgq[4], duq[4], hq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq[q], duq[q], hq[q]);
+                emit_chunk(static_cast<__nv_bfloat16*>(P.out0), P.ld, row, col0, P.M, P.N, dgq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(P.out1), P.ld, row, col0, P.M, P.N, duq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(P.out2), P.ld, row, col0, P.M, P.N, hq, stg);
+            }
+            __syncwarp();
+            if (++cslot == static_cast<uint32_t>(kGuRing)) cslot = 0;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(c.acce + 8u * abuf, 0));
+        if (++abuf == 2) {
+            abuf = 0;
+            aphase ^= 1u;
+        }
+    }
+    cp_async_wait_all();
+}
+
 template <int EPI>
 __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_base, uint32_t rank,
                                               const SmemCtl& c) {
+    if constexpr (EPI == EPI_SWIGLU_BWD && kGuRing > 0) {
+        pair_epilogue_bwd_ring<EPI>(a, tmem_base, rank, c);
+        return;
+    }
     constexpr int NACC = EPI == EPI_SWIGLU_FWD ? 2 : 1;
     const PairProb& P = a.prob;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
