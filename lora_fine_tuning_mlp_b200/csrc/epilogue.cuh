@@ -138,9 +138,6 @@ struct PartialSrc {
     }
 };
 
-// One output tile row per thread: `row` (may be >= M: stores are skipped),
-// columns [col_base, col_base + bn); accumulator a's column c is read from
-// `src` at a*bn + c.
 // SwiGLU backward for 8 consecutive columns: dH (fp32) with g, u (bf16 pairs).
 __device__ __forceinline__ void swiglu_bwd8(const uint32_t* dh, const uint4& gq, const uint4& uq, uint4& dgq,
                                             uint4& duq, uint4& hq) {
@@ -217,13 +214,52 @@ __device__ __forceinline__ void emit_chunk(__nv_bfloat16* base, long long ld, in
     }
 }
 
+// TMA stores of 32 x 32 bf16 output blocks.  Each epilogue warp owns three
+// 2 KB shared-memory buffers (512-byte aligned; rows of 64 bytes in the
+// 64-byte swizzle: 16-byte piece q of row r sits at piece q ^ ((r / 2) % 4),
+// so the 32 lanes' row writes hit every bank once per quarter-warp) used in
+// turn; a buffer is rewritten only once the store issued from it three
+// stores earlier has read it.  The tensor map clips rows and columns outside
+// the output.  Warp-uniform state.
+constexpr uint32_t kTmaBlockBytes = 32 * 64;
+constexpr uint32_t kTmaWarpBytes = 3 * kTmaBlockBytes;
+struct TmaStore {
+    const CUtensorMap* map[3];  // out0, out1, out2
+    uint32_t buf;               // this warp's three buffers
+    int next;                   // buffer of the next store
+    // Warp-collective: output `which`, the warp's 32 rows starting at row y
+    // (lane = row; v = its 32 values), columns x .. x + 31.
+    __device__ __forceinline__ void emit(int which, int x, int y, const uint4 (&v)[4]) {
+        const int lane = threadIdx.x & 31;
+        const uint32_t b = buf + static_cast<uint32_t>(next) * kTmaBlockBytes;
+        if (++next == 3) next = 0;
+        if (lane == 0) bulk_wait_read<2>();
+        __syncwarp();
+        const uint32_t rowb = b + static_cast<uint32_t>(lane) * 64u;
+        const uint32_t sw = static_cast<uint32_t>(lane >> 1) & 3u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sts128(rowb + ((static_cast<uint32_t>(q) ^ sw) << 4), v[q]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map[which], b, x, y);
+            bulk_commit();
+        }
+    }
+    // Warp-collective: every store issued so far has completed.
+    __device__ __forceinline__ void drain() const {
+        if ((threadIdx.x & 31) == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+};
+
 // One output tile row per thread: `row` (may be >= M: stores are skipped),
 // columns [col_base, col_base + bn); accumulator a's column c is read from
 // `src` at a*acc_stride + c.  `stg`: this warp's staging area (0 = store
-// directly).
+// directly); `ts`: TMA stores instead (bf16 outputs).
 template <int NACC, int EPI, class Src, bool kPrefetchGU = true>
 __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_base, int bn, const Src& src,
-                                              uint32_t stg = 0, int acc_stride = -1) {
+                                              uint32_t stg = 0, int acc_stride = -1, TmaStore* ts = nullptr) {
     // acc_stride: distance in src columns between the two accumulators
     // (default: bn, when a call covers all of a tile's columns)
     if (acc_stride < 0) acc_stride = bn;
@@ -281,9 +317,15 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             uint4 dgq[4], duq[4], hq[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) swiglu_bwd8(v + 8 * q, gv[q], uv[q], dgq[q], duq[q], hq[q]);
-            emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, dgq, stg);
-            emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, duq, stg);
-            emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
+            if (ts != nullptr) {
+                ts->emit(0, col0, row0, dgq);
+                ts->emit(1, col0, row0, duq);
+                ts->emit(2, col0, row0, hq);
+            } else {
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, dgq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, duq, stg);
+                emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
+            }
             if constexpr (kPrefetchGU) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -307,7 +349,10 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                     w[q].z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
                     w[q].w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
                 }
-                emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, w, stg);
+                if (ts != nullptr)
+                    ts->emit(0, col0, row - (threadIdx.x & 31), w);
+                else
+                    emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, w, stg);
             } else if constexpr (EPI == EPI_F32) {
 #pragma unroll
                 for (int acc = 0; acc < NACC; ++acc) {
@@ -344,9 +389,16 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
                     uq[q] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
                     hq[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 }
-                emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, gq, stg);
-                emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, uq, stg);
-                emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
+                if (ts != nullptr) {
+                    const int row0 = row - (threadIdx.x & 31);
+                    ts->emit(0, col0, row0, gq);
+                    ts->emit(1, col0, row0, uq);
+                    ts->emit(2, col0, row0, hq);
+                } else {
+                    emit_chunk(static_cast<__nv_bfloat16*>(o.out0), o.ld, row, col0, o.M, o.N, gq, stg);
+                    emit_chunk(static_cast<__nv_bfloat16*>(o.out1), o.ld, row, col0, o.M, o.N, uq, stg);
+                    emit_chunk(static_cast<__nv_bfloat16*>(o.out2), o.ld, row, col0, o.M, o.N, hq, stg);
+                }
             }
         }
     }

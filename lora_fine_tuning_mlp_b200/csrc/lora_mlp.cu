@@ -169,7 +169,7 @@ EncodeTiledFn encode_fn() {
 // (row stride ld elements) with a box_inner x box_outer box.  Out-of-range
 // elements of a box read as zero.
 bool encode_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t box_inner,
-                uint32_t box_outer) {
+                uint32_t box_outer, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
@@ -177,7 +177,7 @@ bool encode_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, i
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -386,6 +386,17 @@ struct PairBuilder {
     }
     int a_k(const void* p, int64_t rows, int64_t K, int64_t ld) { return map(p, K, rows, ld, kBK, kBM); }
     int b_k(const void* p, int64_t Nn, int64_t K, int64_t ld) { return map(p, K, Nn, ld, kBK, kPairHalfN); }
+    // bf16 output [M, N] (row stride prob.ld) as 32 x 32 blocks in the 64-byte
+    // swizzle, for the epilogue's TMA stores.
+    int out_map(const void* p) {
+        if (nmaps >= kMaxMaps) {
+            ok = false;
+            return 0;
+        }
+        if (!encode_map(&a.maps[nmaps], p, a.prob.N, a.prob.M, a.prob.ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            ok = false;
+        return nmaps++;
+    }
     int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
     void seg(int amap, int b0, int b1, int row0, int row1, int k0, int k1, int64_t k_len) {
         PairProb& p = a.prob;
@@ -422,6 +433,13 @@ int pair_tail_splits(int tiles, int clusters, int nkb) {
 
 template <bool B_MN, int EPI>
 int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, float* tail_part, int* tail_ctr) {
+    if constexpr (pair_tma_store<EPI>()) {
+        b.a.prob.omap[0] = b.out_map(b.a.prob.out0);
+        if (EPI != EPI_BF16) {
+            b.a.prob.omap[1] = b.out_map(b.a.prob.out1);
+            b.a.prob.omap[2] = b.out_map(b.a.prob.out2);
+        }
+    }
     if (!b.ok) return LORA_MLP_ERR_CUDA;
     PairArgs& a = b.a;
     a.nmaps = b.nmaps;
@@ -431,8 +449,8 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_splits = 1;
     a.tail_part = tail_part;
     a.tail_ctr = tail_ctr;
-    // epilogue store staging per warp, then the dH epilogue's g/u rings
-    const uint32_t staging = 128 + pair_epi_warps<EPI>() * kStageWarpBytes + pair_ring_bytes<EPI>();
+    // (512-byte alignment) epilogue store staging per warp, then the dH epilogue's g/u rings
+    const uint32_t staging = 512 + pair_epi_warps<EPI>() * pair_stage_warp_bytes<EPI>() + pair_ring_bytes<EPI>();
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kPairStageBytes);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
