@@ -58,8 +58,10 @@ constexpr uint32_t kSmemLimit = 232448;  // max dynamic shared memory per block 
 #endif
 // The tail split pays off for launches with a plain bf16 store epilogue (the
 // down and dX GEMMs: -55 us and -15 us per step on the Llama-3-8B shapes,
-// measured interleaved) but not for the SwiGLU epilogues (+31 us, +39 us),
-// so those launches run without it.
+// measured interleaved) but not for the SwiGLU epilogues (+31 us, +39 us;
+// the gate/up GEMM again +2 % and +3 % on the Llama-3-8B and TinyLlama-1.1B
+// shapes with its TMA-store epilogue, in two or four K ranges), so those
+// launches run without it.
 #ifndef LMLP_TAIL_SPLIT_SWIGLU
 #define LMLP_TAIL_SPLIT_SWIGLU 0
 #endif
