@@ -431,6 +431,7 @@ def b200_arm(args, cfg):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     run_e2e(args.steps)
+    trainer.finish()  # the last step's gradients are home before the clock stops
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -482,7 +483,8 @@ def b200_arm(args, cfg):
             "e2e": {"value": replicas.job_throughput(N, args.steps, ems, world), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "what": "api.HostBatchTrainer: per step H2D of X and dOut from pinned host (overlapped with "
-                            "the previous step's compute), forward+backward, D2H of the six adapter grads"},
+                            "the previous step's compute), forward+backward, D2H of the six adapter grads "
+                            "(overlapped with the next step's compute)"},
             "gpu_launches": launches,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},

@@ -228,8 +228,11 @@ class HostBatchTrainer:
     """Forward + backward over batches that live in (pinned) host memory.
 
     The host-to-device copy of the next batch runs on its own stream while the
-    current batch computes (two device buffers, ordered by CUDA events), and
-    each step's adapter gradients are copied back to pinned host memory.
+    current batch computes, and each step's adapter gradients are copied back
+    to pinned host memory on a third stream while the next step computes.
+    Inputs and gradients are double-buffered on the device (and the
+    gradients on the host), ordered by CUDA events: a device buffer is
+    refilled only once the step that used it, or its copy back, is done.
     Every step still moves its own inputs and result across PCIe; only the
     overlap with compute is new.
     """
@@ -244,12 +247,18 @@ class HostBatchTrainer:
         self.dOut = [torch.empty((N, d), dtype=BF16, device=dev) for _ in range(2)]
         self.out = torch.empty((N, d), dtype=BF16, device=dev)
         self.dX = torch.empty((N, d), dtype=BF16, device=dev)
-        self.grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
-        self.grads_host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in self.grads.items()}
+        names = ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")
+        self.grads = [{("d" + k): torch.empty_like(getattr(w, k)) for k in names} for _ in range(2)]
+        self.grads_host = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in g.items()}
+                           for g in self.grads]
         self.wsf, self.wsb = Workspace(), Workspace()
         self.copy_stream = torch.cuda.Stream(device=dev)
+        self.d2h_stream = torch.cuda.Stream(device=dev)
         self.ready = [torch.cuda.Event(), torch.cuda.Event()]
         self.free = [torch.cuda.Event(), torch.cuda.Event()]
+        self.computed = [torch.cuda.Event(), torch.cuda.Event()]
+        self.fetched = [torch.cuda.Event(), torch.cuda.Event()]
+        self.fetch_pending = [False, False]
         self.slot = 0
         self.primed = False
 
@@ -264,13 +273,14 @@ class HostBatchTrainer:
         return 2 * self.N * self.w.d * 2
 
     def d2h_bytes(self) -> int:
-        return sum(v.numel() * v.element_size() for v in self.grads.values())
+        return sum(v.numel() * v.element_size() for v in self.grads[0].values())
 
     def step(self, Xh, dOh, next_Xh=None, next_dOh=None):
         """One training step on host batch (Xh, dOh); if the next batch is
         given, its copy is started so that it overlaps this step's compute.
-        Returns the dict of pinned host adapter gradients (valid once the
-        current stream has been synchronised)."""
+        Returns the dict of pinned host adapter gradients of this step: valid
+        after `finish()` and a synchronisation of the current stream (or the
+        device), and until the step after next overwrites them."""
         cur = self.slot
         if not self.primed:
             self._stage(cur, Xh, dOh)
@@ -280,20 +290,35 @@ class HostBatchTrainer:
             self._stage(nxt, next_Xh, next_dOh)
         stream = torch.cuda.current_stream(self.dev)
         stream.wait_event(self.ready[cur])
+        if self.fetch_pending[cur]:
+            stream.wait_event(self.fetched[cur])  # this slot's gradients from two steps ago are home
+        grads = self.grads[cur]
         if self.gamma is None:
             o, saved = forward(self.X[cur], self.w, out=self.out, workspace=self.wsf)
-            backward(self.X[cur], self.w, saved, self.dOut[cur], dX=self.dX, grads=self.grads, workspace=self.wsb)
+            backward(self.X[cur], self.w, saved, self.dOut[cur], dX=self.dX, grads=grads, workspace=self.wsb)
         else:
             o, saved = block_forward(self.X[cur], self.w, self.gamma, self.eps, out=self.out, workspace=self.wsf)
-            block_backward(self.X[cur], self.w, self.gamma, saved, self.dOut[cur], dX=self.dX, grads=self.grads,
+            block_backward(self.X[cur], self.w, self.gamma, saved, self.dOut[cur], dX=self.dX, grads=grads,
                            workspace=self.wsb)
         self.free[cur].record(stream)
-        for k, v in self.grads.items():
-            self.grads_host[k].copy_(v, non_blocking=True)
+        self.computed[cur].record(stream)
+        with torch.cuda.stream(self.d2h_stream):
+            self.d2h_stream.wait_event(self.computed[cur])
+            for k, v in grads.items():
+                self.grads_host[cur][k].copy_(v, non_blocking=True)
+            self.fetched[cur].record(self.d2h_stream)
+        self.fetch_pending[cur] = True
         self.slot = nxt
         if next_Xh is None:
             self.primed = False
-        return self.grads_host
+        return self.grads_host[cur]
+
+    def finish(self):
+        """Orders the current stream after every gradient copy issued so far."""
+        stream = torch.cuda.current_stream(self.dev)
+        for i in range(2):
+            if self.fetch_pending[i]:
+                stream.wait_event(self.fetched[i])
 
 
 # ----------------------------------------------------------------------------- LoRA linear
