@@ -737,6 +737,46 @@ int check_weights(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
 // buffer, or for int4 weights a just-in-time dequantisation into workspace
 // buffer `slot` (two buffers serve the whole pass: gate and up together,
 // then down).
+// int4 frozen weights: the dequantisation launches run on a side stream, so
+// that each overlaps a launch that does not read its buffer (fork and join
+// through events; the caller's stream stays the only one it has to order).
+#ifndef LMLP_INT4_OVERLAP
+#define LMLP_INT4_OVERLAP 1
+#endif
+
+// One non-blocking side stream per device, created on first use.
+int side_stream(cudaStream_t* out) {
+    static cudaStream_t streams[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_MLP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        return LORA_MLP_ERR_CUDA;
+    *out = streams[dev];
+    return LORA_MLP_OK;
+}
+
+// The events of one call's fork/join edges, released when the call returns
+// (a pending event is released by CUDA once it completes).
+struct StreamLinks {
+    cudaEvent_t ev[8] = {};
+    int n = 0;
+    ~StreamLinks() {
+        for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+    }
+    // `to` waits for everything issued to `from` so far.
+    int link(cudaStream_t from, cudaStream_t to) {
+        if (n >= 8) return LORA_MLP_ERR_CUDA;
+        cudaEvent_t& e = ev[n];
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+        ++n;
+        if (cudaEventRecord(e, from) != cudaSuccess || cudaStreamWaitEvent(to, e, 0) != cudaSuccess)
+            return LORA_MLP_ERR_CUDA;
+        return LORA_MLP_OK;
+    }
+};
+
 int frozen_weight(const Plan& pl, const lora_mlp_weights* w, int which, uint8_t* ws, const size_t* off, int slot,
                   int sms, cudaStream_t st, const void** out) {
     const void* bf[3] = {w->Wg, w->Wu, w->Wd};
@@ -789,6 +829,17 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
     const void* W[3] = {nullptr, nullptr, nullptr};
+    // int4: Wg, Wu dequantised beside F0; Wd (into Wg's buffer, once F1 is
+    // done with it) beside F2
+    const bool overlap = pl.int4 && LMLP_INT4_OVERLAP;
+    cudaStream_t qs = st;
+    StreamLinks links;
+    if (overlap) {
+        LMLP_TRY(side_stream(&qs));
+        LMLP_TRY(links.link(st, qs));
+        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, qs, &W[0]));
+        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, qs, &W[1]));
+    }
 
     {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
@@ -804,8 +855,12 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
         LMLP_TRY((launch_gemm<2, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
-    LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, st, &W[0]));
-    LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, st, &W[1]));
+    if (overlap) {
+        LMLP_TRY(links.link(qs, st));
+    } else {
+        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, st, &W[0]));
+        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, st, &W[1]));
+    }
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
         PairBuilder b(N, dff, 128);
         const int ax = b.a_k(X, N, d, d);
@@ -822,6 +877,10 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.ld = dff;
         LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
     }
+    if (overlap) {
+        LMLP_TRY(links.link(st, qs));
+        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, qs, &W[2]));
+    }
     {  // F2: S_d = s h Ad^T  -> Sd [N, r] and saved S_d^T [r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ah = b.a_k(h, N, dff, dff);
@@ -834,7 +893,10 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(r), Sd, r, sv + pl.s_sdT, nullptr, pl.ldN, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
     }
-    LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, st, &W[2]));
+    if (overlap)
+        LMLP_TRY(links.link(qs, st));
+    else
+        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, st, &W[2]));
     {  // F3: out = h Wd^T + S_d Bd^T
         PairBuilder b(N, d, 256);
         const int ah = b.a_k(h, N, dff, dff);
@@ -881,6 +943,16 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
     const void* W[3] = {nullptr, nullptr, nullptr};
+    // int4: Wd dequantised beside B0; Wg (into the second buffer) beside B1;
+    // Wu (into Wd's buffer, once B1 is done with it) beside B-mid
+    const bool overlap = pl.int4 && LMLP_INT4_OVERLAP;
+    cudaStream_t qs = st;
+    StreamLinks links;
+    if (overlap) {
+        LMLP_TRY(side_stream(&qs));
+        LMLP_TRY(links.link(st, qs));
+        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, qs, &W[2]));
+    }
 
     // adapter B matrices as K-major operands of the rank-r projections
     {  // B0: T_d = s dOut Bd -> Td [N, r], Td^T [r, ldN];  dBd = dOut^T S_d
@@ -904,7 +976,12 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.fin(p1, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B0_lowrank_out_dBd", ctr)));
     }
-    LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, st, &W[2]));
+    if (overlap) {
+        LMLP_TRY(links.link(qs, st));
+        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 1, di.sms, qs, &W[0]));
+    } else {
+        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, st, &W[2]));
+    }
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
         PairBuilder b(N, dff, 256);
         const int a = b.a_k(dOut, N, d, d);
@@ -921,6 +998,10 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p.out2 = hb;
         p.ld = dff;
         LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
+    }
+    if (overlap) {
+        LMLP_TRY(links.link(st, qs));
+        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 0, di.sms, qs, &W[1]));
     }
     {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
        //        dAd = T_d^T h (written transposed);  dBg = dg^T S_g, dBu = du^T S_u
@@ -978,8 +1059,12 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         });
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B_mid_lowrank_grads", ctr)));
     }
-    LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 0, di.sms, st, &W[0]));
-    LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 1, di.sms, st, &W[1]));
+    if (overlap) {
+        LMLP_TRY(links.link(qs, st));
+    } else {
+        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 0, di.sms, st, &W[0]));
+        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 1, di.sms, st, &W[1]));
+    }
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
         PairBuilder b(N, d, 256);
         const int adg = b.a_k(dg, N, dff, dff);

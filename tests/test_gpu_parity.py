@@ -180,6 +180,35 @@ def test_autograd_function_matches_api():
         assert np.array_equal(getattr(w, k).grad.float().double().cpu().numpy(), ref["d" + k]), k
 
 
+def test_host_batch_trainer_back_to_back_steps():
+    """Steps queued with no synchronisation in between: each step's gradient
+    copy back must follow its own backward and finish before the step after
+    next overwrites the device buffer, so the last two steps' host gradients
+    equal the device-resident results bit for bit."""
+    cfg_a = synth.custom(384, 256, 512, 16, 16.0, seed_index=36)
+    inputs = [synth.make_inputs(synth.custom(384, 256, 512, 16, 16.0, seed_index=36 + i)) for i in range(3)]
+    dev = torch.device("cuda:0")
+    w = api.weights_from_host(inputs[0], cfg_a.alpha, dev)
+    host = [(torch.from_numpy(i["X"].view("int16")).view(torch.bfloat16).pin_memory(),
+             torch.from_numpy(i["dOut"].view("int16")).view(torch.bfloat16).pin_memory()) for i in inputs]
+    trainer = api.HostBatchTrainer(w, cfg_a.N, dev)
+    order = [0, 1, 2, 1, 0]
+    returned = []
+    for i, b in enumerate(order):
+        nxt = host[order[i + 1]] if i + 1 < len(order) else (None, None)
+        returned.append(trainer.step(host[b][0], host[b][1], nxt[0], nxt[1]))
+    trainer.finish()
+    torch.cuda.synchronize()
+    for i in (len(order) - 2, len(order) - 1):
+        X = host[order[i]][0].to(dev)
+        dOut = host[order[i]][1].to(dev)
+        _, saved = api.forward(X, w)
+        _, ref = api.backward(X, w, saved, dOut)
+        torch.cuda.synchronize()
+        for k in ref:
+            assert torch.equal(returned[i][k], ref[k].cpu()), (i, k)
+
+
 def test_host_batch_trainer_matches_device_path():
     """Host batches through the overlapped-copy trainer give the same gradients
     as the device-resident calls, batch after batch."""
