@@ -214,15 +214,16 @@ __device__ __forceinline__ void emit_chunk(__nv_bfloat16* base, long long ld, in
     }
 }
 
-// TMA stores of 32 x 32 bf16 output blocks.  Each epilogue warp owns three
-// 2 KB shared-memory buffers (512-byte aligned; rows of 64 bytes in the
+// TMA stores of 32 x 32 bf16 output blocks.  Each epilogue warp owns
+// kTmaBufs 2 KB shared-memory buffers (512-byte aligned; rows of 64 bytes in the
 // 64-byte swizzle: 16-byte piece q of row r sits at piece q ^ ((r / 2) % 4),
 // so the 32 lanes' row writes hit every bank once per quarter-warp) used in
-// turn; a buffer is rewritten only once the store issued from it three
+// turn; a buffer is rewritten only once the store issued from it kTmaBufs
 // stores earlier has read it.  The tensor map clips rows and columns outside
 // the output.  Warp-uniform state.
+constexpr int kTmaBufs = 3;
 constexpr uint32_t kTmaBlockBytes = 32 * 64;
-constexpr uint32_t kTmaWarpBytes = 3 * kTmaBlockBytes;
+constexpr uint32_t kTmaWarpBytes = kTmaBufs * kTmaBlockBytes;
 struct TmaStore {
     const CUtensorMap* map[3];  // out0, out1, out2
     uint32_t buf;               // this warp's three buffers
@@ -232,8 +233,8 @@ struct TmaStore {
     __device__ __forceinline__ void emit(int which, int x, int y, const uint4 (&v)[4]) {
         const int lane = threadIdx.x & 31;
         const uint32_t b = buf + static_cast<uint32_t>(next) * kTmaBlockBytes;
-        if (++next == 3) next = 0;
-        if (lane == 0) bulk_wait_read<2>();
+        if (++next == kTmaBufs) next = 0;
+        if (lane == 0) bulk_wait_read<kTmaBufs - 1>();  // this buffer's last store has read it
         __syncwarp();
         const uint32_t rowb = b + static_cast<uint32_t>(lane) * 64u;
         const uint32_t sw = static_cast<uint32_t>(lane >> 1) & 3u;
