@@ -45,7 +45,7 @@ using namespace lmlp;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a layout constant  // split-K sizing target (B200 SM count); a layout constant
+constexpr int kTargetCtas = 148;  // split-K sizing target (B200 SM count); a layout constant
 constexpr int kMaxSplits = 32;
 constexpr size_t kAlign = 256;
 constexpr uint32_t kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
