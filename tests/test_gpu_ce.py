@@ -4,7 +4,7 @@ vocabularies, sampled rows of the 256K-vocabulary workload, and the edge
 cases (one logit, chunk boundaries, padded rows, ignored rows, masked and
 extreme logits, in-place gradient, determinism, a bad label).
 
-Tolerances (derived in the design doc): loss and lse within 1e-4 + 1e-5 |ref|
+Tolerances, from the arithmetic: loss and lse within 1e-4 + 1e-5 |ref|
 (fp32 sums of up to 2^18 exponentials); each gradient element within
 2^-8 |ref| (its bf16 rounding, doubled) + 1e-5 * dloss * s (the fp32 error
 of exp(t - lse) near the label's 1); and max|diff| / max|ref| <= 2e-2 per
