@@ -143,3 +143,79 @@ def test_lora_linear_writes_every_output_and_nothing_past_it():
         runs.append(res)
     for k in runs[0]:
         assert torch.equal(runs[0][k].view(torch.int16), runs[1][k].view(torch.int16)), k
+
+
+@pytest.mark.parametrize("name,ld_pad", [("ce_tiny", 5), ("ce_tiny_softcap", 0)])
+def test_cross_entropy_writes_every_output_and_nothing_past_it(name, ld_pad):
+    """loss and lse for every row, dlogits for every valid column (the padding
+    columns of a row are not the kernel's), nothing past any buffer, and the
+    same bits from poisoned and zeroed buffers."""
+    import numpy as np
+
+    cfg = synth.CE_BY_NAME[name]
+    inp = synth.make_ce_inputs(cfg)
+    N, V = inp["logits"].shape
+    ld = (V + 7) // 8 * 8 + 8 * ld_pad
+    dev = torch.device("cuda:0")
+    z = torch.zeros((N, ld), dtype=torch.int16)
+    z[:, :V] = torch.from_numpy(inp["logits"].view(np.int16))
+    z = z.view(torch.bfloat16).to(dev)
+    lab = torch.from_numpy(np.asarray(inp["labels"], dtype=np.int64)).to(dev)
+    dl = torch.from_numpy(np.asarray(inp["dloss"], dtype=np.float32)).to(dev)
+    shape = _lib.make_ce_shape(N, V, ld, cfg.logit_scale, cfg.softcap, synth.CE_IGNORE_INDEX)
+    wsb = _lib.ce_sizes(shape)
+    runs = []
+    for body in (0xFF, 0x00):
+        loss = Carved(N * 4, body, dev)
+        lse = Carved(N * 4, body, dev)
+        ws = Carved(wsb, body, dev)
+        dz = Carved(N * ld * 2, body, dev)
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        _lib.check(_lib.ce_forward(shape, ctypes.c_void_p(z.data_ptr()), ctypes.c_void_p(lab.data_ptr()),
+                                   loss.ptr(), lse.ptr(), ws.ptr(), wsb, stream), "lora_ce_forward")
+        _lib.check(_lib.ce_backward(shape, ctypes.c_void_p(z.data_ptr()), ctypes.c_void_p(lab.data_ptr()),
+                                    lse.ptr(), ctypes.c_void_p(dl.data_ptr()), dz.ptr(), stream), "lora_ce_backward")
+        torch.cuda.synchronize()
+        res = {"loss": loss.buf[: N * 4].view(torch.float32), "dlogits": dz.bf16((N, ld))[:, :V]}
+        valid = lab != synth.CE_IGNORE_INDEX
+        res["lse"] = lse.buf[: N * 4].view(torch.float32)[valid]
+        for k, t in res.items():
+            assert not torch.isnan(t).any(), f"{k}: elements left unwritten"
+        for k, c in {"loss": loss, "lse": lse, "workspace": ws, "dlogits": dz}.items():
+            assert c.guard_ok(), f"{k}: written past its end"
+        runs.append({k: v.clone() for k, v in res.items()})
+    for k in runs[0]:
+        assert torch.equal(runs[0][k].view(torch.int16) if runs[0][k].dtype == torch.bfloat16 else runs[0][k],
+                           runs[1][k].view(torch.int16) if runs[1][k].dtype == torch.bfloat16 else runs[1][k]), k
+
+
+def test_rmsnorm_writes_every_output_and_nothing_past_it():
+    import numpy as np
+
+    dev = torch.device("cuda:0")
+    rng = np.random.default_rng(47)
+    for N, d in ((3, 136), (257, 4096), (5, 20480)):   # one-row-per-CTA and wide-row kernels
+        x = torch.from_numpy(rng.standard_normal((N, d)).astype(np.float32)).to(torch.bfloat16).to(dev)
+        gamma = torch.from_numpy(rng.uniform(0.5, 1.5, d).astype(np.float32)).to(torch.bfloat16).to(dev)
+        dy = torch.from_numpy(rng.standard_normal((N, d)).astype(np.float32)).to(torch.bfloat16).to(dev)
+        runs = []
+        for body in (0xFF, 0x00):
+            y = Carved(N * d * 2, body, dev)
+            rstd = Carved(N * 4, body, dev)
+            dx = Carved(N * d * 2, body, dev)
+            stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+            p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+            _lib.check(_lib.rmsnorm_forward(N, d, 1e-5, p(x), p(gamma), y.ptr(), rstd.ptr(), stream),
+                       "lora_rmsnorm_forward")
+            _lib.check(_lib.rmsnorm_backward(N, d, p(x), p(gamma), rstd.ptr(), p(dy), dx.ptr(), stream),
+                       "lora_rmsnorm_backward")
+            torch.cuda.synchronize()
+            res = {"y": y.bf16((N, d)), "rstd": rstd.buf[: N * 4].view(torch.float32), "dx": dx.bf16((N, d))}
+            for k, t in res.items():
+                assert not torch.isnan(t).any(), f"{k} (N={N}, d={d}): elements left unwritten"
+            for k, c in {"y": y, "rstd": rstd, "dx": dx}.items():
+                assert c.guard_ok(), f"{k} (N={N}, d={d}): written past its end"
+            runs.append({k: v.clone().view(torch.int32 if v.dtype == torch.float32 else torch.int16)
+                         for k, v in res.items()})
+        for k in runs[0]:
+            assert torch.equal(runs[0][k], runs[1][k]), (k, N, d)
