@@ -297,12 +297,16 @@ def config_dict(cfg, block=False):
         d["workload"] = "llama3_8b_block" if cfg.name == "llama3_8b_mlp" else cfg.name + "_block"
         d["prenorm"] = f"RMSNorm (frozen gain), eps {synth.RMS_EPS}; out = MLP(RMSNorm(X))"
         return d
+    w_mb = 3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6
+    x_mb, h_mb = 2 * cfg.N * cfg.d / 1e6, 2 * cfg.N * cfg.d_ff / 1e6
+    sizes = "frozen weights %.0f MB, X %.0f MB, g/u/h %.0f MB each" % (w_mb, x_mb, h_mb)
+    # a step reads the weights, X, dOut and writes/reads g, u, h, dg, du
+    step_mb = w_mb + 2 * x_mb + 5 * h_mb
+    l2 = ("no flush: a step's operands exceed the 126 MB L2 (%s)" % sizes if step_mb > 126.0 else
+          "no flush; a step's operands fit in the 126 MB L2 (%s): a launch-bound parity case, not a "
+          "throughput workload" % sizes)
     return {"workload": cfg.name, "N_tokens": cfg.N, "d": cfg.d, "d_ff": cfg.d_ff, "r": cfg.r, "alpha": cfg.alpha,
-            "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
-            "l2": "no flush: a step's operands exceed the 126 MB L2 (frozen weights %.0f MB, X %.0f MB, "
-                  "g/u/h %.0f MB each)" % (3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6,
-                                            2 * cfg.N * cfg.d / 1e6, 2 * cfg.N * cfg.d_ff / 1e6),
-            "parallelism": "replicas"}
+            "frozen_weights": "int4_b64" if cfg.int4 else "bf16", "l2": l2, "parallelism": "replicas"}
 
 
 def b200_arm(args, cfg):
