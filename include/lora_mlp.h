@@ -48,7 +48,9 @@ extern "C" {
 #endif
 
 #define LORA_MLP_OK 0
-#define LORA_MLP_ERR_INVALID_ARG (-1)         /* null pointer, non-positive size, non-finite alpha */
+#define LORA_MLP_ERR_INVALID_ARG (-1)         /* null pointer, memory that is not the current device's
+                                                 (host, another device's, unknown), non-positive size,
+                                                 non-finite alpha */
 #define LORA_MLP_ERR_UNSUPPORTED_SHAPE (-2)   /* divisibility or range rule above violated        */
 #define LORA_MLP_ERR_MISALIGNED (-3)          /* a device pointer is not 16-byte aligned          */
 #define LORA_MLP_ERR_WORKSPACE_TOO_SMALL (-4) /* workspace_bytes below lora_mlp_sizes()           */
@@ -125,6 +127,16 @@ int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, 
  * 0, or LORA_MLP_ERR_DEVICE_TIMEOUT if any kernel gave up a bounded wait since
  * the last call.  Synchronises `stream`. */
 int lora_mlp_device_status(void* stream, int* status);
+
+/* The check every entry point applies to each pointer argument, on its own
+ * (no launch): LORA_MLP_ERR_INVALID_ARG for NULL or for memory that is not
+ * device or managed memory of the current device (pageable or page-locked
+ * host memory, another device's memory, an address CUDA does not know);
+ * LORA_MLP_ERR_MISALIGNED when p is not a multiple of `alignment` bytes
+ * (0 or 1: no alignment check); else LORA_MLP_OK.  The entry points make it
+ * after their other argument checks and before enqueueing anything, so a
+ * host pointer is refused instead of reaching a kernel. */
+int lora_mlp_check_pointer(const void* p, size_t alignment);
 
 /* Human-readable name of a return code (static string). */
 const char* lora_mlp_strerror(int code);

@@ -34,6 +34,7 @@ SYMBOLS = (
     "lora_mlp_backward",
     "lora_mlp_dequant_int4",
     "lora_mlp_device_status",
+    "lora_mlp_check_pointer",
     "lora_mlp_strerror",
     "lora_mlp_timing_enable",
     "lora_mlp_timing_collect",
@@ -115,6 +116,7 @@ def lib() -> ctypes.CDLL:
                                             vp, ctypes.POINTER(Grads), vp, sz, vp]
             L.lora_mlp_dequant_int4.argtypes = [vp, vp, i64, i64, vp, vp]
             L.lora_mlp_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+            L.lora_mlp_check_pointer.argtypes = [vp, sz]
             L.lora_mlp_strerror.argtypes = [ctypes.c_int]
             L.lora_mlp_strerror.restype = ctypes.c_char_p
             L.lora_mlp_timing_enable.argtypes = [ctypes.c_int]
@@ -146,7 +148,8 @@ def lib() -> ctypes.CDLL:
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
                          "lora_mlp_dequant_int4",
-                         "lora_mlp_device_status", "lora_mlp_timing_enable", "lora_mlp_timing_collect",
+                         "lora_mlp_device_status", "lora_mlp_check_pointer", "lora_mlp_timing_enable",
+                         "lora_mlp_timing_collect",
                          "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward",
                          "lora_rmsnorm_forward", "lora_rmsnorm_backward", "lora_mlp_block_sizes",
                          "lora_mlp_block_forward", "lora_mlp_block_backward", "lora_ce_sizes",
@@ -199,6 +202,11 @@ def backward(shape: Shape, weights: Weights, X, g, u, saved, dOut, dX, grads: Gr
 
 def dequant_int4(packed, scales, rows, cols, w_bf16, stream) -> int:
     return lib().lora_mlp_dequant_int4(packed, scales, int(rows), int(cols), w_bf16, stream)
+
+
+def check_pointer(ptr, alignment: int = 16) -> int:
+    """The entry points' pointer check on its own (no launch): a LORA_MLP code."""
+    return lib().lora_mlp_check_pointer(ptr, int(alignment))
 
 
 def device_status(stream) -> int:

@@ -727,6 +727,36 @@ int check_weights(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
     return LORA_MLP_OK;
 }
 
+// Memory the kernels may touch: device or managed memory of the current
+// device, as CUDA reports it.  Ordinary or page-locked host memory, another
+// device's memory and addresses CUDA does not know are refused on the host,
+// after the other argument checks and before anything is enqueued.
+bool device_memory(const void* p) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (at.type == cudaMemoryTypeManaged) return true;
+    return at.type == cudaMemoryTypeDevice && at.device == dev;
+}
+int check_memory(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!device_memory(p)) return LORA_MLP_ERR_INVALID_ARG;
+    return LORA_MLP_OK;
+}
+int check_weight_memory(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
+    const int rc = check_memory({w->Wg, w->Wu, w->Wd, w->Ag, w->Bg, w->Au, w->Bu, w->Ad, w->Bd});
+    if (rc != LORA_MLP_OK) return rc;
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_memory({w->Sg, w->Su, w->Sd});
+    return LORA_MLP_OK;
+}
+
 #define LMLP_TRY(expr)              \
     do {                            \
         const int rc_ = (expr);     \
@@ -815,6 +845,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     LMLP_TRY(check_ptrs({X, out, g, u, saved, workspace}));
     const Plan pl = make_plan(*shape);
     if (workspace_bytes < pl.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w));
+    LMLP_TRY(check_memory({X, out, g, u, saved, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -922,6 +954,9 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
                          grads->dAd, grads->dBd}));
     const Plan pl = make_plan(*shape);
     if (workspace_bytes < pl.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w));
+    LMLP_TRY(check_memory({X, g, u, saved, dOut, dX, workspace, grads->dAg, grads->dBg, grads->dAu, grads->dBu,
+                           grads->dAd, grads->dBd}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1103,9 +1138,16 @@ int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, 
     if (rows < 1 || cols < 1) return LORA_MLP_ERR_INVALID_ARG;
     if (cols % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     LMLP_TRY(check_ptrs({packed, scales, w_bf16}));
+    LMLP_TRY(check_memory({packed, scales, w_bf16}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     return launch_dequant(packed, scales, rows, cols, w_bf16, di.sms, static_cast<cudaStream_t>(stream));
+}
+
+int lora_mlp_check_pointer(const void* p, size_t alignment) {
+    if (p == nullptr) return LORA_MLP_ERR_INVALID_ARG;
+    if (alignment > 1 && reinterpret_cast<uintptr_t>(p) % alignment) return LORA_MLP_ERR_MISALIGNED;
+    return device_memory(p) ? LORA_MLP_OK : LORA_MLP_ERR_INVALID_ARG;
 }
 
 int lora_mlp_device_status(void* stream, int* status) {
@@ -1275,6 +1317,11 @@ int check_lin_weights(const lora_linear_shape* sh, const lora_linear_weights* w)
     if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_ptrs({w->S});
     return LORA_MLP_OK;
 }
+int check_lin_weight_memory(const lora_linear_shape* sh, const lora_linear_weights* w) {
+    LMLP_TRY(check_memory({w->W, w->A, w->B}));
+    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_memory({w->S});
+    return LORA_MLP_OK;
+}
 
 // The bf16 frozen weight: the caller's, or int4 dequantised into the workspace.
 int lin_frozen_weight(const LinPlan& pl, const lora_linear_weights* w, uint8_t* ws, size_t off, int sms,
@@ -1309,6 +1356,8 @@ int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weight
     LMLP_TRY(check_ptrs({X, Y, saved, workspace}));
     const LinPlan pl = make_lin_plan(*shape);
     if (workspace_bytes < pl.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_lin_weight_memory(shape, w));
+    LMLP_TRY(check_memory({X, Y, saved, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1357,6 +1406,8 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
     LMLP_TRY(check_ptrs({X, saved, dY, dX, dA, dB, workspace}));
     const LinPlan pl = make_lin_plan(*shape);
     if (workspace_bytes < pl.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_lin_weight_memory(shape, w));
+    LMLP_TRY(check_memory({X, saved, dY, dX, dA, dB, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1528,6 +1579,7 @@ int lora_rmsnorm_forward(int64_t N, int64_t d, float eps, const void* x, const v
     LMLP_TRY(validate_norm(N, d));
     if (!std::isfinite(eps) || eps < 0.0f) return LORA_MLP_ERR_INVALID_ARG;
     LMLP_TRY(check_ptrs({x, gamma, y, rstd}));
+    LMLP_TRY(check_memory({x, gamma, y, rstd}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     return launch_rmsnorm_fwd(N, d, eps, x, gamma, nullptr, static_cast<float*>(rstd), y, di.sms,
@@ -1538,6 +1590,7 @@ int lora_rmsnorm_backward(int64_t N, int64_t d, const void* x, const void* gamma
                           void* dx, void* stream) {
     LMLP_TRY(validate_norm(N, d));
     LMLP_TRY(check_ptrs({x, gamma, rstd, dy, dx}));
+    LMLP_TRY(check_memory({x, gamma, rstd, dy, dx}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     return launch_rmsnorm_bwd(N, d, x, gamma, static_cast<const float*>(rstd), dy, dx, di.sms,
@@ -1563,6 +1616,8 @@ int lora_mlp_block_forward(const lora_mlp_shape* shape, const lora_mlp_weights* 
     LMLP_TRY(check_ptrs({gamma, X, out, g, u, saved, workspace}));
     const BlockPlan b = make_block_plan(*shape);
     if (workspace_bytes < b.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w));
+    LMLP_TRY(check_memory({gamma, X, out, g, u, saved, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1582,6 +1637,8 @@ int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights*
     LMLP_TRY(check_ptrs({gamma, X, g, u, saved, dOut, dX, workspace}));
     const BlockPlan b = make_block_plan(*shape);
     if (workspace_bytes < b.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w));
+    LMLP_TRY(check_memory({gamma, X, g, u, saved, dOut, dX, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1669,6 +1726,7 @@ int lora_ce_forward(const lora_ce_shape* shape, const void* logits, const int64_
         return LORA_MLP_ERR_MISALIGNED;
     const CePlan pl = make_ce_plan(*shape);
     if (workspace_bytes < pl.total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_memory({logits, labels, loss, lse, workspace}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1697,6 +1755,7 @@ int lora_ce_backward(const lora_ce_shape* shape, const void* logits, const int64
     if (!aligned(logits, 16) || !aligned(dlogits, 16) || !aligned(labels, 8) || !aligned(lse, 4) ||
         !aligned(dloss, 4))
         return LORA_MLP_ERR_MISALIGNED;
+    LMLP_TRY(check_memory({logits, labels, lse, dloss, dlogits}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);

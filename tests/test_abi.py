@@ -129,6 +129,13 @@ def test_backward_argument_errors(L):
                                bws, None) == _lib.ERR_INVALID_ARG
 
 
+def test_pointer_check_without_gpu(L):
+    assert _lib.check_pointer(None) == _lib.ERR_INVALID_ARG
+    assert _lib.check_pointer(FAKE + 8, 16) == _lib.ERR_MISALIGNED
+    # an aligned address that no CUDA device owns (none here) is refused
+    assert _lib.check_pointer(FAKE, 16) == _lib.ERR_INVALID_ARG
+
+
 def test_dequant_argument_errors(L):
     assert _lib.dequant_int4(FAKE, FAKE, 4, 100, FAKE, None) == _lib.ERR_UNSUPPORTED_SHAPE
     assert _lib.dequant_int4(FAKE, FAKE, 0, 64, FAKE, None) == _lib.ERR_INVALID_ARG

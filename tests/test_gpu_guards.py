@@ -219,3 +219,36 @@ def test_rmsnorm_writes_every_output_and_nothing_past_it():
                          for k, v in res.items()})
         for k in runs[0]:
             assert torch.equal(runs[0][k], runs[1][k]), (k, N, d)
+
+
+def test_host_memory_is_refused_before_any_launch():
+    """The pointer check accepts device memory only; an entry point handed a
+    host pointer returns LORA_MLP_ERR_INVALID_ARG without enqueueing work."""
+    dev = torch.device("cuda:0")
+    pageable = torch.zeros(4096, dtype=torch.uint8)
+    pinned = torch.zeros(4096, dtype=torch.uint8).pin_memory()
+    device = torch.zeros(4096, dtype=torch.uint8, device=dev)
+    assert _lib.check_pointer(pageable.data_ptr(), 16) == _lib.ERR_INVALID_ARG
+    assert _lib.check_pointer(pinned.data_ptr(), 16) == _lib.ERR_INVALID_ARG
+    assert _lib.check_pointer(device.data_ptr(), 16) == _lib.OK
+    assert _lib.check_pointer(device.data_ptr() + 8, 16) == _lib.ERR_MISALIGNED
+    # an entry point given a host X (everything else on the device)
+    cfg = synth.custom(64, 64, 128, 8, 16.0, seed_index=48)
+    inp = synth.make_inputs(cfg)
+    w = api.weights_from_host(inp, cfg.alpha, dev)
+    shape = w.shape(cfg.N)
+    fws, _, svs = _lib.sizes(shape)
+    X_host = torch.zeros((cfg.N, cfg.d), dtype=torch.bfloat16).pin_memory()
+    out = torch.empty((cfg.N, cfg.d), dtype=torch.bfloat16, device=dev)
+    g = torch.empty((cfg.N, cfg.d_ff), dtype=torch.bfloat16, device=dev)
+    u = torch.empty_like(g)
+    saved = torch.empty(max(svs, 256), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(fws, 256), dtype=torch.uint8, device=dev)
+    before = _lib.launch_count()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    rc = _lib.forward(shape, w.c_struct(), p(X_host), p(out), p(g), p(u), p(saved), p(ws), ws.numel(),
+                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == _lib.ERR_INVALID_ARG
+    assert _lib.launch_count() == before
+    torch.cuda.synchronize()
+    assert _lib.device_status(None) == 0
