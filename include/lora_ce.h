@@ -57,7 +57,8 @@ typedef struct {
     int64_t ignore_index;  /* label of rows that take no part (e.g. -100) */
 } lora_ce_shape;
 
-/* Workspace bytes of lora_ce_forward (per-chunk partial sums).  Host only. */
+/* Workspace bytes of lora_ce_forward and lora_ce_forward_reduced (per-chunk
+ * partial sums and per-row losses).  Host only. */
 int lora_ce_sizes(const lora_ce_shape* shape, size_t* workspace_bytes);
 
 /* loss [N] and lse [N] (the per-row log-sum-exp of the transformed logits,
@@ -72,6 +73,30 @@ int lora_ce_forward(const lora_ce_shape* shape, const void* logits, const int64_
  * logits in place).  One launch. */
 int lora_ce_backward(const lora_ce_shape* shape, const void* logits, const int64_t* labels, const float* lse,
                      const float* dloss, void* dlogits, void* stream);
+
+/* Reductions of the per-row losses into one loss. */
+#define LORA_CE_REDUCTION_SUM 1  /* sum of the per-row losses                                   */
+#define LORA_CE_REDUCTION_MEAN 2 /* that sum over the number of rows whose label is not
+                                    ignore_index (over 1 when every row is ignored)              */
+
+/* The loss reduced over the rows, computed in the library.  out[0] receives
+ * the reduced loss; out[1] receives d out[0] / d loss_row for a row that
+ * takes part: 1 for SUM, 1 / (rows taking part) for MEAN.  The per-row
+ * losses stay in the workspace; lse [N] as in lora_ce_forward.  The sum runs
+ * in fp64 in a fixed order, so the result is bitwise deterministic.  out is
+ * fp32 [2], 8-byte aligned.  Three launches: the chunk partials, their
+ * per-row combination, and the reduction (one CTA). */
+int lora_ce_forward_reduced(const lora_ce_shape* shape, const void* logits, const int64_t* labels, int reduction,
+                            float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* dlogits [N, ld] for the upstream gradient dout[0] (device fp32 [1]) of the
+ * loss lora_ce_forward_reduced returned: every row that takes part gets
+ * dloss = dout[0] * fwd_out[1], fwd_out being that call's `out` [2];
+ * ignored rows get zeros.  dlogits may be the logits buffer itself, as in
+ * lora_ce_backward.  One launch. */
+int lora_ce_backward_reduced(const lora_ce_shape* shape, const void* logits, const int64_t* labels,
+                             const float* lse, const float* dout, const float* fwd_out, void* dlogits,
+                             void* stream);
 
 /* Reads and clears the device-side status of the cross-entropy kernels
  * (LORA_MLP_OK, or LORA_MLP_ERR_INVALID_ARG after an out-of-range label).

@@ -101,6 +101,12 @@ typedef struct lora_mlp_grads {
 int lora_mlp_sizes(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes,
                    size_t* bwd_workspace_bytes, size_t* saved_bytes);
 
+/* The two workspace sizes alone (the same numbers lora_mlp_sizes gives),
+ * for callers that size scratch separately from the saved buffer.  Host
+ * only; either output pointer may be NULL. */
+int lora_mlp_workspace_size(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes,
+                            size_t* bwd_workspace_bytes);
+
 /* Forward.  X [N, d] in; out [N, d], g [N, d_ff] and u [N, d_ff] (the gate and
  * up pre-activations, rounded to bf16, kept for backward) and `saved` out.
  * H = silu(g) * u is formed from the bf16 g and u in the gate/up GEMM's
@@ -180,10 +186,14 @@ int lora_mlp_debug_force_timeout(int enable, int64_t wait_cycles);
  *  - Shapes whose forward workspace (lora_mlp_sizes) exceeds
  *    LORA_MLP_NOALLOC_SCRATCH_BYTES are rejected with
  *    LORA_MLP_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
- *  - The array is reserved on a device when this entry point is first used
- *    there and held until the process exits.  That first call on a device
- *    also looks up the array's device address and caches it; make it before
- *    any stream capture begins.
+ *  - Under CUDA's lazy module loading (CUDA_MODULE_LOADING=LAZY, the
+ *    default of current CUDA releases) the array is reserved on a device when
+ *    this entry point is first used there.  With CUDA_MODULE_LOADING=EAGER
+ *    every context that loads this library reserves it, 64 MiB per device,
+ *    whether or not the entry point is ever called.  Either way it is held
+ *    until the process exits.  The first call on a device also looks up the
+ *    array's device address and caches it; make it before any stream
+ *    capture begins.
  *  - Every call on a device shares the one array.  Calls whose work may
  *    overlap on the GPU (unordered streams) race and corrupt each other's
  *    results: order them, e.g. on one stream.  Each call clears the part of

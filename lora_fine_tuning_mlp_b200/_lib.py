@@ -21,6 +21,9 @@ ERR_UNSUPPORTED_ARCH = -5
 ERR_CUDA = -6
 ERR_DEVICE_TIMEOUT = -7
 
+CE_REDUCTION_SUM = 1
+CE_REDUCTION_MEAN = 2
+
 WEIGHTS_BF16 = 0
 WEIGHTS_INT4_B64 = 1
 
@@ -30,6 +33,7 @@ GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 # Every symbol include/lora_mlp.h, lora_linear.h, lora_rmsnorm.h and lora_ce.h declare.
 SYMBOLS = (
     "lora_mlp_sizes",
+    "lora_mlp_workspace_size",
     "lora_mlp_forward",
     "lora_mlp_backward",
     "lora_mlp_dequant_int4",
@@ -52,6 +56,8 @@ SYMBOLS = (
     "lora_ce_sizes",
     "lora_ce_forward",
     "lora_ce_backward",
+    "lora_ce_forward_reduced",
+    "lora_ce_backward_reduced",
     "lora_ce_device_status",
 )
 
@@ -143,6 +149,10 @@ def lib() -> ctypes.CDLL:
             L.lora_ce_sizes.argtypes = [ctypes.POINTER(CEShape), ctypes.POINTER(sz)]
             L.lora_ce_forward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, sz, vp]
             L.lora_ce_backward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, vp]
+            L.lora_ce_forward_reduced.argtypes = [ctypes.POINTER(CEShape), vp, vp, ctypes.c_int, vp, vp, vp, sz,
+                                                  vp]
+            L.lora_ce_backward_reduced.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, vp, vp]
+            L.lora_mlp_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(sz), ctypes.POINTER(sz)]
             L.lora_ce_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
@@ -153,7 +163,8 @@ def lib() -> ctypes.CDLL:
                          "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward",
                          "lora_rmsnorm_forward", "lora_rmsnorm_backward", "lora_mlp_block_sizes",
                          "lora_mlp_block_forward", "lora_mlp_block_backward", "lora_ce_sizes",
-                         "lora_ce_forward", "lora_ce_backward", "lora_ce_device_status"):
+                         "lora_ce_forward", "lora_ce_backward", "lora_ce_device_status",
+                         "lora_ce_forward_reduced", "lora_ce_backward_reduced", "lora_mlp_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -180,6 +191,13 @@ def sizes(shape: Shape):
     check(lib().lora_mlp_sizes(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b), ctypes.byref(s)),
           "lora_mlp_sizes")
     return f.value, b.value, s.value
+
+
+def workspace_size(shape: Shape):
+    f, b = ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().lora_mlp_workspace_size(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(b)),
+          "lora_mlp_workspace_size")
+    return f.value, b.value
 
 
 def forward(shape: Shape, weights: Weights, X, out, g, u, saved, workspace, workspace_bytes, stream) -> int:
@@ -300,6 +318,16 @@ def ce_forward(shape: CEShape, logits, labels, loss, lse, workspace, workspace_b
 
 def ce_backward(shape: CEShape, logits, labels, lse, dloss, dlogits, stream) -> int:
     return lib().lora_ce_backward(ctypes.byref(shape), logits, labels, lse, dloss, dlogits, stream)
+
+
+def ce_forward_reduced(shape: CEShape, logits, labels, reduction, out, lse, workspace, workspace_bytes,
+                       stream) -> int:
+    return lib().lora_ce_forward_reduced(ctypes.byref(shape), logits, labels, int(reduction), out, lse, workspace,
+                                         workspace_bytes, stream)
+
+
+def ce_backward_reduced(shape: CEShape, logits, labels, lse, dout, fwd_out, dlogits, stream) -> int:
+    return lib().lora_ce_backward_reduced(ctypes.byref(shape), logits, labels, lse, dout, fwd_out, dlogits, stream)
 
 
 def ce_device_status(stream) -> int:

@@ -605,25 +605,77 @@ def ce_backward(logits: torch.Tensor, labels: torch.Tensor, lse: torch.Tensor, d
     return out
 
 
+def ce_loss(logits: torch.Tensor, labels: torch.Tensor, *, reduction: str = "mean", logit_scale: float = 1.0,
+            softcap: float = 0.0, ignore_index: int = -100, workspace: Workspace | None = None, stream=None):
+    """The cross-entropy reduced over the rows, computed by the library:
+    returns (out [2] fp32, lse [N] fp32), out[0] the summed or mean loss and
+    out[1] its derivative with respect to each row's loss (1, or 1 / rows
+    taking part), the factor ce_backward_reduced applies."""
+    red = {"sum": _lib.CE_REDUCTION_SUM, "mean": _lib.CE_REDUCTION_MEAN}.get(reduction)
+    if red is None:
+        raise ValueError("reduction must be 'sum' or 'mean'")
+    shape = _ce_shape(logits, logit_scale, softcap, ignore_index)
+    N = shape.N
+    _need(labels, "labels", torch.int64, (N,))
+    dev = logits.device
+    out = torch.empty((2,), dtype=torch.float32, device=dev)
+    lse = torch.empty((N,), dtype=torch.float32, device=dev)
+    ws = (workspace or Workspace()).get(_lib.ce_sizes(shape), dev)
+    _lib.check(_lib.ce_forward_reduced(shape, _p(logits), _p(labels), red, _p(out), _p(lse), _p(ws), ws.numel(),
+                                       _stream(stream)), "lora_ce_forward_reduced")
+    return out, lse
+
+
+def ce_backward_reduced(logits: torch.Tensor, labels: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                        fwd_out: torch.Tensor, *, logit_scale: float = 1.0, softcap: float = 0.0,
+                        ignore_index: int = -100, out=None, inplace: bool = False, stream=None):
+    """dlogits [N, V] bf16 for the upstream gradient dout (fp32, one element)
+    of the loss ce_loss returned in fwd_out.  inplace=True writes the
+    gradient over the logits."""
+    shape = _ce_shape(logits, logit_scale, softcap, ignore_index)
+    N = shape.N
+    _need(labels, "labels", torch.int64, (N,))
+    _need(lse, "lse", torch.float32, (N,))
+    _need(fwd_out, "fwd_out", torch.float32, (2,))
+    if dout.numel() != 1 or dout.dtype != torch.float32 or not dout.is_cuda:
+        raise TypeError("dout must be one fp32 CUDA element")
+    if inplace:
+        out = logits
+    elif out is None:
+        out = torch.empty_strided(logits.size(), logits.stride(), dtype=BF16, device=logits.device)
+    elif (out.shape != logits.shape or out.stride() != logits.stride() or out.dtype != BF16 or not out.is_cuda):
+        raise ValueError("out must have the logits' shape, strides and dtype")
+    _lib.check(_lib.ce_backward_reduced(shape, _p(logits), _p(labels), _p(lse), _p(dout), _p(fwd_out), _p(out),
+                                        _stream(stream)), "lora_ce_backward_reduced")
+    return out
+
+
 class CrossEntropyFunction(torch.autograd.Function):
     """Mean cross-entropy over the rows whose label is not ignore_index, with
-    the library's chunked kernels.  Usage:
-    CrossEntropyFunction.apply(logits, labels, logit_scale, softcap, ignore_index).
-    The backward writes the logits' gradient over the logits (they are not
-    needed afterwards), as the pages' kernel does to save memory."""
+    the library's chunked kernels; the mean and its gradient factor are
+    computed in the library.  Usage:
+    CrossEntropyFunction.apply(logits, labels, logit_scale, softcap, ignore_index, inplace).
+    By default the backward writes the logits' gradient to a new buffer.
+    inplace=True writes it over the logits instead, as the pages' kernel does
+    to save memory; the logits' version counter is then bumped, so any other
+    autograd node that saved them raises instead of reading the gradient."""
 
     @staticmethod
-    def forward(ctx, logits, labels, logit_scale=1.0, softcap=0.0, ignore_index=-100):
-        loss, lse = ce_forward(logits, labels, logit_scale=logit_scale, softcap=softcap, ignore_index=ignore_index)
-        n = (labels != ignore_index).sum().clamp_min(1).to(torch.float32)
-        ctx.save_for_backward(logits, labels, lse, n)
-        ctx.cfg = (logit_scale, softcap, ignore_index)
-        return loss.sum() / n
+    def forward(ctx, logits, labels, logit_scale=1.0, softcap=0.0, ignore_index=-100, inplace=False):
+        out, lse = ce_loss(logits, labels, reduction="mean", logit_scale=logit_scale, softcap=softcap,
+                           ignore_index=ignore_index)
+        ctx.save_for_backward(logits, labels, lse, out)
+        ctx.cfg = (logit_scale, softcap, ignore_index, bool(inplace))
+        return out[0]
 
     @staticmethod
     def backward(ctx, g):
-        logits, labels, lse, n = ctx.saved_tensors
-        s, c, ign = ctx.cfg
-        dloss = (g.to(torch.float32) / n).expand(labels.shape[0]).contiguous()
-        dz = ce_backward(logits, labels, lse, dloss, logit_scale=s, softcap=c, ignore_index=ign, inplace=True)
-        return dz, None, None, None, None
+        logits, labels, lse, out = ctx.saved_tensors
+        s, c, ign, inplace = ctx.cfg
+        if g.dtype != torch.float32 or not g.is_cuda:
+            raise TypeError("the upstream gradient of the loss must be fp32 on the GPU")
+        dz = ce_backward_reduced(logits, labels, lse, g.contiguous(), out, logit_scale=s, softcap=c,
+                                 ignore_index=ign, inplace=inplace)
+        if inplace:
+            torch.autograd.graph.increment_version(logits)
+        return dz, None, None, None, None, None

@@ -320,8 +320,13 @@ __device__ __forceinline__ void ce_bwd_tile(const CeArgs& a, const __nv_bfloat16
 // (their logits are not read).  dt/dz = s (1 - (t/c)^2) or s: the factor s
 // is folded into g.  dz may alias z: every element is read before the same
 // thread writes it.
+//
+// The per-row upstream gradient is dloss[row * dloss_stride], times
+// dfactor[1] when dfactor is not null: a reduced loss passes its scalar
+// upstream gradient with stride 0 and the forward's d(reduced)/d(row) factor.
 __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(const CeArgs a, const float* __restrict__ lse,
-                                                           const float* __restrict__ dloss, __nv_bfloat16* dz,
+                                                           const float* __restrict__ dloss, long long dloss_stride,
+                                                           const float* __restrict__ dfactor, __nv_bfloat16* dz,
                                                            long long ld_dz) {
     const long long blk = blockIdx.x;
     const long long row = blk / a.nchunk;
@@ -334,7 +339,8 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(const CeArgs a, cons
     const bool ignored = y == a.ignore;
     const int yr = (y >= c0 && y < c0 + n) ? static_cast<int>(y - c0) : -kCeVec;
     const float L = lse[row];
-    const float g = ignored ? 0.0f : dloss[row] * a.scale;
+    const float gr = dfactor != nullptr ? dloss[row * dloss_stride] * dfactor[1] : dloss[row * dloss_stride];
+    const float g = ignored ? 0.0f : gr * a.scale;
     const int ln = ignored ? 0 : n;  // ignored rows: no loads (the zero stores still run)
 
     uint4 va[kCeItems], vb[kCeItems];
@@ -345,6 +351,41 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(const CeArgs a, cons
         if (k + 1 >= ntiles) break;
         if (k + 2 < ntiles) ce_load_tile(zc, (k + 2) * static_cast<int>(kCeTile), ln, va);
         ce_bwd_tile(a, zc, dc, (k + 1) * static_cast<int>(kCeTile), n, yr, L, g, ignored, vb);
+    }
+}
+
+// The per-row losses reduced to one number by one CTA, in a fixed order (so
+// the result is bitwise deterministic): each thread adds its rows
+// t, t + T, t + 2T, ... in fp64 and counts those not labelled ignore_index,
+// then the threads' totals are added in a fixed tree.  out[0] is the sum
+// (mean = false) or the sum over the count (mean = true; a count of 0 counts
+// as 1); out[1] is d out[0] / d loss_row for a row that takes part: 1, or
+// 1 / count.
+constexpr int kCeReduceThreads = 1024;
+__global__ void __launch_bounds__(kCeReduceThreads) ce_reduce_kernel(const CeArgs a, const float* __restrict__ loss,
+                                                                     bool mean, float* __restrict__ out) {
+    __shared__ double ssum[kCeReduceThreads];
+    __shared__ long long scnt[kCeReduceThreads];
+    double sum = 0.0;
+    long long cnt = 0;
+    for (long long row = threadIdx.x; row < a.N; row += kCeReduceThreads) {
+        sum += static_cast<double>(loss[row]);
+        cnt += a.labels[row] != a.ignore ? 1 : 0;
+    }
+    ssum[threadIdx.x] = sum;
+    scnt[threadIdx.x] = cnt;
+    __syncthreads();
+    for (int h = kCeReduceThreads / 2; h > 0; h >>= 1) {
+        if (static_cast<int>(threadIdx.x) < h) {
+            ssum[threadIdx.x] += ssum[threadIdx.x + h];
+            scnt[threadIdx.x] += scnt[threadIdx.x + h];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double n = static_cast<double>(scnt[0] > 0 ? scnt[0] : 1);
+        out[0] = static_cast<float>(mean ? ssum[0] / n : ssum[0]);
+        out[1] = static_cast<float>(mean ? 1.0 / n : 1.0);
     }
 }
 

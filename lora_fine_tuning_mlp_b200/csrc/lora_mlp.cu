@@ -838,6 +838,10 @@ int lora_mlp_sizes(const lora_mlp_shape* shape, size_t* fwd_workspace_bytes, siz
     return LORA_MLP_OK;
 }
 
+int lora_mlp_workspace_size(const lora_mlp_shape* shape, size_t* fwd_bytes, size_t* bwd_bytes) {
+    return lora_mlp_sizes(shape, fwd_bytes, bwd_bytes, nullptr);
+}
+
 int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out, void* g,
                      void* u, void* saved, void* workspace, size_t workspace_bytes, void* stream) {
     LMLP_TRY(validate_shape(shape));
@@ -1693,7 +1697,7 @@ CeArgs ce_args(const lora_ce_shape* sh, const void* logits, const int64_t* label
 }
 
 struct CePlan {
-    size_t part, ty, total;
+    size_t part, ty, rows, total;  // rows: per-row losses of the reduced forward
 };
 
 CePlan make_ce_plan(const lora_ce_shape& sh) {
@@ -1702,8 +1706,39 @@ CePlan make_ce_plan(const lora_ce_shape& sh) {
     CePlan p;
     p.part = c.take(static_cast<size_t>(sh.N) * nchunk * sizeof(float2));
     p.ty = c.take(static_cast<size_t>(sh.N) * sizeof(float));
+    p.rows = c.take(static_cast<size_t>(sh.N) * sizeof(float));
     p.total = c.off;
     return p;
+}
+
+// The chunk partials and their per-row combination into loss [N] and lse [N].
+int ce_forward_rows(const lora_ce_shape* shape, const CePlan& pl, const CeArgs& a, uint8_t* ws, float* loss,
+                    float* lse, cudaStream_t st) {
+    float2* part = reinterpret_cast<float2*>(ws + pl.part);
+    float* ty = reinterpret_cast<float*>(ws + pl.ty);
+    {
+        LaunchScope scope("CE_fwd_chunks", st);
+        ce_fwd_partial_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(a, part, ty);
+    }
+    LMLP_TRY(last_launch_error());
+    {
+        LaunchScope scope("CE_fwd_combine", st);
+        ce_fwd_combine_kernel<<<static_cast<unsigned>((shape->N + 255) / 256), 256, 0, st>>>(a, part, ty, loss,
+                                                                                            lse);
+    }
+    return last_launch_error();
+}
+
+int ce_backward_impl(const lora_ce_shape* shape, const void* logits, const int64_t* labels, const float* lse,
+                     const float* dloss, long long dloss_stride, const float* dfactor, void* dlogits,
+                     cudaStream_t st) {
+    const CeArgs a = ce_args(shape, logits, labels);
+    {
+        LaunchScope scope("CE_bwd", st);
+        ce_bwd_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(
+            a, lse, dloss, dloss_stride, dfactor, static_cast<__nv_bfloat16*>(dlogits), shape->ld);
+    }
+    return last_launch_error();
 }
 
 }  // namespace
@@ -1731,18 +1766,31 @@ int lora_ce_forward(const lora_ce_shape* shape, const void* logits, const int64_
     LMLP_TRY(device_info(&di));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const CeArgs a = ce_args(shape, logits, labels);
+    return ce_forward_rows(shape, pl, a, static_cast<uint8_t*>(workspace), loss, lse, st);
+}
+
+int lora_ce_forward_reduced(const lora_ce_shape* shape, const void* logits, const int64_t* labels, int reduction,
+                            float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_ce(shape));
+    if (reduction != LORA_CE_REDUCTION_SUM && reduction != LORA_CE_REDUCTION_MEAN) return LORA_MLP_ERR_INVALID_ARG;
+    if (logits == nullptr || labels == nullptr || out == nullptr || lse == nullptr || workspace == nullptr)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (!aligned(logits, 16) || !aligned(labels, 8) || !aligned(out, 8) || !aligned(lse, 4) ||
+        !aligned(workspace, 16))
+        return LORA_MLP_ERR_MISALIGNED;
+    const CePlan pl = make_ce_plan(*shape);
+    if (workspace_bytes < pl.total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_memory({logits, labels, out, lse, workspace}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CeArgs a = ce_args(shape, logits, labels);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    float2* part = reinterpret_cast<float2*>(ws + pl.part);
-    float* ty = reinterpret_cast<float*>(ws + pl.ty);
+    float* rows = reinterpret_cast<float*>(ws + pl.rows);
+    LMLP_TRY(ce_forward_rows(shape, pl, a, ws, rows, lse, st));
     {
-        LaunchScope scope("CE_fwd_chunks", st);
-        ce_fwd_partial_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(a, part, ty);
-    }
-    LMLP_TRY(last_launch_error());
-    {
-        LaunchScope scope("CE_fwd_combine", st);
-        ce_fwd_combine_kernel<<<static_cast<unsigned>((shape->N + 255) / 256), 256, 0, st>>>(a, part, ty, loss,
-                                                                                            lse);
+        LaunchScope scope("CE_fwd_reduce", st);
+        ce_reduce_kernel<<<1, kCeReduceThreads, 0, st>>>(a, rows, reduction == LORA_CE_REDUCTION_MEAN, out);
     }
     return last_launch_error();
 }
@@ -1758,14 +1806,23 @@ int lora_ce_backward(const lora_ce_shape* shape, const void* logits, const int64
     LMLP_TRY(check_memory({logits, labels, lse, dloss, dlogits}));
     DevInfo di;
     LMLP_TRY(device_info(&di));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const CeArgs a = ce_args(shape, logits, labels);
-    {
-        LaunchScope scope("CE_bwd", st);
-        ce_bwd_kernel<<<static_cast<unsigned>(shape->N * a.nchunk), kCeThreads, 0, st>>>(
-            a, lse, dloss, static_cast<__nv_bfloat16*>(dlogits), shape->ld);
-    }
-    return last_launch_error();
+    return ce_backward_impl(shape, logits, labels, lse, dloss, 1, nullptr, dlogits, static_cast<cudaStream_t>(stream));
+}
+
+int lora_ce_backward_reduced(const lora_ce_shape* shape, const void* logits, const int64_t* labels,
+                             const float* lse, const float* dout, const float* fwd_out, void* dlogits,
+                             void* stream) {
+    LMLP_TRY(validate_ce(shape));
+    if (logits == nullptr || labels == nullptr || lse == nullptr || dout == nullptr || fwd_out == nullptr ||
+        dlogits == nullptr)
+        return LORA_MLP_ERR_INVALID_ARG;
+    if (!aligned(logits, 16) || !aligned(dlogits, 16) || !aligned(labels, 8) || !aligned(lse, 4) ||
+        !aligned(dout, 4) || !aligned(fwd_out, 8))
+        return LORA_MLP_ERR_MISALIGNED;
+    LMLP_TRY(check_memory({logits, labels, lse, dout, fwd_out, dlogits}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return ce_backward_impl(shape, logits, labels, lse, dout, 0, fwd_out, dlogits, static_cast<cudaStream_t>(stream));
 }
 
 int lora_ce_device_status(void* stream, int* status) {

@@ -3,8 +3,11 @@
 // device memory themselves (see include/lora_mlp.h for who and why).
 //
 // The array lives in this translation unit, so it belongs to a module of its
-// own: CUDA loads that module, and reserves the array on a device, only when
-// this entry point is first used there, and keeps it until the process exits.
+// own.  Under lazy module loading (CUDA_MODULE_LOADING=LAZY, the default)
+// CUDA loads that module, and reserves the array on a device, only when this
+// entry point is first used there; with CUDA_MODULE_LOADING=EAGER every
+// context that loads the library reserves it.  It is kept until the process
+// exits.
 #include <cuda_runtime.h>
 
 #include <cstdint>

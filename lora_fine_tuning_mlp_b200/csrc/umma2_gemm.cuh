@@ -202,10 +202,14 @@ __device__ __forceinline__ PairUnit pair_decode(const PairArgs& a, int u) {
     return r;
 }
 
+// Returns the number of stages it filled.  Both CTAs' loads of a stage
+// count on the leader's full barrier, so the leader's count is what
+// drain_loads needs.
 template <bool B_MN>
-__device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, uint32_t rank, bool leader,
-                                              const SmemCtl& c) {
+__device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t base, uint32_t rank, bool leader,
+                                                   const SmemCtl& c) {
     const PairProb& P = a.prob;
+    long long issued = 0;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
     int stage = 0;
     uint32_t phase = 0;
@@ -220,7 +224,7 @@ __device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, 
             }
             const PairSeg& S = P.seg[seg];
             const int k0 = (kb - seg_kb0) * kBK;
-            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c)) return;
+            if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c)) return issued;
             const uint32_t fb_local = c.full + 8u * stage;
             if (leader) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
             const uint32_t fb = mapa_shared(fb_local, 0);
@@ -236,12 +240,14 @@ __device__ __forceinline__ void pair_producer(const PairArgs& a, uint32_t base, 
             } else {
                 tma_load_2d_pair(sB, bm, fb, bk, brow);
             }
+            ++issued;
             if (++stage == a.stages) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
     }
+    return issued;
 }
 
 // The MMA issuer.  One thread feeds the tensor core, and on the projection
@@ -606,7 +612,13 @@ __global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(cons
 #endif
 
     if (warp == 0) {
-        if (lane == 0) pair_producer<B_MN>(args, base, rank, leader, c);
+        if (lane == 0) {
+            // The leader waits for both CTAs' loads (they count on its full
+            // barriers); the other CTA cannot leave before it, since the
+            // cluster barrier below holds it until the leader arrives.
+            const long long issued = pair_producer<B_MN>(args, base, rank, leader, c);
+            if (leader) drain_loads(c.full, args.stages, issued, c.wait_limit);
+        }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0 && leader) {

@@ -151,6 +151,24 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, con
 }
 
 
+// Before a CTA leaves, every TMA load it issued has to have landed: a copy
+// still in flight would write into shared memory that the next CTA on the SM
+// may own.  On the normal path the MMA issuer has consumed every stage, so
+// this returns at once; after a bounded wait gave up it waits, again bounded
+// and regardless of the abort flag, for the last phase issued into each
+// stage's full barrier (issue i went to stage i % stages with phase parity
+// (i / stages) & 1).  One deadline covers all stages.
+__device__ __forceinline__ void drain_loads(uint32_t full, int stages, long long issued, long long limit) {
+    const long long t0 = clock64();
+    for (int s = 0; s < stages && s < issued; ++s) {
+        const long long i = s + static_cast<long long>(stages) * ((issued - 1 - s) / stages);
+        const uint32_t parity = static_cast<uint32_t>((i / stages) & 1);
+        while (!mbar_try_wait(full + 8u * static_cast<uint32_t>(s), parity)) {
+            if (clock64() - t0 > limit) return;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // roles
 
@@ -174,9 +192,11 @@ constexpr int kLoadBurst = LMLP_LOAD_BURST;
 // are walked directly, and the per-segment tensor maps and byte count are
 // looked up once per segment, not per K block.  A separate wait cursor runs
 // up to one burst ahead of the issue cursor.
+// Returns the number of stages it filled (issued loads into).
 template <int NACC>
-__device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
-                                              const SmemCtl& c) {
+__device__ __forceinline__ long long producer_loop(const GemmArgs& a, uint32_t smem_base, uint32_t stage_bytes,
+                                                   const SmemCtl& c) {
+    long long issued = 0;
     int stage = 0;
     uint32_t phase = 0;
     int wst = 0;  // next stage whose release to wait for
@@ -207,7 +227,7 @@ __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_b
             for (int kb = lo; kb < hi; ++kb) {
                 if (credits == 0) {
                     for (int i = 0; i < burst; ++i) {
-                        if (!wait_or_abort(c.empty + 8u * wst, wph ^ 1u, c)) return;
+                        if (!wait_or_abort(c.empty + 8u * wst, wph ^ 1u, c)) return issued;
                         if (++wst == a.stages) {
                             wst = 0;
                             wph ^= 1u;
@@ -236,6 +256,7 @@ __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_b
                         tma_load_2d(sB, bm[acc], fb, k0, n0);
                     }
                 }
+                ++issued;
                 if (++stage == a.stages) {
                     stage = 0;
                     phase ^= 1u;
@@ -243,6 +264,7 @@ __device__ __forceinline__ void producer_loop(const GemmArgs& a, uint32_t smem_b
             }
         }
     }
+    return issued;
 }
 
 // The MMA issuer (one thread).  The rank-r products are tall and skinny: a
@@ -513,7 +535,10 @@ __global__ void __launch_bounds__(kGemmThreads, LMLP_MAX_CPS) umma_gemm_kernel(c
 #endif
 
     if (warp == 0) {
-        if (lane == 0) producer_loop<NACC>(args, base, stage_bytes, c);
+        if (lane == 0) {
+            const long long issued = producer_loop<NACC>(args, base, stage_bytes, c);
+            drain_loads(c.full, args.stages, issued, c.wait_limit);
+        }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {

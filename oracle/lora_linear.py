@@ -53,13 +53,3 @@ def forward_backward(inputs: dict, alpha: float) -> dict:
     res = dict(f)
     res.update(b)
     return res
-
-
-def token_rows(inputs: dict, alpha: float, rows) -> dict:
-    """Y and dX for a subset of tokens (tokens are independent)."""
-    rows = np.asarray(rows)
-    sub = {k: (v[rows] if k in ("X", "dY") else v) for k, v in inputs.items()}
-    p = weights_f64(sub)
-    f = forward(p, alpha)
-    b = backward(p, alpha, p["dY"], f)
-    return {"Y": f["Y"], "dX": b["dX"]}

@@ -272,3 +272,32 @@ def test_ce_argument_errors(L):
     assert _lib.ce_backward(sh, FAKE, FAKE, FAKE + 1, FAKE, FAKE, None) == _lib.ERR_MISALIGNED
     assert L.lora_ce_forward(None, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
     assert L.lora_ce_device_status(None, None) == _lib.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(N=4096, d=4096, d_ff=14336, r=16), dict(N=1, d=136, r=24),
+                                dict(d=256, d_ff=704, fmt=1)])
+def test_workspace_size_is_the_sizes_pair(L, kw):
+    sh = shape(**kw)
+    f, b, _ = _lib.sizes(sh)
+    assert _lib.workspace_size(sh) == (f, b)
+    one = ctypes.c_size_t()
+    assert L.lora_mlp_workspace_size(ctypes.byref(sh), ctypes.byref(one), None) == _lib.OK and one.value == f
+    bad = shape(d=250)
+    assert (L.lora_mlp_workspace_size(ctypes.byref(bad), None, None)
+            == L.lora_mlp_sizes(ctypes.byref(bad), None, None, None) == _lib.ERR_UNSUPPORTED_SHAPE)
+
+
+def test_ce_reduced_argument_errors(L):
+    sh = _lib.make_ce_shape(37, 1000, 1008, 1.0, 30.0)
+    ws = _lib.ce_sizes(sh)
+    mean = _lib.CE_REDUCTION_MEAN
+    fr = _lib.ce_forward_reduced
+    assert fr(sh, FAKE, FAKE, mean, FAKE, FAKE, FAKE, ws - 1, None) == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert fr(sh, FAKE, FAKE, 0, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG      # no reduction
+    assert fr(sh, FAKE, FAKE, 3, FAKE, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert fr(sh, FAKE, FAKE, mean, None, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert fr(sh, FAKE, FAKE, mean, FAKE + 4, FAKE, FAKE, ws, None) == _lib.ERR_MISALIGNED  # out is 8-byte aligned
+    br = _lib.ce_backward_reduced
+    assert br(sh, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert br(sh, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, None) == _lib.ERR_MISALIGNED
+    assert br(sh, FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, None) == _lib.ERR_MISALIGNED
