@@ -24,8 +24,8 @@
  * Kernels: the same tcgen05 engines as the MLP.  Forward is two launches
  * (split-K rank-r product R = s X A^T; CTA-pair GEMM over K = d_in + r),
  * backward three (T and dB in one split-K launch; CTA-pair dX GEMM over
- * K = d_out + r; split-K token reduction for dA), plus one dequantisation
- * launch per pass for int4 weights.
+ * K = d_out + r; split-K token reduction for dA).  int4 weights are
+ * dequantised inside the two CTA-pair GEMMs.
  */
 #ifndef LORA_LINEAR_H
 #define LORA_LINEAR_H

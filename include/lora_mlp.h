@@ -20,12 +20,8 @@
  *    frees device memory, and never synchronises the stream (except
  *    lora_mlp_device_status, which says so).  Work is enqueued on `stream`
  *    (a cudaStream_t passed as void*; NULL = the legacy default stream) on
- *    the current CUDA device.  With int4 weights the forward and backward
- *    also run their dequantisation launches on one library-owned side stream
- *    per device (created on first use), forked from and joined back into
- *    `stream` through events created and released within the call: to the
- *    caller all work still completes in `stream`'s order, and stream capture
- *    of `stream` captures it.
+ *    the current CUDA device.  int4 frozen weights are dequantised inside
+ *    the GEMM kernels that read them; no bf16 copy of a weight is made.
  *  - Float tensors are bf16, row-major, densely packed (leading dimension =
  *    the row length).  Device pointers must be 16-byte aligned.
  *  - Sizes: N >= 1 tokens; d, d_ff multiples of 8 (of 64 for int4 weights);

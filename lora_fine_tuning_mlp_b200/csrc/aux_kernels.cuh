@@ -26,74 +26,142 @@ __device__ __forceinline__ uint64_t div7_rn_neg2(uint64_t neg_x) {
     return f2_fma(e, nr, y);
 }
 
-// fp32 bits of 2^23 + (q + 8) for the two's-complement nibble n (0..15) of
-// code q: q + 8 = n ^ 8, and 2^23 + m is exact in fp32 for m < 2^23.
-__device__ __forceinline__ uint32_t nibble_bits(uint32_t n) { return 0x4B000000u | (n ^ 8u); }
+// prmt: byte k of the result is byte (c >> 4k) & 7 of {b, a} (a's bytes
+// 0-3, then b's), or, when bit 3 of that selector nibble is set, that
+// byte's sign bit replicated over all eight bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
 
-// Eight codes (one 4-byte word, element 2k in the low nibble of byte k) ->
-// eight bf16 values (fp32(q) * fp32(scale)) / 7, rounded to nearest-even
-// bf16.  The product is exact and the quotient correctly rounded (div7_rn);
-// a non-finite scale takes IEEE's own divide (inf / 7 = inf, NaN stays NaN).
-template <bool kFinite>
-__device__ __forceinline__ uint4 dequant_word(uint32_t word, float scale) {
-    uint32_t o[4];
-    const uint64_t c8 = f2_packf(8388616.0f, 8388616.0f);  // 2^23 + 8
-    const uint64_t ns2 = f2_packf(-scale, -scale);
+// The sixteen bf16 values one block-int4 scale gives, as byte tables for
+// prmt lookups.  Code nibble n (two's complement, q = n or n - 16) takes
+//   T[n] = bf16_rne(fl(q * scale) / 7),
+// which for n >= 8 is -T'[16 - n] with T'[m] = bf16_rne(fl(m * scale) / 7):
+// q * scale is exact in fp32 and round-to-nearest-even is symmetric, so the
+// nine quotients m = 0..8 give every value.  lo[0], lo[1] hold the low bytes
+// of T[0..7], lo[2], lo[3] those of T[8..15]; hi likewise the high bytes.
+struct Int4Lut {
+    uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ Int4Lut int4_lut(float scale) {
+    float y[10];
+    if (fabsf(scale) <= 65504.0f) {
+        // finite: the exact products m * scale, divided by 7 with the
+        // correctly rounded sequence div7_rn_neg2, two quotients per step
+        const uint64_t ns2 = f2_packf(-scale, -scale);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t bl = nibble_bits((word >> (8 * j)) & 0xFu);
-        const uint32_t bh = nibble_bits((word >> (8 * j + 4)) & 0xFu);
-        // (2^23 + q + 8) - (2^23 + 8) = q exactly (+0 for code 0); q * (-scale)
-        // is -(q * scale) exactly, the sign of a zero included
-        const uint64_t neg_x = f2_mul(f2_sub(f2_pack(bl, bh), c8), ns2);
-        float lo, hi;
-        if (kFinite) {
-            f2_unpack(div7_rn_neg2(neg_x), lo, hi);
-        } else {
-            f2_unpack(neg_x, lo, hi);
-            lo = __fdiv_rn(lo, -7.0f);
-            hi = __fdiv_rn(hi, -7.0f);
+        for (int m = 0; m < 10; m += 2) {
+            const uint64_t q2 = div7_rn_neg2(f2_mul(f2_packf(static_cast<float>(m), static_cast<float>(m + 1)), ns2));
+            f2_unpack(q2, y[m], y[m + 1]);
         }
-        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        o[j] = *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        // inf or NaN: IEEE's own multiply and divide (0 * inf is NaN)
+#pragma unroll
+        for (int m = 0; m < 10; ++m) y[m] = __fdiv_rn(static_cast<float>(m) * scale, 7.0f);
+    }
+    const uint32_t p01 = bf16x2_bits(y[0], y[1]), p23 = bf16x2_bits(y[2], y[3]);
+    const uint32_t p45 = bf16x2_bits(y[4], y[5]), p67 = bf16x2_bits(y[6], y[7]);
+    const uint32_t n87 = bf16x2_bits(y[8], y[7]), n65 = bf16x2_bits(y[6], y[5]);
+    const uint32_t n43 = bf16x2_bits(y[4], y[3]), n21 = bf16x2_bits(y[2], y[1]);
+    Int4Lut t;
+    t.lo[0] = prmt(p01, p23, 0x6420u);
+    t.hi[0] = prmt(p01, p23, 0x7531u);
+    t.lo[1] = prmt(p45, p67, 0x6420u);
+    t.hi[1] = prmt(p45, p67, 0x7531u);
+    t.lo[2] = prmt(n87, n65, 0x6420u);               // codes 8..11: magnitudes 8, 7, 6, 5
+    t.hi[2] = prmt(n87, n65, 0x7531u) ^ 0x80808080u;  // negated: sign bit of the high byte
+    t.lo[3] = prmt(n43, n21, 0x6420u);               // codes 12..15: magnitudes 4, 3, 2, 1
+    t.hi[3] = prmt(n43, n21, 0x7531u) ^ 0x80808080u;
+    return t;
+}
+
+// Eight codes (one 4-byte word, element e in nibble e) -> eight bf16 values
+// (16 bytes, element e at bytes 2e, 2e + 1), by table lookup: the low three
+// bits of each nibble pick a byte of the code-0..7 or the code-8..15 table,
+// and the nibble's bit 3 picks the table.
+__device__ __forceinline__ uint4 int4_expand8(uint32_t w, const Int4Lut& t) {
+    const uint32_t sel = w & 0x77777777u;
+    const uint32_t w4 = w << 4;
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t sh = h ? sel >> 16 : sel;
+        // 0xFF for the elements whose code is negative: the sign bit of
+        // nibble e is the top bit of a byte of w << 4 (e even) or of w (e odd)
+        const uint32_t neg = prmt(w4, w, h ? 0xFBEAu : 0xD9C8u);
+        const uint32_t lo = (prmt(t.lo[0], t.lo[1], sh) & ~neg) | (prmt(t.lo[2], t.lo[3], sh) & neg);
+        const uint32_t hi = (prmt(t.hi[0], t.hi[1], sh) & ~neg) | (prmt(t.hi[2], t.hi[3], sh) & neg);
+        o[2 * h] = prmt(lo, hi, 0x5140u);      // elements 4h, 4h + 1
+        o[2 * h + 1] = prmt(lo, hi, 0x7362u);  // elements 4h + 2, 4h + 3
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// One thread per 8-code group per step: packed codes [rows, cols/2] bytes
-// and scales [rows, cols/64] are row-major, so group g (elements 8g .. 8g+7)
-// is the 4-byte code word g, its scale is scale g/8 and its output the 16
-// bytes at element 8g.  A CTA takes kDqUnroll x 256 consecutive groups and
-// issues all their loads before converting, so a warp's loads and stores
-// cover contiguous 128-byte and 512-byte spans and several are in flight.
-// Everything runs on the FMA and integer pipes, two lanes per fp32
-// instruction.
-constexpr int kDqThreads = 256;
-constexpr int kDqUnroll = 4;
+// One 64-element block ("line"): 32 bytes of codes -> 128 bytes of bf16.
+__device__ __forceinline__ void int4_line(uint4 c0, uint4 c1, float scale, uint4 (&out)[8]) {
+    const Int4Lut t = int4_lut(scale);
+    out[0] = int4_expand8(c0.x, t);
+    out[1] = int4_expand8(c0.y, t);
+    out[2] = int4_expand8(c0.z, t);
+    out[3] = int4_expand8(c0.w, t);
+    out[4] = int4_expand8(c1.x, t);
+    out[5] = int4_expand8(c1.y, t);
+    out[6] = int4_expand8(c1.z, t);
+    out[7] = int4_expand8(c1.w, t);
+}
 
-__global__ void __launch_bounds__(kDqThreads) dequant_int4_kernel(const uint32_t* __restrict__ packed,
+// The standalone dequantisation: one thread per line.  Codes [rows, cols/2]
+// and scales [rows, cols/64] are row-major, so line L (elements 64L ..) is
+// code bytes 32L .., scale L and output bytes 128L ..; the GEMMs' dequant
+// warps run the same int4_line on their stage's lines.
+constexpr int kDqThreads = 128;
+
+__global__ void __launch_bounds__(kDqThreads) dequant_int4_kernel(const uint4* __restrict__ packed,
                                                                   const __half* __restrict__ scales,
-                                                                  long long ngroups,
-                                                                  __nv_bfloat16* __restrict__ w) {
-    const long long span = static_cast<long long>(kDqThreads) * kDqUnroll;
-    for (long long g0 = static_cast<long long>(blockIdx.x) * span + threadIdx.x; g0 < ngroups;
-         g0 += static_cast<long long>(gridDim.x) * span) {
-        uint32_t word[kDqUnroll];
-        float sc[kDqUnroll];
+                                                                  long long nlines, uint4* __restrict__ w) {
+    for (long long L = static_cast<long long>(blockIdx.x) * kDqThreads + threadIdx.x; L < nlines;
+         L += static_cast<long long>(gridDim.x) * kDqThreads) {
+        const uint4 c0 = __ldcs(packed + 2 * L), c1 = __ldcs(packed + 2 * L + 1);
+        uint4 o[8];
+        int4_line(c0, c1, __half2float(scales[L]), o);
 #pragma unroll
-        for (int k = 0; k < kDqUnroll; ++k) {
-            const long long g = g0 + k * kDqThreads;
-            word[k] = g < ngroups ? __ldcs(packed + g) : 0u;
-            sc[k] = g < ngroups ? __half2float(scales[g >> 3]) : 0.0f;
-        }
-#pragma unroll
-        for (int k = 0; k < kDqUnroll; ++k) {
-            const long long g = g0 + k * kDqThreads;
-            if (g >= ngroups) break;
-            const uint4 v = fabsf(sc[k]) <= 65504.0f ? dequant_word<true>(word[k], sc[k])  // finite scale
-                                                     : dequant_word<false>(word[k], sc[k]);
-            __stcs(reinterpret_cast<uint4*>(w) + g, v);
-        }
+        for (int q = 0; q < 8; ++q) __stcs(w + 8 * L + q, o[q]);
+    }
+}
+
+// Block scales [rows, nb] (nb = cols / 64) -> their transpose [nb, rows], so
+// that the scales of one 64-column block of consecutive rows are contiguous
+// and a GEMM stage can fetch them with one TMA box.  Up to three matrices per
+// launch (blockIdx.z), 32 x 32 tiles through shared memory.
+struct ScaleT {
+    const unsigned short* src[3];
+    unsigned short* dst[3];
+    int rows[3], nb[3];
+};
+
+__global__ void __launch_bounds__(256) scale_transpose_kernel(const ScaleT a) {
+    __shared__ unsigned short tile[32][33];
+    const int z = blockIdx.z;
+    const int rows = a.rows[z], nb = a.nb[z];
+    const int r0 = blockIdx.x * 32, b0 = blockIdx.y * 32;
+    if (r0 >= rows || b0 >= nb) return;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+    for (int i = ty; i < 32; i += 8) {
+        const int r = r0 + i, b = b0 + tx;
+        if (r < rows && b < nb) tile[i][tx] = a.src[z][static_cast<long long>(r) * nb + b];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int b = b0 + i, r = r0 + tx;
+        if (r < rows && b < nb) a.dst[z][static_cast<long long>(b) * rows + r] = tile[tx][i];
     }
 }
 

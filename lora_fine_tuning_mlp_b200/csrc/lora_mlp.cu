@@ -183,6 +183,24 @@ bool encode_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tiled, unswizzled TMA descriptor of a byte matrix [outer, inner] (row
+// stride ld bytes, a multiple of 16) with a box_inner x box_outer box: the
+// packed codes of an int4 weight.  Out-of-range bytes read as zero.
+// (elem = 2: a 16-bit matrix, the transposed int4 scales; ld then in
+// elements.)
+bool encode_map_u8(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t box_inner,
+                   uint32_t box_outer, int elem = 1) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * static_cast<cuuint64_t>(elem)};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
@@ -400,6 +418,36 @@ struct PairBuilder {
         return nmaps++;
     }
     int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
+    // Packed int4 codes of a weight [rows, cols] (uint8 [rows, cols/2]):
+    // read K-major (K = cols), 32 bytes x 128 rows per box, or MN-major
+    // (K = rows), 32 bytes x 64 rows per box.
+    int q_map(const void* codes, int64_t rows, int64_t cols, bool mn) {
+        if (nmaps >= kMaxMaps) {
+            ok = false;
+            return 0;
+        }
+        if (!encode_map_u8(&a.maps[nmaps], codes, cols / 2, rows, cols / 2, 32, mn ? 64 : kPairHalfN)) ok = false;
+        return nmaps++;
+    }
+    // The transposed scales [cols/64, rows] of a weight [rows, cols]: one
+    // box holds the scales of 128 consecutive rows (K-major B) or 64 (MN-major).
+    int s_map(const void* st, int64_t rows, int64_t cols, bool mn) {
+        if (nmaps >= kMaxMaps) {
+            ok = false;
+            return 0;
+        }
+        if (!encode_map_u8(&a.maps[nmaps], st, rows, cols / 64, rows, mn ? 64 : kPairHalfN, 1, 2)) ok = false;
+        return nmaps++;
+    }
+    // Marks segment `sg` as reading int4 B: code and scale maps of halves 0 / 1.
+    void quant(int sg, int q0, int q1, int s0, int s1) {
+        PairSeg& S = a.prob.seg[sg];
+        S.q4 = 1;
+        S.qmap[0] = q0;
+        S.qmap[1] = q1;
+        S.smap[0] = s0;
+        S.smap[1] = s1;
+    }
     void seg(int amap, int b0, int b1, int row0, int row1, int k0, int k1, int64_t k_len) {
         PairProb& p = a.prob;
         if (p.nsegs >= kMaxSegs) {
@@ -433,7 +481,7 @@ int pair_tail_splits(int tiles, int clusters, int nkb) {
     return 2;
 }
 
-template <bool B_MN, int EPI>
+template <bool B_MN, int EPI, bool Q4 = false>
 int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, float* tail_part, int* tail_ctr) {
     if constexpr (pair_tma_store<EPI>()) {
         b.a.prob.omap[0] = b.out_map(b.a.prob.out0);
@@ -453,12 +501,14 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_ctr = tail_ctr;
     // (512-byte alignment) epilogue store staging per warp, then the dH epilogue's g/u rings
     const uint32_t staging = 512 + pair_epi_warps<EPI>() * pair_stage_warp_bytes<EPI>() + pair_ring_bytes<EPI>();
+    constexpr uint32_t kSB = pair_stage_bytes<Q4>();
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
-    int stages = static_cast<int>(budget / kPairStageBytes);
+    int stages = static_cast<int>(budget / kSB);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
+    if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
-    const size_t smem = 1024 + static_cast<size_t>(stages) * kPairStageBytes + gemm_ctl_bytes() + staging;
-    auto kern = umma2_gemm_kernel<B_MN, EPI>;
+    const size_t smem = 1024 + static_cast<size_t>(stages) * kSB + gemm_ctl_bytes() + staging;
+    auto kern = umma2_gemm_kernel<B_MN, EPI, Q4>;
     static int max_clusters[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -470,7 +520,7 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(pair_threads<EPI>(), 1, 1);
+    cfg.blockDim = dim3(pair_threads<EPI, Q4>(), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
@@ -510,17 +560,36 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
 
 int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
                    cudaStream_t st) {
-    const long long ngroups = rows * cols / 8;  // 8 codes per 4-byte word
-    const long long span = static_cast<long long>(kDqThreads) * kDqUnroll;
-    long long blocks = (ngroups + span - 1) / span;
+    const long long nlines = rows * (cols / 64);  // one scale and 64 elements per line
+    long long blocks = (nlines + kDqThreads - 1) / kDqThreads;
     const long long cap = static_cast<long long>(sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     {
         LaunchScope scope("dequant_int4", st);
         dequant_int4_kernel<<<static_cast<int>(blocks), kDqThreads, 0, st>>>(
-            static_cast<const uint32_t*>(packed), static_cast<const __half*>(scales), ngroups,
-            static_cast<__nv_bfloat16*>(w));
+            static_cast<const uint4*>(packed), static_cast<const __half*>(scales), nlines, static_cast<uint4*>(w));
+    }
+    return last_launch_error();
+}
+
+// Transposes up to three block-scale matrices [rows, cols/64] into
+// [cols/64, rows] (scale_transpose_kernel), one launch.
+int launch_scale_t(int n, const void* const* src, void* const* dst, const int64_t* rows, const int64_t* cols,
+                   cudaStream_t st) {
+    ScaleT a{};
+    unsigned gx = 1, gy = 1;
+    for (int i = 0; i < n; ++i) {
+        a.src[i] = static_cast<const unsigned short*>(src[i]);
+        a.dst[i] = static_cast<unsigned short*>(dst[i]);
+        a.rows[i] = static_cast<int>(rows[i]);
+        a.nb[i] = static_cast<int>(cols[i] / 64);
+        gx = std::max(gx, static_cast<unsigned>((rows[i] + 31) / 32));
+        gy = std::max(gy, static_cast<unsigned>((cols[i] / 64 + 31) / 32));
+    }
+    {
+        LaunchScope scope("int4_scales_t", st);
+        scale_transpose_kernel<<<dim3(gx, gy, n), 256, 0, st>>>(a);
     }
     return last_launch_error();
 }
@@ -594,9 +663,9 @@ struct Plan {
     int splits[SK_COUNT][kMaxProbs];
     size_t part_off[SK_COUNT][kMaxProbs];  // float offset of each problem's partials
     // forward workspace
-    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_w[2], f_total;  // f_w: int4 dequant buffers
+    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_st[3], f_total;  // f_st: int4 scales, transposed
     // backward workspace
-    size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_w[2], b_total;
+    size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_st[3], b_total;
     size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
     // saved
     size_t s_sgT, s_suT, s_sdT, s_total;
@@ -655,8 +724,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.ctr_bytes = static_cast<size_t>(std::max<int64_t>(max_tiles, 2 * kTailMaxUnits) + 8) * sizeof(int);
 
     const size_t bf = 2, f32 = 4;
-    const size_t Nz = N, dz = d, fz = dff, rz = r, ldN = p.ldN;
-    const size_t wsz = fz * dz * bf;  // one dequantised frozen weight (all three have d*d_ff elements)
+    const size_t Nz = N, fz = dff, rz = r, ldN = p.ldN;
 
     Carver f;
     p.f_h = f.take(Nz * fz * bf);
@@ -665,7 +733,8 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
     p.f_tail = f.take(kTailPartFloats * f32);
-    for (int i = 0; i < 2; ++i) p.f_w[i] = p.int4 ? f.take(wsz) : 0;
+    const size_t stsz = static_cast<size_t>(d) * static_cast<size_t>(dff) / 64 * 2;  // one weight's scales
+    for (int i = 0; i < 3; ++i) p.f_st[i] = p.int4 ? f.take(stsz) : 0;
     p.f_total = f.off;
 
     Carver b;
@@ -679,7 +748,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
-    for (int i = 0; i < 2; ++i) p.b_w[i] = p.int4 ? b.take(wsz) : 0;
+    for (int i = 0; i < 3; ++i) p.b_st[i] = p.int4 ? b.take(stsz) : 0;
     p.b_total = b.off;
 
     Carver sv;
@@ -763,63 +832,14 @@ int check_weight_memory(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
         if (rc_ != LORA_MLP_OK) return rc_; \
     } while (0)
 
-// The bf16 frozen weight `which` (0 = Wg, 1 = Wu, 2 = Wd): the caller's
-// buffer, or for int4 weights a just-in-time dequantisation into workspace
-// buffer `slot` (two buffers serve the whole pass: gate and up together,
-// then down).
-// int4 frozen weights: the dequantisation launches run on a side stream, so
-// that each overlaps a launch that does not read its buffer (fork and join
-// through events; the caller's stream stays the only one it has to order).
-#ifndef LMLP_INT4_OVERLAP
-#define LMLP_INT4_OVERLAP 1
-#endif
-
-// One non-blocking side stream per device, created on first use.
-int side_stream(cudaStream_t* out) {
-    static cudaStream_t streams[kMaxDevices] = {};
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_MLP_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(mu);
-    if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-        return LORA_MLP_ERR_CUDA;
-    *out = streams[dev];
-    return LORA_MLP_OK;
-}
-
-// The events of one call's fork/join edges, released when the call returns
-// (a pending event is released by CUDA once it completes).
-struct StreamLinks {
-    cudaEvent_t ev[8] = {};
-    int n = 0;
-    ~StreamLinks() {
-        for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
-    }
-    // `to` waits for everything issued to `from` so far.
-    int link(cudaStream_t from, cudaStream_t to) {
-        if (n >= 8) return LORA_MLP_ERR_CUDA;
-        cudaEvent_t& e = ev[n];
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-        ++n;
-        if (cudaEventRecord(e, from) != cudaSuccess || cudaStreamWaitEvent(to, e, 0) != cudaSuccess)
-            return LORA_MLP_ERR_CUDA;
-        return LORA_MLP_OK;
-    }
-};
-
-int frozen_weight(const Plan& pl, const lora_mlp_weights* w, int which, uint8_t* ws, const size_t* off, int slot,
-                  int sms, cudaStream_t st, const void** out) {
-    const void* bf[3] = {w->Wg, w->Wu, w->Wd};
-    if (!pl.int4) {
-        *out = bf[which];
-        return LORA_MLP_OK;
-    }
-    const void* sc[3] = {w->Sg, w->Su, w->Sd};
-    const int64_t rows = which == 2 ? pl.d : pl.d_ff;
-    const int64_t cols = which == 2 ? pl.d_ff : pl.d;
-    LMLP_TRY(launch_dequant(bf[which], sc[which], rows, cols, ws + off[slot], sms, st));
-    *out = ws + off[slot];
-    return LORA_MLP_OK;
+// int4: the three weights' scales, transposed into the workspace at off[0..2]
+// (Wg, Wu, Wd) for the GEMMs' scale maps.
+int mlp_scales_t(const Plan& pl, const lora_mlp_weights* w, uint8_t* ws, const size_t* off, cudaStream_t st) {
+    const void* src[3] = {w->Sg, w->Su, w->Sd};
+    void* dst[3] = {ws + off[0], ws + off[1], ws + off[2]};
+    const int64_t rows[3] = {pl.d_ff, pl.d_ff, pl.d};
+    const int64_t cols[3] = {pl.d, pl.d, pl.d_ff};
+    return launch_scale_t(3, src, dst, rows, cols, st);
 }
 
 }  // namespace
@@ -864,19 +884,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    const void* W[3] = {nullptr, nullptr, nullptr};
-    // int4: Wg, Wu dequantised beside F0; Wd (into Wg's buffer, once F1 is
-    // done with it) beside F2
-    const bool overlap = pl.int4 && LMLP_INT4_OVERLAP;
-    cudaStream_t qs = st;
-    StreamLinks links;
-    if (overlap) {
-        LMLP_TRY(side_stream(&qs));
-        LMLP_TRY(links.link(st, qs));
-        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, qs, &W[0]));
-        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, qs, &W[1]));
-    }
-
+    if (pl.int4) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.f_st, st));
     {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ax = b.a_k(X, N, d, d);
@@ -891,18 +899,12 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
         LMLP_TRY((launch_gemm<2, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
-    if (overlap) {
-        LMLP_TRY(links.link(qs, st));
-    } else {
-        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.f_w, 0, di.sms, st, &W[0]));
-        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.f_w, 1, di.sms, st, &W[1]));
-    }
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
         PairBuilder b(N, dff, 128);
         const int ax = b.a_k(X, N, d, d);
         const int asgu = b.a_k(Sgu, N, 2 * r, 2 * r);
-        const int bwg = b.b_k(W[0], dff, d, d);
-        const int bwu = b.b_k(W[1], dff, d, d);
+        const int bwg = pl.int4 ? b.q_map(w->Wg, dff, d, false) : b.b_k(w->Wg, dff, d, d);
+        const int bwu = pl.int4 ? b.q_map(w->Wu, dff, d, false) : b.b_k(w->Wu, dff, d, d);
         const int bbg = b.b_k(w->Bg, dff, r, r);
         const int bbu = b.b_k(w->Bu, dff, r, r);
         b.seg(ax, bwg, bwu, 0, 0, 0, 0, d);
@@ -911,11 +913,12 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.out1 = u;
         b.a.prob.out2 = h;
         b.a.prob.ld = dff;
-        LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
-    }
-    if (overlap) {
-        LMLP_TRY(links.link(st, qs));
-        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, qs, &W[2]));
+        if (pl.int4) {
+            b.quant(0, bwg, bwu, b.s_map(ws + pl.f_st[0], dff, d, false), b.s_map(ws + pl.f_st[1], dff, d, false));
+            LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD, true>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
+        }
     }
     {  // F2: S_d = s h Ad^T  -> Sd [N, r] and saved S_d^T [r, ldN]
         GemmBuilder b(pl.bn_r);
@@ -929,21 +932,23 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.fin(p, pl.s, static_cast<int>(r), Sd, r, sv + pl.s_sdT, nullptr, pl.ldN, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "F2_lowrank_mid", ctr)));
     }
-    if (overlap)
-        LMLP_TRY(links.link(qs, st));
-    else
-        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.f_w, 0, di.sms, st, &W[2]));
     {  // F3: out = h Wd^T + S_d Bd^T
         PairBuilder b(N, d, 256);
         const int ah = b.a_k(h, N, dff, dff);
         const int asd = b.a_k(Sd, N, r, r);
-        const int bwd = b.b_k(W[2], d, dff, dff);
+        const int bwd = pl.int4 ? b.q_map(w->Wd, d, dff, false) : b.b_k(w->Wd, d, dff, dff);
         const int bbd = b.b_k(w->Bd, d, r, r);
         b.seg(ah, bwd, bwd, 0, kPairHalfN, 0, 0, dff);
         b.seg(asd, bbd, bbd, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = out;
         b.a.prob.ld = d;
-        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down", tailp, ctr)));
+        if (pl.int4) {
+            const int sd = b.s_map(ws + pl.f_st[2], d, dff, false);
+            b.quant(0, bwd, bwd, sd, sd);
+            LMLP_TRY((launch_pair<false, EPI_BF16, true>(b, di.sms, st, "F3_down", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down", tailp, ctr)));
+        }
     }
     return LORA_MLP_OK;
 }
@@ -978,21 +983,10 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    if (pl.int4) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.b_st, st));
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
-    const void* W[3] = {nullptr, nullptr, nullptr};
-    // int4: Wd dequantised beside B0; Wg (into the second buffer) beside B1;
-    // Wu (into Wd's buffer, once B1 is done with it) beside B-mid
-    const bool overlap = pl.int4 && LMLP_INT4_OVERLAP;
-    cudaStream_t qs = st;
-    StreamLinks links;
-    if (overlap) {
-        LMLP_TRY(side_stream(&qs));
-        LMLP_TRY(links.link(st, qs));
-        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, qs, &W[2]));
-    }
-
     // adapter B matrices as K-major operands of the rank-r projections
     {  // B0: T_d = s dOut Bd -> Td [N, r], Td^T [r, ldN];  dBd = dOut^T S_d
         const int* sp = pl.splits[SK_B0];
@@ -1015,17 +1009,11 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.fin(p1, 1.0f, static_cast<int>(r), grads->dBd, r, nullptr, nullptr, 0, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B0_lowrank_out_dBd", ctr)));
     }
-    if (overlap) {
-        LMLP_TRY(links.link(qs, st));
-        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 1, di.sms, qs, &W[0]));
-    } else {
-        LMLP_TRY(frozen_weight(pl, w, 2, ws, pl.b_w, 0, di.sms, st, &W[2]));
-    }
     {  // B1: dH = dOut Wd + T_d Ad, SwiGLU backward in the epilogue
         PairBuilder b(N, dff, 256);
         const int a = b.a_k(dOut, N, d, d);
         const int atd = b.a_k(Td, N, r, r);
-        const int bwd = b.b_mn(W[2], d, dff, dff);
+        const int bwd = pl.int4 ? b.q_map(w->Wd, d, dff, true) : b.b_mn(w->Wd, d, dff, dff);
         const int bad = b.b_mn(w->Ad, r, dff, dff);
         b.seg(a, bwd, bwd, 0, kPairHalfN, 0, 0, d);
         b.seg(atd, bad, bad, 0, kPairHalfN, 0, 0, r);
@@ -1036,11 +1024,13 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p.out1 = du;
         p.out2 = hb;
         p.ld = dff;
-        LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
-    }
-    if (overlap) {
-        LMLP_TRY(links.link(st, qs));
-        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 0, di.sms, qs, &W[1]));
+        if (pl.int4) {
+            const int sd = b.s_map(ws + pl.b_st[2], d, dff, true);
+            b.quant(0, bwd, bwd, sd, sd);
+            LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD, true>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
+        }
     }
     {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
        //        dAd = T_d^T h (written transposed);  dBg = dg^T S_g, dBu = du^T S_u
@@ -1098,20 +1088,14 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         });
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B_mid_lowrank_grads", ctr)));
     }
-    if (overlap) {
-        LMLP_TRY(links.link(qs, st));
-    } else {
-        LMLP_TRY(frozen_weight(pl, w, 0, ws, pl.b_w, 0, di.sms, st, &W[0]));
-        LMLP_TRY(frozen_weight(pl, w, 1, ws, pl.b_w, 1, di.sms, st, &W[1]));
-    }
     {  // B4: dX = dg Wg + du Wu + T_g Ag + T_u Au
         PairBuilder b(N, d, 256);
         const int adg = b.a_k(dg, N, dff, dff);
         const int adu = b.a_k(du, N, dff, dff);
         const int atg = b.a_k(Tgu, N, r, 2 * r);
         const int atu = b.a_k(Tgu + r, N, r, 2 * r);
-        const int bwg = b.b_mn(W[0], dff, d, d);
-        const int bwu = b.b_mn(W[1], dff, d, d);
+        const int bwg = pl.int4 ? b.q_map(w->Wg, dff, d, true) : b.b_mn(w->Wg, dff, d, d);
+        const int bwu = pl.int4 ? b.q_map(w->Wu, dff, d, true) : b.b_mn(w->Wu, dff, d, d);
         const int bag = b.b_mn(w->Ag, r, d, d);
         const int bau = b.b_mn(w->Au, r, d, d);
         b.seg(adg, bwg, bwg, 0, kPairHalfN, 0, 0, dff);
@@ -1120,7 +1104,15 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.seg(atu, bau, bau, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = dX;
         b.a.prob.ld = d;
-        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX", tailp, ctr)));
+        if (pl.int4) {
+            const int sg = b.s_map(ws + pl.b_st[0], dff, d, true);
+            const int su = b.s_map(ws + pl.b_st[1], dff, d, true);
+            b.quant(0, bwg, bwg, sg, sg);
+            b.quant(1, bwu, bwu, su, su);
+            LMLP_TRY((launch_pair<true, EPI_BF16, true>(b, di.sms, st, "B4_dX", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX", tailp, ctr)));
+        }
     }
     {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]  (written transposed: dAg, dAu [r, d])
         GemmBuilder b(pl.bn_2r);
@@ -1243,8 +1235,8 @@ struct LinPlan {
     int splits[LK_COUNT][kMaxProbs];
     size_t part_off[LK_COUNT][kMaxProbs];
     size_t ctr_bytes;
-    size_t f_r, f_part, f_ctr, f_tail, f_w, f_total;
-    size_t b_t, b_tT, b_part, b_ctr, b_tail, b_w, b_total;
+    size_t f_r, f_part, f_ctr, f_tail, f_st, f_total;  // f_st, b_st: int4 scales, transposed
+    size_t b_t, b_tT, b_part, b_ctr, b_tail, b_st, b_total;
     size_t s_rT, s_total;
 };
 
@@ -1280,13 +1272,13 @@ LinPlan make_lin_plan(const lora_linear_shape& sh) {
     }
     p.ctr_bytes = static_cast<size_t>(std::max<int64_t>(max_tiles, 2 * kTailMaxUnits) + 8) * sizeof(int);
     const size_t bf = 2, f32 = 4, rz = r, ldN = p.ldN;
-    const size_t wsz = static_cast<size_t>(dout) * di * bf;
     Carver f;
     p.f_r = f.take(static_cast<size_t>(N) * rz * bf);
     p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
     p.f_tail = f.take(kTailPartFloats * f32);
-    p.f_w = p.int4 ? f.take(wsz) : 0;
+    const size_t stsz = static_cast<size_t>(dout) * static_cast<size_t>(di) / 64 * 2;
+    p.f_st = p.int4 ? f.take(stsz) : 0;
     p.f_total = f.off;
     Carver b;
     p.b_t = b.take(static_cast<size_t>(N) * rz * bf);
@@ -1294,7 +1286,7 @@ LinPlan make_lin_plan(const lora_linear_shape& sh) {
     p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
-    p.b_w = p.int4 ? b.take(wsz) : 0;
+    p.b_st = p.int4 ? b.take(stsz) : 0;
     p.b_total = b.off;
     Carver sv;
     p.s_rT = sv.take(rz * ldN * bf);
@@ -1324,18 +1316,6 @@ int check_lin_weights(const lora_linear_shape* sh, const lora_linear_weights* w)
 int check_lin_weight_memory(const lora_linear_shape* sh, const lora_linear_weights* w) {
     LMLP_TRY(check_memory({w->W, w->A, w->B}));
     if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_memory({w->S});
-    return LORA_MLP_OK;
-}
-
-// The bf16 frozen weight: the caller's, or int4 dequantised into the workspace.
-int lin_frozen_weight(const LinPlan& pl, const lora_linear_weights* w, uint8_t* ws, size_t off, int sms,
-                      cudaStream_t st, const void** out) {
-    if (!pl.int4) {
-        *out = w->W;
-        return LORA_MLP_OK;
-    }
-    LMLP_TRY(launch_dequant(w->W, w->S, pl.dout, pl.din, ws + off, sms, st));
-    *out = ws + off;
     return LORA_MLP_OK;
 }
 
@@ -1373,6 +1353,11 @@ int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weight
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    if (pl.int4) {
+        const void* src = w->S;
+        void* dst = ws + pl.f_st;
+        LMLP_TRY(launch_scale_t(1, &src, &dst, &pl.dout, &pl.din, st));
+    }
     {  // L0: R = s X A^T -> R [N, r], saved R^T [r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ax = b.a_k(X, N, din, din);
@@ -1385,19 +1370,23 @@ int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weight
         b.fin(p, pl.s, static_cast<int>(r), R, r, sv + pl.s_rT, nullptr, pl.ldN, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L0_lowrank_in", ctr)));
     }
-    const void* W = nullptr;
-    LMLP_TRY(lin_frozen_weight(pl, w, ws, pl.f_w, di.sms, st, &W));
     {  // L1: Y = X W^T + R B^T
         PairBuilder b(N, dout, 256);
         const int ax = b.a_k(X, N, din, din);
         const int ar = b.a_k(R, N, r, r);
-        const int bw = b.b_k(W, dout, din, din);
+        const int bw = pl.int4 ? b.q_map(w->W, dout, din, false) : b.b_k(w->W, dout, din, din);
         const int bb = b.b_k(w->B, dout, r, r);
         b.seg(ax, bw, bw, 0, kPairHalfN, 0, 0, din);
         b.seg(ar, bb, bb, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = Y;
         b.a.prob.ld = dout;
-        LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
+        if (pl.int4) {
+            const int sm = b.s_map(ws + pl.f_st, dout, din, false);
+            b.quant(0, bw, bw, sm, sm);
+            LMLP_TRY((launch_pair<false, EPI_BF16, true>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
+        }
     }
     return LORA_MLP_OK;
 }
@@ -1424,6 +1413,11 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
     int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    if (pl.int4) {
+        const void* src = w->S;
+        void* dst = ws + pl.b_st;
+        LMLP_TRY(launch_scale_t(1, &src, &dst, &pl.dout, &pl.din, st));
+    }
     {  // L2: T = s dY B -> T [N, r], T^T [r, ldN];  dB = dY^T R (R from saved, already s-scaled)
         const int* sp = pl.splits[LK_TDB];
         GemmBuilder b(pl.bn_r64);
@@ -1445,19 +1439,23 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
         b.fin(p1, 1.0f, static_cast<int>(r), dB, r, nullptr, nullptr, 0, static_cast<int>(r));
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "L2_lowrank_out_dB", ctr)));
     }
-    const void* W = nullptr;
-    LMLP_TRY(lin_frozen_weight(pl, w, ws, pl.b_w, di.sms, st, &W));
     {  // L3: dX = dY W + T A
         PairBuilder b(N, din, 256);
         const int ady = b.a_k(dY, N, dout, dout);
         const int at = b.a_k(T, N, r, r);
-        const int bw = b.b_mn(W, dout, din, din);
+        const int bw = pl.int4 ? b.q_map(w->W, dout, din, true) : b.b_mn(w->W, dout, din, din);
         const int ba = b.b_mn(w->A, r, din, din);
         b.seg(ady, bw, bw, 0, kPairHalfN, 0, 0, dout);
         b.seg(at, ba, ba, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = dX;
         b.a.prob.ld = din;
-        LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
+        if (pl.int4) {
+            const int sm = b.s_map(ws + pl.b_st, dout, din, true);
+            b.quant(0, bw, bw, sm, sm);
+            LMLP_TRY((launch_pair<true, EPI_BF16, true>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
+        } else {
+            LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
+        }
     }
     {  // L4: dA^T = X^T T  (written transposed: dA [r, d_in])
         GemmBuilder b(pl.bn_r);

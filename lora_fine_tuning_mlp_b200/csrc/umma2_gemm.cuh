@@ -21,10 +21,19 @@
 //     rank-r extension is one K = 2r segment: A = [S_g | S_u], half 0 reads
 //     Bg at K offset 0 and half 1 reads Bu at K offset -r, the zero fill of
 //     out-of-range columns supplying the two zero blocks.
+//
+// Block-int4 frozen weights (the Q4 instantiation) are dequantised inside
+// the kernel: for a segment whose B is int4, each CTA's producer brings the
+// packed codes of its B half into a small "raw" slot of the stage by TMA,
+// four dequant warps turn them into bf16 in the 128-byte-swizzled layout the
+// tensor core reads (the same bytes a TMA load of the bf16 weight would have
+// written), and arrive on the leader's full barrier.  The bf16 copy of the
+// weight never exists in global memory.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "aux_kernels.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
@@ -64,9 +73,20 @@ __host__ __device__ constexpr int pair_epi_warps() {
     return EPI == EPI_SWIGLU_BWD ? LMLP_PAIR_EPI_WARPS_BWD
                                  : (EPI == EPI_SWIGLU_FWD ? LMLP_PAIR_EPI_WARPS_FWD : LMLP_PAIR_EPI_WARPS_BF16);
 }
-template <int EPI>
+// int4 B: warps after the epilogue's that dequantise the codes of each
+// stage, one 64-element line (one scale) per thread: the 128 rows of a
+// K-major B half, or the 64 K rows x two 64-column chunks of an MN-major one.
+constexpr int kQ4Warps = 4;
+constexpr uint32_t kQ4CodeBytes = kPairHalfN * kBK / 2;  // 4 KB of codes per CTA and stage
+constexpr uint32_t kQ4ScaleBytes = kPairHalfN * 2;        // 128 fp16 scales
+constexpr uint32_t kQ4RawBytes = 5 * 1024;                // codes, scales, padding: stages stay 1 KB aligned
+template <bool Q4>
+__host__ __device__ constexpr uint32_t pair_stage_bytes() {
+    return kPairStageBytes + (Q4 ? kQ4RawBytes : 0u);
+}
+template <int EPI, bool Q4 = false>
 __host__ __device__ constexpr int pair_threads() {
-    return (2 + pair_epi_warps<EPI>()) * 32;
+    return (2 + pair_epi_warps<EPI>() + (Q4 ? kQ4Warps : 0)) * 32;
 }
 // The dH epilogue's g and u stream through a per-warp ring of shared-memory
 // slots filled by cp.async, LMLP_BWD_GU_RING chunks deep: the next chunk (at
@@ -130,6 +150,15 @@ struct PairSeg {
     int b_k[2];    // K-coordinate offset of each half
     int kblocks;
     int k_len;
+    // int4 B (Q4 launches): the codes come through the uint8 maps qmap
+    // (K-major: [rows, K/2], box 32 B x 128 rows; MN-major: [K, cols/2], box
+    // 32 B x 64 rows) and the scales through smap, maps of their transpose
+    // [cols/64, rows] (K-major: box 128 x 1; MN-major: box 64 x 1), both into
+    // the stage's raw slot.  Outside the weight both read as TMA's zero fill,
+    // so those lines dequantise to zeros.
+    int q4;
+    int qmap[2];
+    int smap[2];
 };
 
 struct PairProb {
@@ -205,9 +234,10 @@ __device__ __forceinline__ PairUnit pair_decode(const PairArgs& a, int u) {
 // Returns the number of stages it filled.  Both CTAs' loads of a stage
 // count on the leader's full barrier, so the leader's count is what
 // drain_loads needs.
-template <bool B_MN>
+template <bool B_MN, bool Q4>
 __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t base, uint32_t rank, bool leader,
                                                    const SmemCtl& c) {
+    constexpr uint32_t kSB = pair_stage_bytes<Q4>();
     const PairProb& P = a.prob;
     long long issued = 0;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
@@ -225,20 +255,44 @@ __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t b
             const PairSeg& S = P.seg[seg];
             const int k0 = (kb - seg_kb0) * kBK;
             if (!wait_or_abort(c.empty + 8u * stage, phase ^ 1u, c)) return issued;
+            const bool q4 = Q4 && S.q4 != 0;
             const uint32_t fb_local = c.full + 8u * stage;
-            if (leader) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
+            // int4 B reaches the stage through the dequant warps, whose
+            // arrivals (not bytes) the full barrier counts
+            if (leader) mbar_arrive_expect_tx(fb_local, q4 ? 2u * kATileBytes : 2u * kPairStageBytes);
             const uint32_t fb = mapa_shared(fb_local, 0);
-            const uint32_t sA = base + stage * kPairStageBytes;
+            const uint32_t sA = base + stage * kSB;
             const uint32_t sB = sA + kATileBytes;
             tma_load_2d_pair(sA, &a.maps[S.a_map], fb, k0, mb * kPairBM + static_cast<int>(rank) * kBM);
-            const CUtensorMap* bm = &a.maps[S.b_map[rank]];
             const int brow = nb * P.tile_n + S.b_row[rank];
             const int bk = k0 + S.b_k[rank];
-            if (B_MN) {
-                tma_load_2d_pair(sB, bm, fb, brow, bk);
-                tma_load_2d_pair(sB + 8192u, bm, fb, brow + 64, bk);
+            if (q4) {
+                // the codes of this CTA's B half into the raw slot, counted on
+                // this CTA's own raw barrier (x in bytes: brow and bk are
+                // multiples of 64, so x is 16-byte aligned)
+                const uint32_t rf = c.rawf + 8u * stage;
+                const uint32_t raw = sA + kPairStageBytes;
+                const CUtensorMap* qm = &a.maps[S.qmap[rank]];
+                const CUtensorMap* sm = &a.maps[S.smap[rank]];
+                mbar_arrive_expect_tx(rf, kQ4CodeBytes + kQ4ScaleBytes);
+                if (B_MN) {
+                    tma_load_2d(raw, qm, rf, brow >> 1, bk);
+                    tma_load_2d(raw + kQ4CodeBytes / 2, qm, rf, (brow + 64) >> 1, bk);
+                    tma_load_2d(raw + kQ4CodeBytes, sm, rf, bk, brow >> 6);
+                    tma_load_2d(raw + kQ4CodeBytes + kQ4ScaleBytes / 2, sm, rf, bk, (brow >> 6) + 1);
+                } else {
+                    tma_load_2d(raw, qm, rf, bk >> 1, brow);
+                    tma_load_2d(raw + kQ4CodeBytes, sm, rf, brow, bk >> 6);
+                }
             } else {
-                tma_load_2d_pair(sB, bm, fb, bk, brow);
+                const CUtensorMap* bm = &a.maps[S.b_map[rank]];
+                if (B_MN) {
+                    tma_load_2d_pair(sB, bm, fb, brow, bk);
+                    tma_load_2d_pair(sB + 8192u, bm, fb, brow + 64, bk);
+                } else {
+                    tma_load_2d_pair(sB, bm, fb, bk, brow);
+                }
+                if (Q4) mbar_arrive(c.rawf + 8u * stage);  // nothing to convert: release the dequant warps
             }
             ++issued;
             if (++stage == a.stages) {
@@ -258,7 +312,7 @@ __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t b
 // partial) and forms each stage's descriptors by adding offsets to those of
 // stage 0 instead of re-encoding them.  Measured on the Llama-3-8B MLP
 // shapes: 725-811 -> 574-681 SM cycles per K block.
-template <bool B_MN>
+template <bool B_MN, bool Q4>
 __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint32_t tmem_base, const SmemCtl& c) {
     const PairProb& P = a.prob;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
@@ -268,7 +322,7 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     const uint64_t a0 = sw128_desc(base, 16u, 1024u);
     const uint64_t b0 = B_MN ? sw128_desc(base + kATileBytes, 8192u, 1024u)
                              : sw128_desc(base + kATileBytes, 16u, 1024u);
-    constexpr uint32_t kStageStep = kPairStageBytes >> 4;
+    constexpr uint32_t kStageStep = pair_stage_bytes<Q4>() >> 4;
     constexpr uint32_t kAStep = 32u >> 4;                        // next 16-wide K slice of A
     constexpr uint32_t kBStep = B_MN ? (2048u >> 4) : (32u >> 4);  // ... of B
     int stage = 0;
@@ -288,7 +342,8 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
             const int k_len = P.seg[sg].k_len;
             seg_kb0 += nkb;
             for (int kb = lo; kb < hi; ++kb) {
-                if (!wait_or_abort(c.full + 8u * stage, phase, c)) return;
+                // int4: the other CTA's dequant warps wrote its B half
+                if (!wait_or_abort<Q4>(c.full + 8u * stage, phase, c)) return;
                 tc_fence_after();
                 const uint64_t ad = a0 + static_cast<uint64_t>(stage * kStageStep);
                 const uint64_t bd = b0 + static_cast<uint64_t>(stage * kStageStep);
@@ -314,6 +369,114 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
         if (++abuf == 2) {
             abuf = 0;
             aphase ^= 1u;
+        }
+    }
+}
+
+// The dequant warps of an int4 launch.  They walk the same (unit, K block)
+// sequence as the producer, two stages at a time.  For each pair they wait
+// for both stages' raw barriers; each thread reads its line's 32 code bytes
+// and its scale from each raw slot, expands both lines (int4_line; the two
+// are independent, so their dependent chains interleave) and writes the
+// stages whose B is int4 into their B tiles at the 128-byte swizzle (16-byte
+// piece w of tile row R at piece w ^ (R mod 8)), then fences its writes to
+// the async proxy.  Each warp then arrives once per stage on the leader's
+// full barrier.  Every input arrives by TMA: the warps hold no outstanding
+// global loads that their arrive would wait for.  Measured on the Llama-3-8B
+// int4 shapes, one warp expanding one line at a time was latency-bound
+// (about 740 cycles per stage against the tensor core's 512).
+#ifndef LMLP_Q4_BATCH
+#define LMLP_Q4_BATCH 2
+#endif
+template <bool B_MN>
+__device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int t) {
+    constexpr int kBatch = LMLP_Q4_BATCH;
+    const PairProb& P = a.prob;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    const int lane = threadIdx.x & 31;
+    constexpr uint32_t kSB = pair_stage_bytes<true>();
+    const int lrow = B_MN ? (t & 63) : t;  // tile row: N row (K-major) or K row (MN-major)
+    const int lj = B_MN ? (t >> 6) : 0;    // 64-column chunk (MN-major)
+    const uint32_t raw_off = kPairStageBytes + static_cast<uint32_t>(lj) * (kQ4CodeBytes / 2) +
+                             static_cast<uint32_t>(lrow) * 32u;
+    // the scales: one 128-entry run (K-major), or one 64-entry run per chunk
+    const uint32_t sc_off = kPairStageBytes + kQ4CodeBytes + static_cast<uint32_t>(t) * 2u;
+    const uint32_t out_off = kATileBytes + static_cast<uint32_t>(lj) * 8192u + static_cast<uint32_t>(lrow) * 128u;
+    const uint32_t swz = static_cast<uint32_t>(lrow & 7);
+    // read order of the two 16-byte halves: alternating every four rows puts
+    // the eight rows of a quarter-warp on distinct bank groups
+    const uint32_t h0 = static_cast<uint32_t>((lrow >> 2) & 1) * 16u;
+    int stage = 0;
+    uint32_t phase = 0;
+    int u = cid, seg = 0, seg_kb0 = 0, kb = 0, kb1 = 0;
+    auto start_unit = [&]() {
+        if (u < a.total_units) {
+            const PairUnit tu = pair_decode(a, u);
+            kb = tu.kb0;
+            kb1 = tu.kb1;
+            seg = 0;
+            seg_kb0 = 0;
+        }
+    };
+    start_unit();
+    while (u < a.total_units) {
+        // the next kBatch positions: their stages, phases and whether B is int4
+        int n = 0;
+        int bst[kBatch];
+        uint32_t bph[kBatch];
+        bool bq[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            bst[j] = stage;
+            bph[j] = phase;
+            bq[j] = false;
+            if (u < a.total_units) {
+                while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                    seg_kb0 += P.seg[seg].kblocks;
+                    ++seg;
+                }
+                bq[j] = P.seg[seg].q4 != 0;
+                ++n;
+                if (++stage == a.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++kb >= kb1) {
+                    u += ncl;
+                    start_unit();
+                }
+            }
+        }
+        uint4 x[kBatch][2];
+        float sc[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (j < n && !wait_or_abort(c.rawf + 8u * bst[j], bph[j], c)) return;
+            // (a bf16 stage's raw slot holds stale codes: read and expanded, never stored)
+            const uint32_t sb = base + static_cast<uint32_t>(bst[j]) * kSB;
+            const uint4 x0 = lds128(sb + raw_off + h0);
+            const uint4 x1 = lds128(sb + raw_off + (h0 ^ 16u));
+            x[j][0] = h0 ? x1 : x0;
+            x[j][1] = h0 ? x0 : x1;
+            sc[j] = __half2float(__ushort_as_half(lds16(sb + sc_off)));
+        }
+        uint4 o[kBatch][8];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) int4_line(x[j][0], x[j][1], sc[j], o[j]);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (j < n && bq[j]) {
+                const uint32_t sb = base + static_cast<uint32_t>(bst[j]) * kSB;
+#pragma unroll
+                for (uint32_t w = 0; w < 8; ++w) sts128(sb + out_off + ((w ^ swz) << 4), o[j][w]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                if (j < n) mbar_arrive_remote(mapa_shared(c.full + 8u * bst[j], 0));
         }
     }
 }
@@ -563,12 +726,13 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     if (ts != nullptr) ts->drain();
 }
 
-template <bool B_MN, int EPI>
-__global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
+template <bool B_MN, int EPI, bool Q4 = false>
+__global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
+    umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t ctl = base + args.stages * kPairStageBytes;
+    const uint32_t ctl = base + args.stages * pair_stage_bytes<Q4>();
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
     const SmemCtl c = make_ctl(ctl, ctl_ptr, args.wait_limit);
@@ -583,8 +747,10 @@ __global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(cons
     if (warp == 0 && lane < args.nmaps) tma_prefetch_desc(&args.maps[lane]);
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < args.stages; ++s) {
-            mbar_init(c.full + 8u * s, 1);
+            // int4: the leader's arrive.expect_tx plus one arrival per dequant warp of both CTAs
+            mbar_init(c.full + 8u * s, Q4 ? 1 + 2 * kQ4Warps : 1);
             mbar_init(c.empty + 8u * s, 1);
+            if (Q4) mbar_init(c.rawf + 8u * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(c.accf + 8u * b, 1);
@@ -616,13 +782,14 @@ __global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(cons
             // The leader waits for both CTAs' loads (they count on its full
             // barriers); the other CTA cannot leave before it, since the
             // cluster barrier below holds it until the leader arrives.
-            const long long issued = pair_producer<B_MN>(args, base, rank, leader, c);
+            const long long issued = pair_producer<B_MN, Q4>(args, base, rank, leader, c);
             if (leader) drain_loads(c.full, args.stages, issued, c.wait_limit);
+            if (Q4) drain_loads(c.rawf, args.stages, issued, c.wait_limit);  // this CTA's code loads
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            pair_mma<B_MN>(args, base, tmem_base, c);
+            pair_mma<B_MN, Q4>(args, base, tmem_base, c);
             umma_commit_pair(c.drain, 1);
             const long long t0 = clock64();
             while (!mbar_try_wait(c.drain, 0)) {
@@ -630,8 +797,10 @@ __global__ void __launch_bounds__(pair_threads<EPI>(), 1) umma2_gemm_kernel(cons
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp < 2 + pair_epi_warps<EPI>()) {
         pair_epilogue<EPI>(args, tmem_base, rank, c);
+    } else if constexpr (Q4) {
+        pair_dequant<B_MN>(args, base, c, static_cast<int>(threadIdx.x) - (2 + pair_epi_warps<EPI>()) * 32);
     }
 
     tc_fence_before();

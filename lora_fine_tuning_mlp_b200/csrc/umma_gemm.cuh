@@ -129,17 +129,21 @@ __device__ int g_lmlp_status;  // LORA_MLP_ERR_DEVICE_TIMEOUT once any bounded w
 
 struct SmemCtl {
     uint32_t full, empty, accf, acce, drain, never;  // barrier addresses (shared); `never` is never arrived on
+    uint32_t rawf;  // per-stage "codes landed" barriers of the CTA-pair GEMM with int4 B (unused otherwise)
     uint32_t tmem_slot;
     volatile int* abort_flag;
     volatile int* fin_flag;
     long long wait_limit;  // SM cycles a wait may spin before giving up
 };
 
-// Bounded wait that also gives up as soon as another role of this CTA gave up.
+// Bounded wait that also gives up as soon as another role of this CTA gave
+// up.  kCluster: acquire at cluster scope (see mbar_try_wait_cluster).
+template <bool kCluster = false>
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, const SmemCtl& c) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto ready = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (ready()) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!ready()) {
         if (*c.abort_flag) return false;
         if (clock64() - t0 > c.wait_limit) {
             *c.abort_flag = 1;
@@ -460,7 +464,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
 // ---------------------------------------------------------------------------
 // kernel
 
-__host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 6) + 16u; }
+__host__ __device__ constexpr uint32_t gemm_ctl_bytes() { return 8u * (2 * kMaxStages + 6) + 16u + 8u * kMaxStages; }
 
 // Barrier/flag block that follows the operand stages in shared memory.
 __device__ __forceinline__ SmemCtl make_ctl(uint32_t ctl, uint8_t* ctl_ptr, long long wait_limit) {
@@ -472,6 +476,7 @@ __device__ __forceinline__ SmemCtl make_ctl(uint32_t ctl, uint8_t* ctl_ptr, long
     c.drain = c.acce + 16u;
     c.never = c.drain + 8u;
     c.tmem_slot = c.never + 8u;
+    c.rawf = c.tmem_slot + 16u;
     c.wait_limit = wait_limit;
     c.abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 4u - ctl));
     c.fin_flag = reinterpret_cast<volatile int*>(ctl_ptr + (c.tmem_slot + 8u - ctl));

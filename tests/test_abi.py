@@ -55,14 +55,22 @@ def test_sizes_are_positive_and_grow_with_N(L):
     assert b1 >= 3 * 512 * 704 * 2
 
 
-def test_int4_workspace_holds_dequantised_weights(L):
+def test_int4_workspace_holds_no_dequantised_weight(L):
     with pytest.raises(_lib.LoraMLPError) as e:
         _lib.sizes(shape(d=256, d_ff=712, fmt=1))   # 712 is not a multiple of 64
     assert e.value.code == _lib.ERR_UNSUPPORTED_SHAPE
-    f1, b1, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=1))
-    f0b, b0b, _ = _lib.sizes(shape(d=256, d_ff=768, fmt=0))
-    # two dequantised weights at a time (gate and up together, then down)
-    assert f1 - f0b >= 2 * 256 * 768 * 2 and b1 - b0b >= 2 * 256 * 768 * 2
+    # int4 weights are dequantised inside the GEMMs: the scratch is the bf16
+    # path's plus the three weights' block scales in transposed order
+    for kw in (dict(d=256, d_ff=768), dict(N=4096, d=4096, d_ff=14336, r=16)):
+        f4, b4, s4 = _lib.sizes(shape(fmt=1, **kw))
+        f0, b0, s0 = _lib.sizes(shape(fmt=0, **kw))
+        scales = 3 * (kw["d"] * kw["d_ff"] // 64 * 2 + 256)
+        assert s4 == s0 and 0 < f4 - f0 <= scales and 0 < b4 - b0 <= scales
+        assert f4 - f0 < kw["d"] * kw["d_ff"] * 2 // 16     # far below one bf16 weight
+    lf = _lib.LinShape(4096, 4096, 1024, 16, 16.0, 1)
+    lb = _lib.LinShape(4096, 4096, 1024, 16, 16.0, 0)
+    (f4, b4, _), (f0, b0, _) = _lib.lin_sizes(lf), _lib.lin_sizes(lb)
+    assert 0 < f4 - f0 <= 4096 * 1024 // 64 * 2 + 256 and 0 < b4 - b0 <= 4096 * 1024 // 64 * 2 + 256
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -162,9 +170,10 @@ def test_linear_sizes(L):
     f2, b2, s2 = _lib.lin_sizes(lshape(N=4096))
     assert 0 < f1 < f2 and 0 < b1 < b2 and 0 < s1 < s2
     assert s1 >= 8 * 304 * 2          # s X A^T kept as bf16 [r, N padded to 8]
+    # int4 weights are dequantised inside the GEMMs: no bf16 copy in the scratch
     f4, b4, _ = _lib.lin_sizes(lshape(d_in=256, fmt=1))
     f0, b0, _ = _lib.lin_sizes(lshape(d_in=256, fmt=0))
-    assert f4 - f0 >= 320 * 256 * 2 and b4 - b0 >= 320 * 256 * 2
+    assert f4 - f0 < 320 * 256 * 2 // 16 and b4 - b0 < 320 * 256 * 2 // 16
 
 
 @pytest.mark.parametrize("kw,code", [

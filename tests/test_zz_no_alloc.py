@@ -30,8 +30,9 @@ def relerr(a, b):
     return float(np.max(np.abs(a - b))) / (den if den > 0 else 1.0)
 
 
-@pytest.mark.parametrize("cfg", [synth.CONFIGS[0], synth.custom(1000, 512, 1408, 32, 64.0, seed_index=41)],
-                         ids=lambda c: f"N{c.N}_d{c.d}_dff{c.d_ff}_r{c.r}")
+@pytest.mark.parametrize("cfg", [synth.CONFIGS[0], synth.custom(1000, 512, 1408, 32, 64.0, seed_index=41),
+                                 synth.custom(512, 256, 704, 8, 16.0, int4=True, seed_index=42)],
+                         ids=lambda c: f"N{c.N}_d{c.d}_dff{c.d_ff}_r{c.r}" + ("_int4" if c.int4 else ""))
 def test_noalloc_forward_matches_forward_on_two_calls(cfg):
     libbuild.build()
     assert torch.cuda.is_available()
