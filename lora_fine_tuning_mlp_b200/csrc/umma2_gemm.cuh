@@ -73,10 +73,21 @@ __host__ __device__ constexpr int pair_epi_warps() {
     return EPI == EPI_SWIGLU_BWD ? LMLP_PAIR_EPI_WARPS_BWD
                                  : (EPI == EPI_SWIGLU_FWD ? LMLP_PAIR_EPI_WARPS_FWD : LMLP_PAIR_EPI_WARPS_BF16);
 }
-// int4 B: warps after the epilogue's that dequantise the codes of each
-// stage, one 64-element line (one scale) per thread: the 128 rows of a
-// K-major B half, or the 64 K rows x two 64-column chunks of an MN-major one.
-constexpr int kQ4Warps = 4;
+// int4 B: the launch runs four warpgroups.  WG0: the producer (warp 0) and
+// the MMA issuer (warp 1), warps 2 and 3 idle; WG1 (warps 4-7): the
+// epilogue; WG2 and WG3 (warps 8-15): the dequant warps, WG2 converting the
+// even stages of the K sequence and WG3 the odd ones, one 64-element line
+// (one scale) per thread: the 128 rows of a K-major B half, or the 64 K rows
+// x two 64-column chunks of an MN-major one.  The expansion is bound by the
+// integer pipe's issue rate: one warp per SM sub-partition took ~640 cycles
+// per stage against the tensor core's 512, two ~430 (measured).  So that
+// sixteen warps fit, setmaxnreg moves registers from the producer/MMA and
+// dequant warpgroups to the epilogue's.
+constexpr int kQ4Warps = 4;  // dequant warps of one CTA that arrive per stage (one warpgroup)
+constexpr int kQ4Groups = 2;
+constexpr int kQ4RegsCtl = 80, kQ4RegsEpi = 232, kQ4RegsDq = 88;
+static_assert(128 * (kQ4RegsCtl + kQ4RegsEpi) + 256 * kQ4RegsDq <= 512 * 128,
+              "the warpgroups' register counts must fit the 128 a thread of a 512-thread block launches with");
 constexpr uint32_t kQ4CodeBytes = kPairHalfN * kBK / 2;  // 4 KB of codes per CTA and stage
 constexpr uint32_t kQ4ScaleBytes = kPairHalfN * 2;        // 128 fp16 scales
 constexpr uint32_t kQ4RawBytes = 5 * 1024;                // codes, scales, padding: stages stay 1 KB aligned
@@ -86,7 +97,12 @@ __host__ __device__ constexpr uint32_t pair_stage_bytes() {
 }
 template <int EPI, bool Q4 = false>
 __host__ __device__ constexpr int pair_threads() {
-    return (2 + pair_epi_warps<EPI>() + (Q4 ? kQ4Warps : 0)) * 32;
+    return Q4 ? 16 * 32 : (2 + pair_epi_warps<EPI>()) * 32;
+}
+// First epilogue warp: 2, or 4 (warpgroup 1) in an int4 launch.
+template <bool Q4>
+__host__ __device__ constexpr int pair_epi_first() {
+    return Q4 ? 4 : 2;
 }
 // The dH epilogue's g and u stream through a per-warp ring of shared-memory
 // slots filled by cp.async, LMLP_BWD_GU_RING chunks deep: the next chunk (at
@@ -373,24 +389,18 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     }
 }
 
-// The dequant warps of an int4 launch.  They walk the same (unit, K block)
-// sequence as the producer, two stages at a time.  For each pair they wait
-// for both stages' raw barriers; each thread reads its line's 32 code bytes
-// and its scale from each raw slot, expands both lines (int4_line; the two
-// are independent, so their dependent chains interleave) and writes the
-// stages whose B is int4 into their B tiles at the 128-byte swizzle (16-byte
-// piece w of tile row R at piece w ^ (R mod 8)), then fences its writes to
-// the async proxy.  Each warp then arrives once per stage on the leader's
-// full barrier.  Every input arrives by TMA: the warps hold no outstanding
-// global loads that their arrive would wait for.  Measured on the Llama-3-8B
-// int4 shapes, one warp expanding one line at a time was latency-bound
-// (about 740 cycles per stage against the tensor core's 512).
-#ifndef LMLP_Q4_BATCH
-#define LMLP_Q4_BATCH 2
-#endif
+// The dequant warps of an int4 launch, one warpgroup per parity of the
+// position in the (unit, K block) sequence the producer walks.  For each of
+// its stages a warpgroup waits for the stage's raw barrier; if the stage's B
+// is int4, each thread reads its line's 32 code bytes and its scale from the
+// raw slot, expands them (int4_line) and writes the 128 bytes into the
+// stage's B tile at the 128-byte swizzle (16-byte piece w of tile row R at
+// piece w ^ (R mod 8)), then fences its writes to the async proxy.  Each warp
+// then arrives once on the leader's full barrier.  Every input arrives by
+// TMA: the warps hold no outstanding global loads that their arrive would
+// wait for.
 template <bool B_MN>
-__device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int t) {
-    constexpr int kBatch = LMLP_Q4_BATCH;
+__device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int group, int t) {
     const PairProb& P = a.prob;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
     const int lane = threadIdx.x & 31;
@@ -408,75 +418,35 @@ __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, c
     const uint32_t h0 = static_cast<uint32_t>((lrow >> 2) & 1) * 16u;
     int stage = 0;
     uint32_t phase = 0;
-    int u = cid, seg = 0, seg_kb0 = 0, kb = 0, kb1 = 0;
-    auto start_unit = [&]() {
-        if (u < a.total_units) {
-            const PairUnit tu = pair_decode(a, u);
-            kb = tu.kb0;
-            kb1 = tu.kb1;
-            seg = 0;
-            seg_kb0 = 0;
-        }
-    };
-    start_unit();
-    while (u < a.total_units) {
-        // the next kBatch positions: their stages, phases and whether B is int4
-        int n = 0;
-        int bst[kBatch];
-        uint32_t bph[kBatch];
-        bool bq[kBatch];
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            bst[j] = stage;
-            bph[j] = phase;
-            bq[j] = false;
-            if (u < a.total_units) {
-                while (kb >= seg_kb0 + P.seg[seg].kblocks) {
-                    seg_kb0 += P.seg[seg].kblocks;
-                    ++seg;
-                }
-                bq[j] = P.seg[seg].q4 != 0;
-                ++n;
-                if (++stage == a.stages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-                if (++kb >= kb1) {
-                    u += ncl;
-                    start_unit();
-                }
+    int pos = 0;  // position in this CTA's sequence: this warpgroup takes those of its parity
+    for (int u = cid; u < a.total_units; u += ncl) {
+        const PairUnit tu = pair_decode(a, u);
+        int seg = 0, seg_kb0 = 0;
+        for (int kb = tu.kb0; kb < tu.kb1; ++kb, ++pos) {
+            while (kb >= seg_kb0 + P.seg[seg].kblocks) {
+                seg_kb0 += P.seg[seg].kblocks;
+                ++seg;
             }
-        }
-        uint4 x[kBatch][2];
-        float sc[kBatch];
+            if ((pos & 1) == group) {
+                if (!wait_or_abort(c.rawf + 8u * stage, phase, c)) return;
+                if (P.seg[seg].q4) {
+                    const uint32_t sb = base + static_cast<uint32_t>(stage) * kSB;
+                    const uint4 x0 = lds128(sb + raw_off + h0);
+                    const uint4 x1 = lds128(sb + raw_off + (h0 ^ 16u));
+                    const float sc = __half2float(__ushort_as_half(lds16(sb + sc_off)));
+                    uint4 o[8];
+                    int4_line(h0 ? x1 : x0, h0 ? x0 : x1, sc, o);
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            if (j < n && !wait_or_abort(c.rawf + 8u * bst[j], bph[j], c)) return;
-            // (a bf16 stage's raw slot holds stale codes: read and expanded, never stored)
-            const uint32_t sb = base + static_cast<uint32_t>(bst[j]) * kSB;
-            const uint4 x0 = lds128(sb + raw_off + h0);
-            const uint4 x1 = lds128(sb + raw_off + (h0 ^ 16u));
-            x[j][0] = h0 ? x1 : x0;
-            x[j][1] = h0 ? x0 : x1;
-            sc[j] = __half2float(__ushort_as_half(lds16(sb + sc_off)));
-        }
-        uint4 o[kBatch][8];
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) int4_line(x[j][0], x[j][1], sc[j], o[j]);
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            if (j < n && bq[j]) {
-                const uint32_t sb = base + static_cast<uint32_t>(bst[j]) * kSB;
-#pragma unroll
-                for (uint32_t w = 0; w < 8; ++w) sts128(sb + out_off + ((w ^ swz) << 4), o[j][w]);
+                    for (uint32_t w = 0; w < 8; ++w) sts128(sb + out_off + ((w ^ swz) << 4), o[w]);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa_shared(c.full + 8u * stage, 0));
             }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j)
-                if (j < n) mbar_arrive_remote(mapa_shared(c.full + 8u * bst[j], 0));
+            if (++stage == a.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
         }
     }
 }
@@ -487,7 +457,7 @@ __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, c
 // the matrix), and the consumer reads its row of each chunk back from shared
 // memory.  Each chunk is one cp.async group, so waiting until kGuRing - 1
 // groups remain in flight means the oldest chunk has landed.
-template <int EPI>
+template <int EPI, int kFirst>
 __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32_t tmem_base, uint32_t rank,
                                                        const SmemCtl& c) {
     const PairProb& P = a.prob;
@@ -496,14 +466,14 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
     const int lane = threadIdx.x & 31;
     const int quarter = warp & 3;
     constexpr int kGroups = pair_epi_warps<EPI>() / 4;
-    const int group = (warp - 2) >> 2;
+    const int group = (warp - kFirst) >> 2;
     const int gcols = 256 / kGroups;
     const int gcol0 = group * gcols;
     const int nch = gcols >> 5;
     const uint32_t area = pair_epi_area(c);
-    const uint32_t stg = area + static_cast<uint32_t>(warp - 2) * pair_stage_warp_bytes<EPI>();
+    const uint32_t stg = area + static_cast<uint32_t>(warp - kFirst) * pair_stage_warp_bytes<EPI>();
     const uint32_t ring = area + pair_epi_warps<EPI>() * pair_stage_warp_bytes<EPI>() +
-                          static_cast<uint32_t>(warp - 2) * (kGuRing * kGuSlotBytes);
+                          static_cast<uint32_t>(warp - kFirst) * (kGuRing * kGuSlotBytes);
     TmaStore ts;
     ts.map[0] = &a.maps[P.omap[0]];
     ts.map[1] = &a.maps[P.omap[1]];
@@ -613,11 +583,11 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
     if constexpr (pair_tma_store<EPI>()) ts.drain();
 }
 
-template <int EPI>
+template <int EPI, int kFirst>
 __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_base, uint32_t rank,
                                               const SmemCtl& c) {
     if constexpr (EPI == EPI_SWIGLU_BWD && kGuRing > 0) {
-        pair_epilogue_bwd_ring<EPI>(a, tmem_base, rank, c);
+        pair_epilogue_bwd_ring<EPI, kFirst>(a, tmem_base, rank, c);
         return;
     }
     constexpr int NACC = EPI == EPI_SWIGLU_FWD ? 2 : 1;
@@ -631,7 +601,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     // Two groups hold half the registers per thread: they load g and u chunk
     // by chunk instead of one chunk ahead.
     constexpr bool kPrefetch = kGroups == 1;
-    const int group = (warp - 2) >> 2;
+    const int group = (warp - kFirst) >> 2;
     EpiOut o;
     o.out0 = P.out0;
     o.out1 = P.out1;
@@ -651,7 +621,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     // by 1-2% and costs the latter about as much).
     const uint32_t stg = pair_stage_warp_bytes<EPI>() == 0u
                              ? 0u
-                             : pair_epi_area(c) + static_cast<uint32_t>(warp - 2) * pair_stage_warp_bytes<EPI>();
+                             : pair_epi_area(c) + static_cast<uint32_t>(warp - kFirst) * pair_stage_warp_bytes<EPI>();
     TmaStore tsv;
     TmaStore* ts = nullptr;
     if constexpr (pair_tma_store<EPI>()) {
@@ -705,7 +675,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
         if (t.tail >= 0) {
             __threadfence();
             pair_epi_bar<EPI>();
-            if (threadIdx.x == 64) {
+            if (threadIdx.x == kFirst * 32) {
                 int* ctr = a.tail_ctr + t.tail * 2 + rank;
                 const int old = atomicAdd(ctr, 1);
                 const int last = old == a.tail_splits - 1;
@@ -724,6 +694,18 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
         }
     }
     if (ts != nullptr) ts->drain();
+}
+
+// Per-warpgroup register budgets (all four warps of a warpgroup execute the
+// same instruction).  .dec gives registers back to the block's pool; .inc
+// waits until the pool holds enough.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 template <bool B_MN, int EPI, bool Q4 = false>
@@ -777,7 +759,9 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
     grid_launch_dependents();
 #endif
 
-    if (warp == 0) {
+    static_assert(!Q4 || pair_epi_warps<EPI>() == 4, "an int4 launch runs one epilogue warpgroup");
+    constexpr int kFirst = pair_epi_first<Q4>();
+    auto producer_role = [&]() {
         if (lane == 0) {
             // The leader waits for both CTAs' loads (they count on its full
             // barriers); the other CTA cannot leave before it, since the
@@ -787,7 +771,8 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
             if (Q4) drain_loads(c.rawf, args.stages, issued, c.wait_limit);  // this CTA's code loads
         }
         __syncwarp();
-    } else if (warp == 1) {
+    };
+    auto mma_role = [&]() {
         if (lane == 0 && leader) {
             pair_mma<B_MN, Q4>(args, base, tmem_base, c);
             umma_commit_pair(c.drain, 1);
@@ -797,10 +782,27 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
             }
         }
         __syncwarp();
-    } else if (warp < 2 + pair_epi_warps<EPI>()) {
-        pair_epilogue<EPI>(args, tmem_base, rank, c);
-    } else if constexpr (Q4) {
-        pair_dequant<B_MN>(args, base, c, static_cast<int>(threadIdx.x) - (2 + pair_epi_warps<EPI>()) * 32);
+    };
+    if constexpr (Q4) {
+        // each warpgroup's role runs inside the branch that sets its register
+        // budget, so that the compiler allocates for it accordingly
+        if (warp < 4) {
+            regs_dec<kQ4RegsCtl>();
+            if (warp == 0) producer_role();
+            else if (warp == 1) mma_role();
+            // warps 2 and 3: idle
+        } else if (warp < 8) {
+            regs_inc<kQ4RegsEpi>();
+            pair_epilogue<EPI, kFirst>(args, tmem_base, rank, c);
+        } else {
+            regs_dec<kQ4RegsDq>();
+            const int dq = static_cast<int>(threadIdx.x) - 8 * 32;  // 0 .. 255
+            pair_dequant<B_MN>(args, base, c, dq >> 7, dq & 127);
+        }
+    } else {
+        if (warp == 0) producer_role();
+        else if (warp == 1) mma_role();
+        else pair_epilogue<EPI, kFirst>(args, tmem_base, rank, c);
     }
 
     tc_fence_before();
