@@ -399,6 +399,8 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
 // then arrives once on the leader's full barrier.  Every input arrives by
 // TMA: the warps hold no outstanding global loads that their arrive would
 // wait for.
+// The launcher gives int4 launches an even number of stages, so each stage
+// is always converted by the same warpgroup.
 template <bool B_MN>
 __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int group, int t) {
     const PairProb& P = a.prob;

@@ -117,3 +117,35 @@ def test_every_adapter_gradient_against_token_block_sums(cfg):
     errs = {k: relerr(got[k], ref[k]) for k in GRADS}
     bad = {k: v for k, v in errs.items() if not v <= TOL}
     assert not bad, f"{cfg.name}: {bad} (all {errs})"
+
+
+def test_int4_full_size_is_bitwise_the_bf16_path_every_run():
+    """The int4 kernels dequantise in-kernel through rings of shared-memory
+    slots shared by several warp roles; a wrong hand-off shows as a few stale
+    lines in a stage, differing from run to run.  At full size (where the
+    rings wrap thousands of times), five forward + backward passes must each
+    give exactly the bits of the bf16 path on the dequantised weights."""
+    cfg = synth.BY_NAME["llama3_8b_mlp_int4"]
+    _cache.clear()
+    torch.cuda.empty_cache()
+    inp = synth.make_inputs(cfg)
+    deq = dict(inp)
+    for k in ("Wg", "Wu", "Wd"):
+        deq[k] = oracle.dequant_int4(inp[k + "_q"], inp[k + "_scale"])
+        del deq[k + "_q"], deq[k + "_scale"]
+    dev = torch.device("cuda:0")
+    w4 = api.weights_from_host(inp, cfg.alpha, dev)
+    w16 = api.weights_from_host(deq, cfg.alpha, dev)
+    X = api.to_device_bf16(inp["X"], dev)
+    dOut = api.to_device_bf16(inp["dOut"], dev)
+    ref_out, ref_saved = api.forward(X, w16)
+    ref_dX, ref_grads = api.backward(X, w16, ref_saved, dOut)
+    ref = {"out": ref_out, "g": ref_saved.g, "u": ref_saved.u, "dX": ref_dX, **ref_grads}
+    for rep in range(5):
+        out, saved = api.forward(X, w4)
+        dX, grads = api.backward(X, w4, saved, dOut)
+        got = {"out": out, "g": saved.g, "u": saved.u, "dX": dX, **grads}
+        torch.cuda.synchronize()
+        bad = {k: int((got[k].view(torch.int16) != ref[k].view(torch.int16)).sum()) for k in ref}
+        assert not any(bad.values()), (rep, bad)
+    assert _lib.device_status(None) == 0
