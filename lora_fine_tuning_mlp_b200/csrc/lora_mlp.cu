@@ -505,13 +505,6 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kSB);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
-    // int4: an even number of stages.  The two dequant warpgroups take
-    // alternate positions of the K sequence, so with an even ring every use of
-    // a stage falls to the same warpgroup as its previous use; a warpgroup,
-    // working in order, is then never more than one phase behind a stage's
-    // barriers.  With an odd ring one warpgroup could run two phases ahead of
-    // the other and a barrier's phase parity would alias.
-    if (Q4) stages &= ~1;
     if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     const size_t smem = 1024 + static_cast<size_t>(stages) * kSB + gemm_ctl_bytes() + staging;

@@ -399,8 +399,13 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
 // then arrives once on the leader's full barrier.  Every input arrives by
 // TMA: the warps hold no outstanding global loads that their arrive would
 // wait for.
-// The launcher gives int4 launches an even number of stages, so each stage
-// is always converted by the same warpgroup.
+// A stage is always converted by the same warpgroup (stage index mod 2), so
+// successive uses of a stage's barriers come from one warpgroup working in
+// order, never more than one phase behind them; with an odd stage count the
+// warpgroups' shares differ by one stage in S.  (Splitting by the position's
+// parity instead lets, with an odd count, one warpgroup run two phases ahead
+// of the other on a stage, and the barrier's phase parity aliases: seen as a
+// few stale lines per launch on the Llama-3-8B int4 shapes.)
 template <bool B_MN>
 __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int group, int t) {
     const PairProb& P = a.prob;
@@ -420,16 +425,15 @@ __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, c
     const uint32_t h0 = static_cast<uint32_t>((lrow >> 2) & 1) * 16u;
     int stage = 0;
     uint32_t phase = 0;
-    int pos = 0;  // position in this CTA's sequence: this warpgroup takes those of its parity
     for (int u = cid; u < a.total_units; u += ncl) {
         const PairUnit tu = pair_decode(a, u);
         int seg = 0, seg_kb0 = 0;
-        for (int kb = tu.kb0; kb < tu.kb1; ++kb, ++pos) {
+        for (int kb = tu.kb0; kb < tu.kb1; ++kb) {
             while (kb >= seg_kb0 + P.seg[seg].kblocks) {
                 seg_kb0 += P.seg[seg].kblocks;
                 ++seg;
             }
-            if ((pos & 1) == group) {
+            if ((stage & 1) == group) {
                 if (!wait_or_abort(c.rawf + 8u * stage, phase, c)) return;
                 if (P.seg[seg].q4) {
                     const uint32_t sb = base + static_cast<uint32_t>(stage) * kSB;
