@@ -1,7 +1,7 @@
 """Seeded synthetic inputs for the fused LoRA + SwiGLU MLP.
 
 This module only draws random numbers and rounds them to the storage formats
-(bf16, and the int4 block format of the frozen weights).  It holds none of the
+(bf16, and the int4 and FP8 block formats of the frozen weights).  It holds none of the
 arithmetic of the MLP itself, so both the CUDA path and the CPU oracle can take
 their inputs from here without sharing any of the method.
 
@@ -42,6 +42,7 @@ class Config:
     alpha: float
     int4: bool = False
     index: int = 0
+    fp8: bool = False
 
     @property
     def s(self) -> float:
@@ -70,12 +71,13 @@ CONFIGS = (
     Config("llama3_8b_mlp", 4096, 4096, 14336, 16, 16.0, index=2),
     Config("qwen2_7b_mlp", 8192, 3584, 18944, 64, 128.0, index=3),
     Config("llama3_8b_mlp_int4", 4096, 4096, 14336, 16, 16.0, int4=True, index=4),
+    Config("llama3_8b_mlp_fp8", 4096, 4096, 14336, 16, 16.0, index=5, fp8=True),
 )
 BY_NAME = {c.name: c for c in CONFIGS}
 
 
-def custom(N, d, d_ff, r, alpha, int4=False, seed_index=100, name="custom") -> Config:
-    return Config(name, N, d, d_ff, r, float(alpha), int4=int4, index=seed_index)
+def custom(N, d, d_ff, r, alpha, int4=False, seed_index=100, name="custom", fp8=False) -> Config:
+    return Config(name, N, d, d_ff, r, float(alpha), int4=int4, index=seed_index, fp8=fp8)
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -115,12 +117,38 @@ def quantize_int4(w: np.ndarray):
     return packed, scale16
 
 
+FP8_MAX = 448.0  # largest finite E4M3 value
+
+
+def quantize_fp8(w: np.ndarray):
+    """Block-quantise a float32 [rows, cols] weight to FP8 E4M3 codes.
+
+    Blocks of 64 consecutive input-dimension elements share one fp32 scale,
+    the block's absolute maximum over 448 (the largest E4M3 value); codes are
+    w / scale rounded to E4M3 (nearest, ties to even, by torch's float8_e4m3fn
+    conversion).  An all-zero block gets scale 0 and codes 0.
+    Returns (codes uint8 [rows, cols], scales float32 [rows, cols/64]).
+    """
+    import torch
+
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    assert cols % INT4_BLOCK == 0
+    blocks = w.reshape(rows, cols // INT4_BLOCK, INT4_BLOCK)
+    scale = (np.abs(blocks).max(axis=2) / np.float32(FP8_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0))
+    x = np.clip(blocks / safe[:, :, None], -FP8_MAX, FP8_MAX).astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(x.reshape(rows, cols))).to(torch.float8_e4m3fn)
+    return codes.view(torch.uint8).numpy().copy(), scale
+
+
 def make_inputs(cfg: Config) -> dict:
     """Draw all inputs of one workload.
 
     Returns a dict of bf16 bit arrays (uint16) keyed by NAMES.  For int4
     workloads it also holds '<W>_q' (packed uint8) and '<W>_scale' (float16)
-    for each frozen weight; the bf16 '<W>' entry is then absent, because the
+    for each frozen weight, for FP8 workloads '<W>_f8' (uint8 E4M3 codes) and
+    '<W>_f8scale' (float32); the bf16 '<W>' entry is then absent, because the
     frozen weight only exists in its quantised form.
     """
     rng = np.random.Generator(np.random.PCG64(cfg.seed))
@@ -150,6 +178,8 @@ def make_inputs(cfg: Config) -> dict:
             q, sc = quantize_int4(f32[k])
             out[k + "_q"] = q
             out[k + "_scale"] = sc
+        elif cfg.fp8 and k in WEIGHT_NAMES:
+            out[k + "_f8"], out[k + "_f8scale"] = quantize_fp8(f32[k])
         else:
             out[k] = f32_to_bf16_bits(f32[k])
         del f32[k]
@@ -178,6 +208,7 @@ class LinearConfig:
     alpha: float
     int4: bool = False
     index: int = 50
+    fp8: bool = False
 
     @property
     def seed(self) -> int:
@@ -213,6 +244,8 @@ def make_linear_inputs(cfg: LinearConfig) -> dict:
     for k, v in f32.items():
         if cfg.int4 and k == "W":
             out["W_q"], out["W_scale"] = quantize_int4(v)
+        elif cfg.fp8 and k == "W":
+            out["W_f8"], out["W_f8scale"] = quantize_fp8(v)
         else:
             out[k] = f32_to_bf16_bits(v)
     return out

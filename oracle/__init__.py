@@ -6,7 +6,9 @@ baseline / reference arm may import it; the product path never does.
 from .lora_mlp import (  # noqa: F401
     backward,
     bf16_to_f64,
+    dequant_fp8,
     dequant_int4,
+    e4m3_to_f64,
     f32_to_bf16_rne,
     forward,
     forward_backward,

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .lora_mlp import bf16_to_f64, dequant_int4
+from .lora_mlp import bf16_to_f64, dequant_fp8, dequant_int4
 
 
 def forward(p: dict, alpha: float) -> dict:
@@ -41,8 +41,10 @@ def backward(p: dict, alpha: float, dY: np.ndarray, fwd: dict | None = None) -> 
 
 def weights_f64(inputs: dict) -> dict:
     p = {k: bf16_to_f64(v) for k, v in inputs.items() if k in ("X", "W", "A", "B", "dY")}
-    if "W" not in p:
+    if "W" not in p and "W_q" in inputs:
         p["W"] = bf16_to_f64(dequant_int4(inputs["W_q"], inputs["W_scale"]))
+    elif "W" not in p:
+        p["W"] = bf16_to_f64(dequant_fp8(inputs["W_f8"], inputs["W_f8scale"]))
     return p
 
 

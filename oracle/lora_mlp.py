@@ -1,5 +1,5 @@
 """fp64 CPU oracle of the fused LoRA + SwiGLU MLP (forward, hand-derived backward,
-int4 dequantisation of the frozen weights).
+dequantisation of block-int4 and block-FP8 frozen weights).
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
 only tests/, __graft_entry__.smoke() and bench.py (its CPU-baseline leg and
@@ -15,14 +15,19 @@ What it follows.
     six hand-written kernel families.
   * "Unsloth 还是 AirLLM？一个炼丹，一个硬跑" (blog.cn-res.vip), section
     核心原理（为什么它快） / "Why it is fast": matrix multiplies and LoRA fused
-    into single kernels; native 4-bit QLoRA for the frozen weights.
+    into single kernels; native 4-bit QLoRA for the frozen weights; FP8 and
+    NVFP4 named as weight formats.
+  * "Unsloth 深度分析报告", section 关键设计决策: FP8 among the hand-written
+    kernel families.
 The pages print no formula.  The forward used here is the plain definition of
 a LoRA-adapted SwiGLU MLP with scale s = alpha / r,
     G = X (Wg + s Bg Ag)^T,  U = X (Wu + s Bu Au)^T,  H = silu(G) * U,
     out = H (Wd + s Bd Ad)^T,
 in the nn.Linear layout (W [out, in], A [r, in], B [out, r]).  The backward
 is that forward's chain rule, written out below; the int4 format is symmetric
-codes in [-7, 7], one fp16 absmax scale per 64 input elements, w = q*scale/7.
+codes in [-7, 7], one fp16 absmax scale per 64 input elements, w = q*scale/7;
+the FP8 format is E4M3 codes with one fp32 scale per 64 input elements,
+w = e4m3 * scale.
 
 Everything is evaluated in float64 from the exact values of the bf16 inputs,
 with every intermediate materialised.  numpy's matmul is the only library
@@ -73,16 +78,52 @@ def dequant_int4(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return f32_to_bf16_rne(w32)
 
 
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact values of FP8 E4M3 codes (the OCP 8-bit floating point format
+    "E4M3": 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; an
+    exponent field of 0 encodes subnormals, m/8 * 2^-6; no infinities; the
+    two codes S.1111.111 are NaN)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_fp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Dequantise a block-FP8 weight to bf16 bits.
+
+    codes: uint8 [rows, cols], FP8 E4M3 (see e4m3_to_f64).  scales: float32
+    [rows, cols/64], one per 64 consecutive input-dimension elements.
+    Per element, in IEEE fp32: w = fp32(e4m3) * scale (one rounding), then
+    rounded to bf16 (nearest, ties to even).  fp32(e4m3) is exact (3
+    mantissa bits, exponents -9..8).
+    """
+    codes = np.asarray(codes, dtype=np.uint8)
+    rows, cols = codes.shape
+    v32 = e4m3_to_f64(codes).astype(np.float32)          # exact
+    s32 = np.repeat(np.asarray(scales, dtype=np.float32), 64, axis=1)
+    assert s32.shape == (rows, cols)
+    with np.errstate(invalid="ignore", over="ignore"):
+        w32 = v32 * s32                                   # IEEE fp32 multiply
+    return f32_to_bf16_rne(w32)
+
+
 def weights_f64(inputs: dict) -> dict:
-    """All float inputs widened to float64; int4 frozen weights dequantised first."""
+    """All float inputs widened to float64; quantised frozen weights
+    (int4: '<W>_q', '<W>_scale'; FP8: '<W>_f8', '<W>_f8scale') dequantised first."""
     p = {}
     for k, v in inputs.items():
-        if k.endswith("_q") or k.endswith("_scale"):
+        if k.endswith(("_q", "_scale", "_f8", "_f8scale")):
             continue
         p[k] = bf16_to_f64(v)
     for w in ("Wg", "Wu", "Wd"):
-        if w not in p:
+        if w not in p and w + "_q" in inputs:
             p[w] = bf16_to_f64(dequant_int4(inputs[w + "_q"], inputs[w + "_scale"]))
+        elif w not in p and w + "_f8" in inputs:
+            p[w] = bf16_to_f64(dequant_fp8(inputs[w + "_f8"], inputs[w + "_f8scale"]))
     return p
 
 
