@@ -189,8 +189,13 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 
+def weight_format_name(cfg) -> str:
+    return "int4_b64" if cfg.int4 else ("fp8_e4m3_b64" if getattr(cfg, "fp8", False) else "bf16")
+
+
 def oracle_inputs(cfg, block=False):
-    c = synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4, seed_index=cfg.index)
+    c = synth.custom(min(cfg.N, 4096), cfg.d, cfg.d_ff, cfg.r, cfg.alpha, cfg.int4, seed_index=cfg.index,
+                     fp8=cfg.fp8)
     return synth.make_block_inputs(c) if block else synth.make_inputs(c)
 
 
@@ -297,7 +302,7 @@ def config_dict(cfg, block=False):
         d["workload"] = "llama3_8b_block" if cfg.name == "llama3_8b_mlp" else cfg.name + "_block"
         d["prenorm"] = f"RMSNorm (frozen gain), eps {synth.RMS_EPS}; out = MLP(RMSNorm(X))"
         return d
-    w_mb = 3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else 2) / 1e6
+    w_mb = 3 * cfg.d * cfg.d_ff * (0.53125 if cfg.int4 else (1.0625 if cfg.fp8 else 2)) / 1e6
     x_mb, h_mb = 2 * cfg.N * cfg.d / 1e6, 2 * cfg.N * cfg.d_ff / 1e6
     sizes = "frozen weights %.0f MB, X %.0f MB, g/u/h %.0f MB each" % (w_mb, x_mb, h_mb)
     # a step reads the weights, X, dOut and writes/reads g, u, h, dg, du
@@ -306,7 +311,7 @@ def config_dict(cfg, block=False):
           "no flush; a step's operands fit in the 126 MB L2 (%s): a launch-bound parity case, not a "
           "throughput workload" % sizes)
     return {"workload": cfg.name, "N_tokens": cfg.N, "d": cfg.d, "d_ff": cfg.d_ff, "r": cfg.r, "alpha": cfg.alpha,
-            "frozen_weights": "int4_b64" if cfg.int4 else "bf16", "l2": l2, "parallelism": "replicas"}
+            "frozen_weights": weight_format_name(cfg), "l2": l2, "parallelism": "replicas"}
 
 
 def b200_arm(args, cfg):
@@ -522,7 +527,7 @@ def linear_flops(cfg) -> dict:
 
 def linear_config_dict(cfg):
     return {"workload": cfg.name, "N_tokens": cfg.N, "d_in": cfg.d_in, "d_out": cfg.d_out, "r": cfg.r,
-            "alpha": cfg.alpha, "frozen_weights": "int4_b64" if cfg.int4 else "bf16",
+            "alpha": cfg.alpha, "frozen_weights": weight_format_name(cfg),
             "l2": "flushed: a 256 MB buffer is written between timed steps",
             "parallelism": "replicas"}
 

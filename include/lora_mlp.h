@@ -20,11 +20,11 @@
  *    frees device memory, and never synchronises the stream (except
  *    lora_mlp_device_status, which says so).  Work is enqueued on `stream`
  *    (a cudaStream_t passed as void*; NULL = the legacy default stream) on
- *    the current CUDA device.  int4 frozen weights are dequantised inside
- *    the GEMM kernels that read them; no bf16 copy of a weight is made.
+ *    the current CUDA device.  int4 and FP8 frozen weights are dequantised
+ *    inside the GEMM kernels that read them; no bf16 copy of a weight is made.
  *  - Float tensors are bf16, row-major, densely packed (leading dimension =
  *    the row length).  Device pointers must be 16-byte aligned.
- *  - Sizes: N >= 1 tokens; d, d_ff multiples of 8 (of 64 for int4 weights);
+ *  - Sizes: N >= 1 tokens; d, d_ff multiples of 8 (of 64 for int4 and FP8 weights);
  *    r a multiple of 8 in [8, 128]; alpha finite.
  *  - Results are written, never accumulated into.  Results are deterministic:
  *    the same inputs give the same bits on every run.
@@ -63,6 +63,15 @@ extern "C" {
  * scales fp16 [out, in/64] row-major.  ("native 4-bit QLoRA": blog.cn-res.vip
  * page, 核心原理; the block layout itself is this library's choice.) */
 #define LORA_MLP_WEIGHTS_INT4_B64 1
+/* FP8 codes: OCP 8-bit floating point E4M3 (1 sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; subnormals m/8 * 2^-6; no infinities; S.1111.111
+ * is NaN), one byte per element, uint8 [out, in]; one fp32 scale per 64
+ * consecutive input-dimension elements, fp32 [out, in/64] row-major:
+ * w = bf16_rne(fp32(e4m3) * scale), the fp32 product rounded once.  (The
+ * pages name FP8 as a kernel family and a weight format without defining
+ * one: "Unsloth 深度分析报告", 关键设计决策; "Unsloth 还是 AirLLM", 核心原理.
+ * The block layout and scale type are this library's choice.) */
+#define LORA_MLP_WEIGHTS_FP8_B64 2
 
 typedef struct lora_mlp_shape {
     int64_t N;             /* tokens (rows of X)          */
@@ -75,7 +84,9 @@ typedef struct lora_mlp_shape {
 
 /* Device pointers.  bf16 format: Wg, Wu [d_ff, d], Wd [d, d_ff] and Sg = Su =
  * Sd = NULL.  int4 format: Wg, Wu uint8 [d_ff, d/2], Wd uint8 [d, d_ff/2]
- * packed codes; Sg, Su fp16 [d_ff, d/64], Sd fp16 [d, d_ff/64].
+ * packed codes; Sg, Su fp16 [d_ff, d/64], Sd fp16 [d, d_ff/64].  FP8 format:
+ * Wg, Wu uint8 [d_ff, d], Wd uint8 [d, d_ff] E4M3 codes; Sg, Su fp32
+ * [d_ff, d/64], Sd fp32 [d, d_ff/64].
  * Adapters, always bf16: Ag, Au [r, d]; Bg, Bu [d_ff, r]; Ad [r, d_ff]; Bd [d, r]. */
 typedef struct lora_mlp_weights {
     const void *Wg, *Wu, *Wd;
@@ -124,6 +135,12 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w,
  * so that its bits can be checked. */
 int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, int64_t cols,
                           void* w_bf16, void* stream);
+
+/* Dequantise one block-FP8 weight (format above) to bf16 [rows, cols]; cols a
+ * multiple of 64.  The same device routine the FP8 path uses, exposed so that
+ * its bits can be checked. */
+int lora_mlp_dequant_fp8(const void* codes, const void* scales, int64_t rows, int64_t cols,
+                         void* w_bf16, void* stream);
 
 /* Reads and clears the library's device status word for the current device:
  * 0, or LORA_MLP_ERR_DEVICE_TIMEOUT if any kernel gave up a bounded wait since

@@ -26,6 +26,7 @@ CE_REDUCTION_MEAN = 2
 
 WEIGHTS_BF16 = 0
 WEIGHTS_INT4_B64 = 1
+WEIGHTS_FP8_B64 = 2
 
 WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Sg", "Su", "Sd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRAD_FIELDS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
@@ -37,6 +38,7 @@ SYMBOLS = (
     "lora_mlp_forward",
     "lora_mlp_backward",
     "lora_mlp_dequant_int4",
+    "lora_mlp_dequant_fp8",
     "lora_mlp_device_status",
     "lora_mlp_check_pointer",
     "lora_mlp_strerror",
@@ -121,6 +123,7 @@ def lib() -> ctypes.CDLL:
             L.lora_mlp_backward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp, vp,
                                             vp, ctypes.POINTER(Grads), vp, sz, vp]
             L.lora_mlp_dequant_int4.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.lora_mlp_dequant_fp8.argtypes = [vp, vp, i64, i64, vp, vp]
             L.lora_mlp_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
             L.lora_mlp_check_pointer.argtypes = [vp, sz]
             L.lora_mlp_strerror.argtypes = [ctypes.c_int]
@@ -157,7 +160,7 @@ def lib() -> ctypes.CDLL:
             L.lora_mlp_launch_count.argtypes = []
             L.lora_mlp_launch_count.restype = ctypes.c_int64
             for name in ("lora_mlp_sizes", "lora_mlp_forward", "lora_mlp_forward_noalloc", "lora_mlp_backward",
-                         "lora_mlp_dequant_int4",
+                         "lora_mlp_dequant_int4", "lora_mlp_dequant_fp8",
                          "lora_mlp_device_status", "lora_mlp_check_pointer", "lora_mlp_timing_enable",
                          "lora_mlp_timing_collect",
                          "lora_linear_sizes", "lora_linear_forward", "lora_linear_backward",
@@ -220,6 +223,10 @@ def backward(shape: Shape, weights: Weights, X, g, u, saved, dOut, dX, grads: Gr
 
 def dequant_int4(packed, scales, rows, cols, w_bf16, stream) -> int:
     return lib().lora_mlp_dequant_int4(packed, scales, int(rows), int(cols), w_bf16, stream)
+
+
+def dequant_fp8(codes, scales, rows, cols, w_bf16, stream) -> int:
+    return lib().lora_mlp_dequant_fp8(codes, scales, int(rows), int(cols), w_bf16, stream)
 
 
 def check_pointer(ptr, alignment: int = 16) -> int:

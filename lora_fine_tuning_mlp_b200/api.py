@@ -45,7 +45,8 @@ class MLPWeights:
 
     bf16 weights: Wg, Wu [d_ff, d], Wd [d, d_ff].  int4 weights: Wg, Wu uint8
     [d_ff, d/2], Wd uint8 [d, d_ff/2] and fp16 scales Sg, Su [d_ff, d/64],
-    Sd [d, d_ff/64].  Adapters (bf16): Ag, Au [r, d]; Bg, Bu [d_ff, r];
+    Sd [d, d_ff/64].  FP8 weights: Wg, Wu float8_e4m3fn [d_ff, d], Wd
+    float8_e4m3fn [d, d_ff] and fp32 scales of the int4 shapes.  Adapters (bf16): Ag, Au [r, d]; Bg, Bu [d_ff, r];
     Ad [r, d_ff]; Bd [d, r].
     """
     Wg: torch.Tensor
@@ -67,6 +68,14 @@ class MLPWeights:
         return self.Wg.dtype == torch.uint8
 
     @property
+    def fp8(self) -> bool:
+        return self.Wg.dtype == torch.float8_e4m3fn
+
+    @property
+    def fmt(self) -> int:
+        return _lib.WEIGHTS_INT4_B64 if self.int4 else (_lib.WEIGHTS_FP8_B64 if self.fp8 else _lib.WEIGHTS_BF16)
+
+    @property
     def r(self) -> int:
         return int(self.Ag.shape[0])
 
@@ -79,8 +88,7 @@ class MLPWeights:
         return int(self.Bg.shape[0])
 
     def shape(self, N: int) -> _lib.Shape:
-        fmt = _lib.WEIGHTS_INT4_B64 if self.int4 else _lib.WEIGHTS_BF16
-        return _lib.make_shape(N, self.d, self.d_ff, self.r, self.alpha, fmt)
+        return _lib.make_shape(N, self.d, self.d_ff, self.r, self.alpha, self.fmt)
 
     def validate(self):
         d, d_ff, r = self.d, self.d_ff, self.r
@@ -91,6 +99,13 @@ class MLPWeights:
             _need(self.Sg, "Sg", torch.float16, (d_ff, d // 64))
             _need(self.Su, "Su", torch.float16, (d_ff, d // 64))
             _need(self.Sd, "Sd", torch.float16, (d, d_ff // 64))
+        elif self.fp8:
+            _need(self.Wg, "Wg", torch.float8_e4m3fn, (d_ff, d))
+            _need(self.Wu, "Wu", torch.float8_e4m3fn, (d_ff, d))
+            _need(self.Wd, "Wd", torch.float8_e4m3fn, (d, d_ff))
+            _need(self.Sg, "Sg", torch.float32, (d_ff, d // 64))
+            _need(self.Su, "Su", torch.float32, (d_ff, d // 64))
+            _need(self.Sd, "Sd", torch.float32, (d, d_ff // 64))
         else:
             _need(self.Wg, "Wg", BF16, (d_ff, d))
             _need(self.Wu, "Wu", BF16, (d_ff, d))
@@ -181,6 +196,18 @@ def dequant_int4(packed: torch.Tensor, scales: torch.Tensor, stream=None) -> tor
     return w
 
 
+def dequant_fp8(codes: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """bf16 [rows, cols] from FP8 E4M3 codes [rows, cols] (float8_e4m3fn or
+    uint8) and fp32 block scales [rows, cols/64], by the library's kernel."""
+    rows, cols = codes.shape
+    if codes.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError("codes must be float8_e4m3fn or uint8")
+    _need(scales, "scales", torch.float32, (rows, cols // 64))
+    w = torch.empty((rows, cols), dtype=BF16, device=codes.device)
+    _lib.check(_lib.dequant_fp8(_p(codes), _p(scales), rows, cols, _p(w), _stream(stream)), "lora_mlp_dequant_fp8")
+    return w
+
+
 class LoRAMLPFunction(torch.autograd.Function):
     """autograd wrapper: out = LoRA-SwiGLU-MLP(X); backward fills X.grad and the
     adapter grads.  Usage: LoRAMLPFunction.apply(X, w, Ag, Bg, Au, Bu, Ad, Bd)
@@ -214,6 +241,10 @@ def weights_from_host(inp: dict, alpha: float, device="cuda") -> MLPWeights:
         for k, s in (("Wg", "Sg"), ("Wu", "Su"), ("Wd", "Sd")):
             kw[k] = torch.from_numpy(inp[k + "_q"]).to(device)
             kw[s] = torch.from_numpy(inp[k + "_scale"]).to(device)
+    elif "Wg_f8" in inp:
+        for k, s in (("Wg", "Sg"), ("Wu", "Su"), ("Wd", "Sd")):
+            kw[k] = torch.from_numpy(inp[k + "_f8"]).view(torch.float8_e4m3fn).to(device)
+            kw[s] = torch.from_numpy(inp[k + "_f8scale"]).to(device)
     else:
         for k in ("Wg", "Wu", "Wd"):
             kw[k] = bf(inp[k])
@@ -329,6 +360,7 @@ class LinearWeights:
     """One frozen projection with a LoRA adapter (nn.Linear layout).
 
     bf16: W [d_out, d_in].  int4: W uint8 [d_out, d_in/2] and fp16 scales
+    S [d_out, d_in/64].  FP8: W float8_e4m3fn [d_out, d_in] and fp32 scales
     S [d_out, d_in/64].  Adapter (bf16): A [r, d_in], B [d_out, r].
     """
     W: torch.Tensor
@@ -340,6 +372,10 @@ class LinearWeights:
     @property
     def int4(self) -> bool:
         return self.W.dtype == torch.uint8
+
+    @property
+    def fp8(self) -> bool:
+        return self.W.dtype == torch.float8_e4m3fn
 
     @property
     def r(self) -> int:
@@ -354,7 +390,7 @@ class LinearWeights:
         return int(self.B.shape[0])
 
     def shape(self, N: int) -> _lib.LinShape:
-        fmt = _lib.WEIGHTS_INT4_B64 if self.int4 else _lib.WEIGHTS_BF16
+        fmt = _lib.WEIGHTS_INT4_B64 if self.int4 else (_lib.WEIGHTS_FP8_B64 if self.fp8 else _lib.WEIGHTS_BF16)
         return _lib.make_lin_shape(N, self.d_in, self.d_out, self.r, self.alpha, fmt)
 
     def validate(self):
@@ -362,6 +398,9 @@ class LinearWeights:
         if self.int4:
             _need(self.W, "W", torch.uint8, (do, di // 2))
             _need(self.S, "S", torch.float16, (do, di // 64))
+        elif self.fp8:
+            _need(self.W, "W", torch.float8_e4m3fn, (do, di))
+            _need(self.S, "S", torch.float32, (do, di // 64))
         else:
             _need(self.W, "W", BF16, (do, di))
         _need(self.A, "A", BF16, (r, di))
@@ -440,6 +479,10 @@ def linear_weights_from_host(inp: dict, alpha: float, device="cuda") -> LinearWe
         return LinearWeights(W=torch.from_numpy(inp["W_q"]).to(device), A=to_device_bf16(inp["A"], device),
                              B=to_device_bf16(inp["B"], device), alpha=float(alpha),
                              S=torch.from_numpy(inp["W_scale"]).to(device))
+    if "W_f8" in inp:
+        return LinearWeights(W=torch.from_numpy(inp["W_f8"]).view(torch.float8_e4m3fn).to(device),
+                             A=to_device_bf16(inp["A"], device), B=to_device_bf16(inp["B"], device),
+                             alpha=float(alpha), S=torch.from_numpy(inp["W_f8scale"]).to(device))
     return LinearWeights(W=to_device_bf16(inp["W"], device), A=to_device_bf16(inp["A"], device),
                          B=to_device_bf16(inp["B"], device), alpha=float(alpha))
 

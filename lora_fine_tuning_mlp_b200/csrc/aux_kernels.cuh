@@ -137,18 +137,76 @@ __global__ void __launch_bounds__(kDqThreads) dequant_int4_kernel(const uint4* _
     }
 }
 
+// ---------------------------------------------------------------- FP8 (E4M3)
+
+// Four codes (one 4-byte word, element e in byte e) -> four bf16 values
+// bf16_rne(fp32(e4m3) * scale): the f16 values widen exactly to fp32, one
+// fp32 multiply per element (two lanes per instruction), one rounding to
+// bf16.  s2 = {scale, scale}.
+__device__ __forceinline__ uint2 fp8_expand4(uint32_t w, uint64_t s2) {
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(h01), "=r"(h23)
+        : "r"(w));
+    float f0, f1, f2, f3;
+    asm("{\n\t.reg .b16 a, b, c, d;\n\tmov.b32 {a, b}, %4;\n\tmov.b32 {c, d}, %5;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\tcvt.f32.f16 %2, c;\n\tcvt.f32.f16 %3, d;\n\t}"
+        : "=f"(f0), "=f"(f1), "=f"(f2), "=f"(f3)
+        : "r"(h01), "r"(h23));
+    float p0, p1, p2, p3;
+    f2_unpack(f2_mul(f2_packf(f0, f1), s2), p0, p1);
+    f2_unpack(f2_mul(f2_packf(f2, f3), s2), p2, p3);
+    return make_uint2(bf16x2_bits(p0, p1), bf16x2_bits(p2, p3));
+}
+
+// One 64-element line: 64 code bytes (c[0] holds elements 0..15) -> 128
+// bytes of bf16 (out[q] holds elements 8q .. 8q + 7).
+__device__ __forceinline__ void fp8_line(const uint4 (&c)[4], float scale, uint4 (&out)[8]) {
+    const uint64_t s2 = f2_packf(scale, scale);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint2 a = fp8_expand4(c[i].x, s2), b = fp8_expand4(c[i].y, s2);
+        const uint2 e = fp8_expand4(c[i].z, s2), f = fp8_expand4(c[i].w, s2);
+        out[2 * i] = make_uint4(a.x, a.y, b.x, b.y);
+        out[2 * i + 1] = make_uint4(e.x, e.y, f.x, f.y);
+    }
+}
+
+// The standalone FP8 dequantisation, one thread per line: codes [rows, cols]
+// and scales [rows, cols/64] (fp32) row-major, so line L is code bytes 64L ..,
+// scale L and output bytes 128L ..  The GEMMs' dequant warps run the same
+// fp8_line on their stage's lines.
+__global__ void __launch_bounds__(kDqThreads) dequant_fp8_kernel(const uint4* __restrict__ codes,
+                                                                 const float* __restrict__ scales,
+                                                                 long long nlines, uint4* __restrict__ w) {
+    for (long long L = static_cast<long long>(blockIdx.x) * kDqThreads + threadIdx.x; L < nlines;
+         L += static_cast<long long>(gridDim.x) * kDqThreads) {
+        uint4 c[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = __ldcs(codes + 4 * L + i);
+        uint4 o[8];
+        fp8_line(c, scales[L], o);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) __stcs(w + 8 * L + q, o[q]);
+    }
+}
+
 // Block scales [rows, nb] (nb = cols / 64) -> their transpose [nb, rows], so
 // that the scales of one 64-column block of consecutive rows are contiguous
 // and a GEMM stage can fetch them with one TMA box.  Up to three matrices per
 // launch (blockIdx.z), 32 x 32 tiles through shared memory.
+// T: unsigned short (int4's fp16 scales) or unsigned int (FP8's fp32 scales).
+template <class T>
 struct ScaleT {
-    const unsigned short* src[3];
-    unsigned short* dst[3];
+    const T* src[3];
+    T* dst[3];
     int rows[3], nb[3];
 };
 
-__global__ void __launch_bounds__(256) scale_transpose_kernel(const ScaleT a) {
-    __shared__ unsigned short tile[32][33];
+template <class T>
+__global__ void __launch_bounds__(256) scale_transpose_kernel(const ScaleT<T> a) {
+    __shared__ T tile[32][33];
     const int z = blockIdx.z;
     const int rows = a.rows[z], nb = a.nb[z];
     const int r0 = blockIdx.x * 32, b0 = blockIdx.y * 32;

@@ -185,19 +185,21 @@ bool encode_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, i
 
 // Tiled, unswizzled TMA descriptor of a byte matrix [outer, inner] (row
 // stride ld bytes, a multiple of 16) with a box_inner x box_outer box: the
-// packed codes of an int4 weight.  Out-of-range bytes read as zero.
-// (elem = 2: a 16-bit matrix, the transposed int4 scales; ld then in
-// elements.)
+// codes of an int4 or FP8 weight.  Out-of-range bytes read as zero.
+// (elem = 2 or 4: a 16- or 32-bit matrix, the transposed block scales; ld
+// then in elements.)
 bool encode_map_u8(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, uint32_t box_inner,
-                   uint32_t box_outer, int elem = 1) {
+                   uint32_t box_outer, int elem = 1, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * static_cast<cuuint64_t>(elem)};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
-    return fn(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr),
-              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    const CUtensorMapDataType ty = elem == 4   ? CU_TENSOR_MAP_DATA_TYPE_UINT32
+                                   : elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    return fn(m, ty, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -418,25 +420,31 @@ struct PairBuilder {
         return nmaps++;
     }
     int b_mn(const void* p, int64_t K, int64_t Nn, int64_t ld) { return map(p, Nn, K, ld, 64, kBK); }
-    // Packed int4 codes of a weight [rows, cols] (uint8 [rows, cols/2]):
-    // read K-major (K = cols), 32 bytes x 128 rows per box, or MN-major
-    // (K = rows), 32 bytes x 64 rows per box.
-    int q_map(const void* codes, int64_t rows, int64_t cols, bool mn) {
+    // The codes of a quantised weight [rows, cols]: int4 (uint8 [rows,
+    // cols/2], 32-byte line rows) or FP8 (uint8 [rows, cols], 64-byte line
+    // rows in TMA's 64-byte swizzle), read K-major (K = cols, 128 rows per
+    // box) or MN-major (K = rows, 64 rows per box).
+    int q_map(const void* codes, int64_t rows, int64_t cols, bool mn, int qf) {
         if (nmaps >= kMaxMaps) {
             ok = false;
             return 0;
         }
-        if (!encode_map_u8(&a.maps[nmaps], codes, cols / 2, rows, cols / 2, 32, mn ? 64 : kPairHalfN)) ok = false;
+        const bool f8 = qf == QF_FP8;
+        const int64_t inner = f8 ? cols : cols / 2;
+        if (!encode_map_u8(&a.maps[nmaps], codes, inner, rows, inner, f8 ? 64 : 32, mn ? 64 : kPairHalfN, 1,
+                           f8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
+            ok = false;
         return nmaps++;
     }
     // The transposed scales [cols/64, rows] of a weight [rows, cols]: one
     // box holds the scales of 128 consecutive rows (K-major B) or 64 (MN-major).
-    int s_map(const void* st, int64_t rows, int64_t cols, bool mn) {
+    int s_map(const void* st, int64_t rows, int64_t cols, bool mn, int qf) {
         if (nmaps >= kMaxMaps) {
             ok = false;
             return 0;
         }
-        if (!encode_map_u8(&a.maps[nmaps], st, rows, cols / 64, rows, mn ? 64 : kPairHalfN, 1, 2)) ok = false;
+        if (!encode_map_u8(&a.maps[nmaps], st, rows, cols / 64, rows, mn ? 64 : kPairHalfN, 1, qf == QF_FP8 ? 4 : 2))
+            ok = false;
         return nmaps++;
     }
     // Marks segment `sg` as reading int4 B: code and scale maps of halves 0 / 1.
@@ -481,8 +489,9 @@ int pair_tail_splits(int tiles, int clusters, int nkb) {
     return 2;
 }
 
-template <bool B_MN, int EPI, bool Q4 = false>
+template <bool B_MN, int EPI, int QF = QF_NONE>
 int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, float* tail_part, int* tail_ctr) {
+    constexpr bool Q4 = QF != QF_NONE;
     if constexpr (pair_tma_store<EPI>()) {
         b.a.prob.omap[0] = b.out_map(b.a.prob.out0);
         if (EPI != EPI_BF16) {
@@ -501,14 +510,14 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     a.tail_ctr = tail_ctr;
     // (512-byte alignment) epilogue store staging per warp, then the dH epilogue's g/u rings
     const uint32_t staging = 512 + pair_epi_warps<EPI>() * pair_stage_warp_bytes<EPI>() + pair_ring_bytes<EPI>();
-    constexpr uint32_t kSB = pair_stage_bytes<Q4>();
+    constexpr uint32_t kSB = pair_stage_bytes<QF>();
     const uint32_t budget = kSmemLimit - 1024 - gemm_ctl_bytes() - staging;
     int stages = static_cast<int>(budget / kSB);
     if (stages > kPairMaxStages) stages = kPairMaxStages;
     if (stages < 2) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     const size_t smem = 1024 + static_cast<size_t>(stages) * kSB + gemm_ctl_bytes() + staging;
-    auto kern = umma2_gemm_kernel<B_MN, EPI, Q4>;
+    auto kern = umma2_gemm_kernel<B_MN, EPI, QF>;
     static int max_clusters[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -558,6 +567,15 @@ int launch_pair(PairBuilder& b, int sms, cudaStream_t st, const char* name, floa
     return last_launch_error();
 }
 
+// launch_pair with the weight format chosen at run time.
+template <bool B_MN, int EPI>
+int launch_pair_q(PairBuilder& b, int qf, int sms, cudaStream_t st, const char* name, float* tail_part,
+                  int* tail_ctr) {
+    if (qf == QF_INT4) return launch_pair<B_MN, EPI, QF_INT4>(b, sms, st, name, tail_part, tail_ctr);
+    if (qf == QF_FP8) return launch_pair<B_MN, EPI, QF_FP8>(b, sms, st, name, tail_part, tail_ctr);
+    return launch_pair<B_MN, EPI, QF_NONE>(b, sms, st, name, tail_part, tail_ctr);
+}
+
 int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
                    cudaStream_t st) {
     const long long nlines = rows * (cols / 64);  // one scale and 64 elements per line
@@ -573,25 +591,47 @@ int launch_dequant(const void* packed, const void* scales, int64_t rows, int64_t
     return last_launch_error();
 }
 
+int launch_dequant_fp8(const void* codes, const void* scales, int64_t rows, int64_t cols, void* w, int sms,
+                       cudaStream_t st) {
+    const long long nlines = rows * (cols / 64);
+    long long blocks = (nlines + kDqThreads - 1) / kDqThreads;
+    const long long cap = static_cast<long long>(sms) * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    {
+        LaunchScope scope("dequant_fp8", st);
+        dequant_fp8_kernel<<<static_cast<int>(blocks), kDqThreads, 0, st>>>(
+            static_cast<const uint4*>(codes), static_cast<const float*>(scales), nlines, static_cast<uint4*>(w));
+    }
+    return last_launch_error();
+}
+
 // Transposes up to three block-scale matrices [rows, cols/64] into
-// [cols/64, rows] (scale_transpose_kernel), one launch.
-int launch_scale_t(int n, const void* const* src, void* const* dst, const int64_t* rows, const int64_t* cols,
-                   cudaStream_t st) {
-    ScaleT a{};
+// [cols/64, rows] (scale_transpose_kernel), one launch; elements of 2 bytes
+// (int4's fp16 scales) or 4 (FP8's fp32 scales).
+template <class T>
+int launch_scale_t_typed(int n, const void* const* src, void* const* dst, const int64_t* rows,
+                         const int64_t* cols, cudaStream_t st) {
+    ScaleT<T> a{};
     unsigned gx = 1, gy = 1;
     for (int i = 0; i < n; ++i) {
-        a.src[i] = static_cast<const unsigned short*>(src[i]);
-        a.dst[i] = static_cast<unsigned short*>(dst[i]);
+        a.src[i] = static_cast<const T*>(src[i]);
+        a.dst[i] = static_cast<T*>(dst[i]);
         a.rows[i] = static_cast<int>(rows[i]);
         a.nb[i] = static_cast<int>(cols[i] / 64);
         gx = std::max(gx, static_cast<unsigned>((rows[i] + 31) / 32));
         gy = std::max(gy, static_cast<unsigned>((cols[i] / 64 + 31) / 32));
     }
     {
-        LaunchScope scope("int4_scales_t", st);
-        scale_transpose_kernel<<<dim3(gx, gy, n), 256, 0, st>>>(a);
+        LaunchScope scope("scales_t", st);
+        scale_transpose_kernel<T><<<dim3(gx, gy, n), 256, 0, st>>>(a);
     }
     return last_launch_error();
+}
+int launch_scale_t(int qf, int n, const void* const* src, void* const* dst, const int64_t* rows,
+                   const int64_t* cols, cudaStream_t st) {
+    return qf == QF_FP8 ? launch_scale_t_typed<unsigned int>(n, src, dst, rows, cols, st)
+                        : launch_scale_t_typed<unsigned short>(n, src, dst, rows, cols, st);
 }
 
 // ----------------------------------------------------------------------------- layout
@@ -657,13 +697,13 @@ constexpr int kSkinnySlots[SK_COUNT] = {kTargetCtas, 2 * kTargetCtas, 2 * kTarge
 struct Plan {
     int64_t N, d, d_ff, r, ldN;
     float s;
-    bool int4;
+    int qf;  // frozen-weight format: QF_NONE (bf16), QF_INT4, QF_FP8
     int bn_r, bn_r64, bn_2r;
     SkinnySpec spec[SK_COUNT][kMaxProbs];
     int splits[SK_COUNT][kMaxProbs];
     size_t part_off[SK_COUNT][kMaxProbs];  // float offset of each problem's partials
     // forward workspace
-    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_st[3], f_total;  // f_st: int4 scales, transposed
+    size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_st[3], f_total;  // f_st: block scales, transposed
     // backward workspace
     size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_st[3], b_total;
     size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
@@ -688,7 +728,9 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.r = sh.r;
     p.ldN = round_up(sh.N, 8);
     p.s = static_cast<float>(static_cast<double>(sh.alpha) / static_cast<double>(sh.r));
-    p.int4 = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64;
+    p.qf = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64  ? QF_INT4
+           : sh.weight_format == LORA_MLP_WEIGHTS_FP8_B64 ? QF_FP8
+                                                           : QF_NONE;
     p.bn_r = static_cast<int>(round_up(sh.r, 32));
     p.bn_r64 = static_cast<int>(round_up(sh.r, 64));
     p.bn_2r = static_cast<int>(round_up(2 * sh.r, 32));
@@ -733,8 +775,9 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
     p.f_tail = f.take(kTailPartFloats * f32);
-    const size_t stsz = static_cast<size_t>(d) * static_cast<size_t>(dff) / 64 * 2;  // one weight's scales
-    for (int i = 0; i < 3; ++i) p.f_st[i] = p.int4 ? f.take(stsz) : 0;
+    // one weight's block scales (fp16 for int4, fp32 for FP8)
+    const size_t stsz = static_cast<size_t>(d) * static_cast<size_t>(dff) / 64 * (p.qf == QF_FP8 ? 4 : 2);
+    for (int i = 0; i < 3; ++i) p.f_st[i] = p.qf ? f.take(stsz) : 0;
     p.f_total = f.off;
 
     Carver b;
@@ -748,7 +791,7 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
-    for (int i = 0; i < 3; ++i) p.b_st[i] = p.int4 ? b.take(stsz) : 0;
+    for (int i = 0; i < 3; ++i) p.b_st[i] = p.qf ? b.take(stsz) : 0;
     p.b_total = b.off;
 
     Carver sv;
@@ -767,11 +810,12 @@ int validate_shape(const lora_mlp_shape* sh) {
     if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
     if (sh->N < 1 || sh->d < 1 || sh->d_ff < 1 || sh->r < 1) return LORA_MLP_ERR_INVALID_ARG;
     if (!std::isfinite(sh->alpha)) return LORA_MLP_ERR_INVALID_ARG;
-    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64)
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64 &&
+        sh->weight_format != LORA_MLP_WEIGHTS_FP8_B64)
         return LORA_MLP_ERR_INVALID_ARG;
     if (sh->d % 8 || sh->d_ff % 8 || sh->r % 8) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     if (sh->r > 128) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64 && (sh->d % 64 || sh->d_ff % 64))
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && (sh->d % 64 || sh->d_ff % 64))
         return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     const int64_t lim = (int64_t{1} << 31) - 1;
     if (sh->N > lim || sh->d > lim || sh->d_ff > lim) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
@@ -792,7 +836,7 @@ int check_weights(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
     if (w == nullptr) return LORA_MLP_ERR_INVALID_ARG;
     int rc = check_ptrs({w->Wg, w->Wu, w->Wd, w->Ag, w->Bg, w->Au, w->Bu, w->Ad, w->Bd});
     if (rc) return rc;
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_ptrs({w->Sg, w->Su, w->Sd});
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16) return check_ptrs({w->Sg, w->Su, w->Sd});
     return LORA_MLP_OK;
 }
 
@@ -822,7 +866,7 @@ int check_memory(std::initializer_list<const void*> ps) {
 int check_weight_memory(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
     const int rc = check_memory({w->Wg, w->Wu, w->Wd, w->Ag, w->Bg, w->Au, w->Bu, w->Ad, w->Bd});
     if (rc != LORA_MLP_OK) return rc;
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_memory({w->Sg, w->Su, w->Sd});
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16) return check_memory({w->Sg, w->Su, w->Sd});
     return LORA_MLP_OK;
 }
 
@@ -832,14 +876,14 @@ int check_weight_memory(const lora_mlp_shape* sh, const lora_mlp_weights* w) {
         if (rc_ != LORA_MLP_OK) return rc_; \
     } while (0)
 
-// int4: the three weights' scales, transposed into the workspace at off[0..2]
+// int4 / FP8: the three weights' scales, transposed into the workspace at off[0..2]
 // (Wg, Wu, Wd) for the GEMMs' scale maps.
 int mlp_scales_t(const Plan& pl, const lora_mlp_weights* w, uint8_t* ws, const size_t* off, cudaStream_t st) {
     const void* src[3] = {w->Sg, w->Su, w->Sd};
     void* dst[3] = {ws + off[0], ws + off[1], ws + off[2]};
     const int64_t rows[3] = {pl.d_ff, pl.d_ff, pl.d};
     const int64_t cols[3] = {pl.d, pl.d, pl.d_ff};
-    return launch_scale_t(3, src, dst, rows, cols, st);
+    return launch_scale_t(pl.qf, 3, src, dst, rows, cols, st);
 }
 
 }  // namespace
@@ -884,7 +928,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    if (pl.int4) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.f_st, st));
+    if (pl.qf) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.f_st, st));
     {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ax = b.a_k(X, N, d, d);
@@ -903,8 +947,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         PairBuilder b(N, dff, 128);
         const int ax = b.a_k(X, N, d, d);
         const int asgu = b.a_k(Sgu, N, 2 * r, 2 * r);
-        const int bwg = pl.int4 ? b.q_map(w->Wg, dff, d, false) : b.b_k(w->Wg, dff, d, d);
-        const int bwu = pl.int4 ? b.q_map(w->Wu, dff, d, false) : b.b_k(w->Wu, dff, d, d);
+        const int bwg = pl.qf ? b.q_map(w->Wg, dff, d, false, pl.qf) : b.b_k(w->Wg, dff, d, d);
+        const int bwu = pl.qf ? b.q_map(w->Wu, dff, d, false, pl.qf) : b.b_k(w->Wu, dff, d, d);
         const int bbg = b.b_k(w->Bg, dff, r, r);
         const int bbu = b.b_k(w->Bu, dff, r, r);
         b.seg(ax, bwg, bwu, 0, 0, 0, 0, d);
@@ -913,12 +957,12 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.out1 = u;
         b.a.prob.out2 = h;
         b.a.prob.ld = dff;
-        if (pl.int4) {
-            b.quant(0, bwg, bwu, b.s_map(ws + pl.f_st[0], dff, d, false), b.s_map(ws + pl.f_st[1], dff, d, false));
-            LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD, true>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<false, EPI_SWIGLU_FWD>(b, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
+        if (pl.qf) {
+            const int sg = b.s_map(ws + pl.f_st[0], dff, d, false, pl.qf);
+            const int su = b.s_map(ws + pl.f_st[1], dff, d, false, pl.qf);
+            b.quant(0, bwg, bwu, sg, su);
         }
+        LMLP_TRY((launch_pair_q<false, EPI_SWIGLU_FWD>(b, pl.qf, di.sms, st, "F1_gate_up_swiglu", tailp, ctr)));
     }
     {  // F2: S_d = s h Ad^T  -> Sd [N, r] and saved S_d^T [r, ldN]
         GemmBuilder b(pl.bn_r);
@@ -936,19 +980,17 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         PairBuilder b(N, d, 256);
         const int ah = b.a_k(h, N, dff, dff);
         const int asd = b.a_k(Sd, N, r, r);
-        const int bwd = pl.int4 ? b.q_map(w->Wd, d, dff, false) : b.b_k(w->Wd, d, dff, dff);
+        const int bwd = pl.qf ? b.q_map(w->Wd, d, dff, false, pl.qf) : b.b_k(w->Wd, d, dff, dff);
         const int bbd = b.b_k(w->Bd, d, r, r);
         b.seg(ah, bwd, bwd, 0, kPairHalfN, 0, 0, dff);
         b.seg(asd, bbd, bbd, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = out;
         b.a.prob.ld = d;
-        if (pl.int4) {
-            const int sd = b.s_map(ws + pl.f_st[2], d, dff, false);
+        if (pl.qf) {
+            const int sd = b.s_map(ws + pl.f_st[2], d, dff, false, pl.qf);
             b.quant(0, bwd, bwd, sd, sd);
-            LMLP_TRY((launch_pair<false, EPI_BF16, true>(b, di.sms, st, "F3_down", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "F3_down", tailp, ctr)));
         }
+        LMLP_TRY((launch_pair_q<false, EPI_BF16>(b, pl.qf, di.sms, st, "F3_down", tailp, ctr)));
     }
     return LORA_MLP_OK;
 }
@@ -983,7 +1025,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
     int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    if (pl.int4) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.b_st, st));
+    if (pl.qf) LMLP_TRY(mlp_scales_t(pl, w, ws, pl.b_st, st));
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
@@ -1013,7 +1055,7 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         PairBuilder b(N, dff, 256);
         const int a = b.a_k(dOut, N, d, d);
         const int atd = b.a_k(Td, N, r, r);
-        const int bwd = pl.int4 ? b.q_map(w->Wd, d, dff, true) : b.b_mn(w->Wd, d, dff, dff);
+        const int bwd = pl.qf ? b.q_map(w->Wd, d, dff, true, pl.qf) : b.b_mn(w->Wd, d, dff, dff);
         const int bad = b.b_mn(w->Ad, r, dff, dff);
         b.seg(a, bwd, bwd, 0, kPairHalfN, 0, 0, d);
         b.seg(atd, bad, bad, 0, kPairHalfN, 0, 0, r);
@@ -1024,13 +1066,11 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p.out1 = du;
         p.out2 = hb;
         p.ld = dff;
-        if (pl.int4) {
-            const int sd = b.s_map(ws + pl.b_st[2], d, dff, true);
+        if (pl.qf) {
+            const int sd = b.s_map(ws + pl.b_st[2], d, dff, true, pl.qf);
             b.quant(0, bwd, bwd, sd, sd);
-            LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD, true>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<true, EPI_SWIGLU_BWD>(b, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
         }
+        LMLP_TRY((launch_pair_q<true, EPI_SWIGLU_BWD>(b, pl.qf, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
     }
     {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
        //        dAd = T_d^T h (written transposed);  dBg = dg^T S_g, dBu = du^T S_u
@@ -1094,8 +1134,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         const int adu = b.a_k(du, N, dff, dff);
         const int atg = b.a_k(Tgu, N, r, 2 * r);
         const int atu = b.a_k(Tgu + r, N, r, 2 * r);
-        const int bwg = pl.int4 ? b.q_map(w->Wg, dff, d, true) : b.b_mn(w->Wg, dff, d, d);
-        const int bwu = pl.int4 ? b.q_map(w->Wu, dff, d, true) : b.b_mn(w->Wu, dff, d, d);
+        const int bwg = pl.qf ? b.q_map(w->Wg, dff, d, true, pl.qf) : b.b_mn(w->Wg, dff, d, d);
+        const int bwu = pl.qf ? b.q_map(w->Wu, dff, d, true, pl.qf) : b.b_mn(w->Wu, dff, d, d);
         const int bag = b.b_mn(w->Ag, r, d, d);
         const int bau = b.b_mn(w->Au, r, d, d);
         b.seg(adg, bwg, bwg, 0, kPairHalfN, 0, 0, dff);
@@ -1104,15 +1144,13 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         b.seg(atu, bau, bau, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = dX;
         b.a.prob.ld = d;
-        if (pl.int4) {
-            const int sg = b.s_map(ws + pl.b_st[0], dff, d, true);
-            const int su = b.s_map(ws + pl.b_st[1], dff, d, true);
+        if (pl.qf) {
+            const int sg = b.s_map(ws + pl.b_st[0], dff, d, true, pl.qf);
+            const int su = b.s_map(ws + pl.b_st[1], dff, d, true, pl.qf);
             b.quant(0, bwg, bwg, sg, sg);
             b.quant(1, bwu, bwu, su, su);
-            LMLP_TRY((launch_pair<true, EPI_BF16, true>(b, di.sms, st, "B4_dX", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "B4_dX", tailp, ctr)));
         }
+        LMLP_TRY((launch_pair_q<true, EPI_BF16>(b, pl.qf, di.sms, st, "B4_dX", tailp, ctr)));
     }
     {  // B5: [dAg; dAu]^T = X^T [T_g | T_u]  (written transposed: dAg, dAu [r, d])
         GemmBuilder b(pl.bn_2r);
@@ -1138,6 +1176,17 @@ int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, 
     DevInfo di;
     LMLP_TRY(device_info(&di));
     return launch_dequant(packed, scales, rows, cols, w_bf16, di.sms, static_cast<cudaStream_t>(stream));
+}
+
+int lora_mlp_dequant_fp8(const void* codes, const void* scales, int64_t rows, int64_t cols, void* w_bf16,
+                         void* stream) {
+    if (rows < 1 || cols < 1) return LORA_MLP_ERR_INVALID_ARG;
+    if (cols % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    LMLP_TRY(check_ptrs({codes, scales, w_bf16}));
+    LMLP_TRY(check_memory({codes, scales, w_bf16}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return launch_dequant_fp8(codes, scales, rows, cols, w_bf16, di.sms, static_cast<cudaStream_t>(stream));
 }
 
 int lora_mlp_check_pointer(const void* p, size_t alignment) {
@@ -1229,13 +1278,13 @@ constexpr int kLinProbs[LK_COUNT] = {1, 2, 1};
 struct LinPlan {
     int64_t N, din, dout, r, ldN;
     float s;
-    bool int4;
+    int qf;  // frozen-weight format
     int bn_r, bn_r64;
     SkinnySpec spec[LK_COUNT][kMaxProbs];
     int splits[LK_COUNT][kMaxProbs];
     size_t part_off[LK_COUNT][kMaxProbs];
     size_t ctr_bytes;
-    size_t f_r, f_part, f_ctr, f_tail, f_st, f_total;  // f_st, b_st: int4 scales, transposed
+    size_t f_r, f_part, f_ctr, f_tail, f_st, f_total;  // f_st, b_st: block scales, transposed
     size_t b_t, b_tT, b_part, b_ctr, b_tail, b_st, b_total;
     size_t s_rT, s_total;
 };
@@ -1248,7 +1297,9 @@ LinPlan make_lin_plan(const lora_linear_shape& sh) {
     p.r = sh.r;
     p.ldN = round_up(sh.N, 8);
     p.s = static_cast<float>(static_cast<double>(sh.alpha) / static_cast<double>(sh.r));
-    p.int4 = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64;
+    p.qf = sh.weight_format == LORA_MLP_WEIGHTS_INT4_B64  ? QF_INT4
+           : sh.weight_format == LORA_MLP_WEIGHTS_FP8_B64 ? QF_FP8
+                                                           : QF_NONE;
     p.bn_r = static_cast<int>(round_up(sh.r, 32));
     p.bn_r64 = static_cast<int>(round_up(sh.r, 64));
     const int64_t N = p.N, di = p.din, dout = p.dout, r = p.r;
@@ -1277,8 +1328,8 @@ LinPlan make_lin_plan(const lora_linear_shape& sh) {
     p.f_part = f.take(part_f * f32);
     p.f_ctr = f.take(p.ctr_bytes);
     p.f_tail = f.take(kTailPartFloats * f32);
-    const size_t stsz = static_cast<size_t>(dout) * static_cast<size_t>(di) / 64 * 2;
-    p.f_st = p.int4 ? f.take(stsz) : 0;
+    const size_t stsz = static_cast<size_t>(dout) * static_cast<size_t>(di) / 64 * (p.qf == QF_FP8 ? 4 : 2);
+    p.f_st = p.qf ? f.take(stsz) : 0;
     p.f_total = f.off;
     Carver b;
     p.b_t = b.take(static_cast<size_t>(N) * rz * bf);
@@ -1286,7 +1337,7 @@ LinPlan make_lin_plan(const lora_linear_shape& sh) {
     p.b_part = b.take(part_b * f32);
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
-    p.b_st = p.int4 ? b.take(stsz) : 0;
+    p.b_st = p.qf ? b.take(stsz) : 0;
     p.b_total = b.off;
     Carver sv;
     p.s_rT = sv.take(rz * ldN * bf);
@@ -1298,10 +1349,11 @@ int validate_lin_shape(const lora_linear_shape* sh) {
     if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
     if (sh->N < 1 || sh->d_in < 1 || sh->d_out < 1 || sh->r < 1) return LORA_MLP_ERR_INVALID_ARG;
     if (!std::isfinite(sh->alpha)) return LORA_MLP_ERR_INVALID_ARG;
-    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64)
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->weight_format != LORA_MLP_WEIGHTS_INT4_B64 &&
+        sh->weight_format != LORA_MLP_WEIGHTS_FP8_B64)
         return LORA_MLP_ERR_INVALID_ARG;
     if (sh->d_in % 8 || sh->d_out % 8 || sh->r % 8 || sh->r > 128) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64 && sh->d_in % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16 && sh->d_in % 64) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     const int64_t lim = (int64_t{1} << 31) - 1;
     if (sh->N > lim || sh->d_in > lim || sh->d_out > lim) return LORA_MLP_ERR_UNSUPPORTED_SHAPE;
     return LORA_MLP_OK;
@@ -1310,12 +1362,12 @@ int validate_lin_shape(const lora_linear_shape* sh) {
 int check_lin_weights(const lora_linear_shape* sh, const lora_linear_weights* w) {
     if (w == nullptr) return LORA_MLP_ERR_INVALID_ARG;
     LMLP_TRY(check_ptrs({w->W, w->A, w->B}));
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_ptrs({w->S});
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16) return check_ptrs({w->S});
     return LORA_MLP_OK;
 }
 int check_lin_weight_memory(const lora_linear_shape* sh, const lora_linear_weights* w) {
     LMLP_TRY(check_memory({w->W, w->A, w->B}));
-    if (sh->weight_format == LORA_MLP_WEIGHTS_INT4_B64) return check_memory({w->S});
+    if (sh->weight_format != LORA_MLP_WEIGHTS_BF16) return check_memory({w->S});
     return LORA_MLP_OK;
 }
 
@@ -1353,10 +1405,10 @@ int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weight
     int* ctr = reinterpret_cast<int*>(ws + pl.f_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.f_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    if (pl.int4) {
+    if (pl.qf) {
         const void* src = w->S;
         void* dst = ws + pl.f_st;
-        LMLP_TRY(launch_scale_t(1, &src, &dst, &pl.dout, &pl.din, st));
+        LMLP_TRY(launch_scale_t(pl.qf, 1, &src, &dst, &pl.dout, &pl.din, st));
     }
     {  // L0: R = s X A^T -> R [N, r], saved R^T [r, ldN]
         GemmBuilder b(pl.bn_r);
@@ -1374,19 +1426,17 @@ int lora_linear_forward(const lora_linear_shape* shape, const lora_linear_weight
         PairBuilder b(N, dout, 256);
         const int ax = b.a_k(X, N, din, din);
         const int ar = b.a_k(R, N, r, r);
-        const int bw = pl.int4 ? b.q_map(w->W, dout, din, false) : b.b_k(w->W, dout, din, din);
+        const int bw = pl.qf ? b.q_map(w->W, dout, din, false, pl.qf) : b.b_k(w->W, dout, din, din);
         const int bb = b.b_k(w->B, dout, r, r);
         b.seg(ax, bw, bw, 0, kPairHalfN, 0, 0, din);
         b.seg(ar, bb, bb, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = Y;
         b.a.prob.ld = dout;
-        if (pl.int4) {
-            const int sm = b.s_map(ws + pl.f_st, dout, din, false);
+        if (pl.qf) {
+            const int sm = b.s_map(ws + pl.f_st, dout, din, false, pl.qf);
             b.quant(0, bw, bw, sm, sm);
-            LMLP_TRY((launch_pair<false, EPI_BF16, true>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<false, EPI_BF16>(b, di.sms, st, "L1_linear_fwd", tailp, ctr)));
         }
+        LMLP_TRY((launch_pair_q<false, EPI_BF16>(b, pl.qf, di.sms, st, "L1_linear_fwd", tailp, ctr)));
     }
     return LORA_MLP_OK;
 }
@@ -1413,10 +1463,10 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
     int* ctr = reinterpret_cast<int*>(ws + pl.b_ctr);
     float* tailp = reinterpret_cast<float*>(ws + pl.b_tail);
     if (cudaMemsetAsync(ctr, 0, pl.ctr_bytes, st) != cudaSuccess) return LORA_MLP_ERR_CUDA;
-    if (pl.int4) {
+    if (pl.qf) {
         const void* src = w->S;
         void* dst = ws + pl.b_st;
-        LMLP_TRY(launch_scale_t(1, &src, &dst, &pl.dout, &pl.din, st));
+        LMLP_TRY(launch_scale_t(pl.qf, 1, &src, &dst, &pl.dout, &pl.din, st));
     }
     {  // L2: T = s dY B -> T [N, r], T^T [r, ldN];  dB = dY^T R (R from saved, already s-scaled)
         const int* sp = pl.splits[LK_TDB];
@@ -1443,19 +1493,17 @@ int lora_linear_backward(const lora_linear_shape* shape, const lora_linear_weigh
         PairBuilder b(N, din, 256);
         const int ady = b.a_k(dY, N, dout, dout);
         const int at = b.a_k(T, N, r, r);
-        const int bw = pl.int4 ? b.q_map(w->W, dout, din, true) : b.b_mn(w->W, dout, din, din);
+        const int bw = pl.qf ? b.q_map(w->W, dout, din, true, pl.qf) : b.b_mn(w->W, dout, din, din);
         const int ba = b.b_mn(w->A, r, din, din);
         b.seg(ady, bw, bw, 0, kPairHalfN, 0, 0, dout);
         b.seg(at, ba, ba, 0, kPairHalfN, 0, 0, r);
         b.a.prob.out0 = dX;
         b.a.prob.ld = din;
-        if (pl.int4) {
-            const int sm = b.s_map(ws + pl.b_st, dout, din, true);
+        if (pl.qf) {
+            const int sm = b.s_map(ws + pl.b_st, dout, din, true, pl.qf);
             b.quant(0, bw, bw, sm, sm);
-            LMLP_TRY((launch_pair<true, EPI_BF16, true>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
-        } else {
-            LMLP_TRY((launch_pair<true, EPI_BF16>(b, di.sms, st, "L3_linear_dX", tailp, ctr)));
         }
+        LMLP_TRY((launch_pair_q<true, EPI_BF16>(b, pl.qf, di.sms, st, "L3_linear_dX", tailp, ctr)));
     }
     {  // L4: dA^T = X^T T  (written transposed: dA [r, d_in])
         GemmBuilder b(pl.bn_r);

@@ -88,12 +88,28 @@ constexpr int kQ4Groups = 2;
 constexpr int kQ4RegsCtl = 80, kQ4RegsEpi = 232, kQ4RegsDq = 88;
 static_assert(128 * (kQ4RegsCtl + kQ4RegsEpi) + 256 * kQ4RegsDq <= 512 * 128,
               "the warpgroups' register counts must fit the 128 a thread of a 512-thread block launches with");
-constexpr uint32_t kQ4CodeBytes = kPairHalfN * kBK / 2;  // 4 KB of codes per CTA and stage
-constexpr uint32_t kQ4ScaleBytes = kPairHalfN * 2;        // 128 fp16 scales
-constexpr uint32_t kQ4RawBytes = 5 * 1024;                // codes, scales, padding: stages stay 1 KB aligned
-template <bool Q4>
+// Frozen-weight formats of the B operand: bf16 (TMA straight into the
+// stage), block-int4 or block-FP8 (codes and scales into a raw slot of the
+// stage, expanded by the dequant warps).
+enum : int { QF_NONE = 0, QF_INT4 = 1, QF_FP8 = 2 };
+// Per CTA and stage: codes of the 128 x 64 B half (4 KB of nibbles, 8 KB of
+// E4M3 bytes), its 128 scales (fp16 or fp32), and the raw slot they share,
+// rounded so that stages stay 1 KB aligned.
+template <int QF>
+__host__ __device__ constexpr uint32_t q_code_bytes() {
+    return QF == QF_FP8 ? kPairHalfN * kBK : kPairHalfN * kBK / 2;
+}
+template <int QF>
+__host__ __device__ constexpr uint32_t q_scale_bytes() {
+    return QF == QF_FP8 ? kPairHalfN * 4 : kPairHalfN * 2;
+}
+template <int QF>
+__host__ __device__ constexpr uint32_t q_raw_bytes() {
+    return QF == QF_NONE ? 0u : (q_code_bytes<QF>() + q_scale_bytes<QF>() + 1023u) & ~1023u;
+}
+template <int QF>
 __host__ __device__ constexpr uint32_t pair_stage_bytes() {
-    return kPairStageBytes + (Q4 ? kQ4RawBytes : 0u);
+    return kPairStageBytes + q_raw_bytes<QF>();
 }
 template <int EPI, bool Q4 = false>
 __host__ __device__ constexpr int pair_threads() {
@@ -250,10 +266,12 @@ __device__ __forceinline__ PairUnit pair_decode(const PairArgs& a, int u) {
 // Returns the number of stages it filled.  Both CTAs' loads of a stage
 // count on the leader's full barrier, so the leader's count is what
 // drain_loads needs.
-template <bool B_MN, bool Q4>
+template <bool B_MN, int QF>
 __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t base, uint32_t rank, bool leader,
                                                    const SmemCtl& c) {
-    constexpr uint32_t kSB = pair_stage_bytes<Q4>();
+    constexpr bool Q4 = QF != QF_NONE;
+    constexpr uint32_t kSB = pair_stage_bytes<QF>();
+    constexpr uint32_t kCode = q_code_bytes<QF>(), kScale = q_scale_bytes<QF>();
     const PairProb& P = a.prob;
     long long issued = 0;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
@@ -290,15 +308,17 @@ __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t b
                 const uint32_t raw = sA + kPairStageBytes;
                 const CUtensorMap* qm = &a.maps[S.qmap[rank]];
                 const CUtensorMap* sm = &a.maps[S.smap[rank]];
-                mbar_arrive_expect_tx(rf, kQ4CodeBytes + kQ4ScaleBytes);
+                // x of a code box in bytes: half an element per nibble, one per E4M3 byte
+                constexpr int kSh = QF == QF_FP8 ? 0 : 1;
+                mbar_arrive_expect_tx(rf, kCode + kScale);
                 if (B_MN) {
-                    tma_load_2d(raw, qm, rf, brow >> 1, bk);
-                    tma_load_2d(raw + kQ4CodeBytes / 2, qm, rf, (brow + 64) >> 1, bk);
-                    tma_load_2d(raw + kQ4CodeBytes, sm, rf, bk, brow >> 6);
-                    tma_load_2d(raw + kQ4CodeBytes + kQ4ScaleBytes / 2, sm, rf, bk, (brow >> 6) + 1);
+                    tma_load_2d(raw, qm, rf, brow >> kSh, bk);
+                    tma_load_2d(raw + kCode / 2, qm, rf, (brow + 64) >> kSh, bk);
+                    tma_load_2d(raw + kCode, sm, rf, bk, brow >> 6);
+                    tma_load_2d(raw + kCode + kScale / 2, sm, rf, bk, (brow >> 6) + 1);
                 } else {
-                    tma_load_2d(raw, qm, rf, bk >> 1, brow);
-                    tma_load_2d(raw + kQ4CodeBytes, sm, rf, brow, bk >> 6);
+                    tma_load_2d(raw, qm, rf, bk >> kSh, brow);
+                    tma_load_2d(raw + kCode, sm, rf, brow, bk >> 6);
                 }
             } else {
                 const CUtensorMap* bm = &a.maps[S.b_map[rank]];
@@ -328,8 +348,9 @@ __device__ __forceinline__ long long pair_producer(const PairArgs& a, uint32_t b
 // partial) and forms each stage's descriptors by adding offsets to those of
 // stage 0 instead of re-encoding them.  Measured on the Llama-3-8B MLP
 // shapes: 725-811 -> 574-681 SM cycles per K block.
-template <bool B_MN, bool Q4>
+template <bool B_MN, int QF>
 __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint32_t tmem_base, const SmemCtl& c) {
+    constexpr bool Q4 = QF != QF_NONE;
     const PairProb& P = a.prob;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
     const uint32_t idesc = idesc_bf16(256u, false, B_MN, 256u);
@@ -338,7 +359,7 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
     const uint64_t a0 = sw128_desc(base, 16u, 1024u);
     const uint64_t b0 = B_MN ? sw128_desc(base + kATileBytes, 8192u, 1024u)
                              : sw128_desc(base + kATileBytes, 16u, 1024u);
-    constexpr uint32_t kStageStep = pair_stage_bytes<Q4>() >> 4;
+    constexpr uint32_t kStageStep = pair_stage_bytes<QF>() >> 4;
     constexpr uint32_t kAStep = 32u >> 4;                        // next 16-wide K slice of A
     constexpr uint32_t kBStep = B_MN ? (2048u >> 4) : (32u >> 4);  // ... of B
     int stage = 0;
@@ -406,18 +427,20 @@ __device__ __forceinline__ void pair_mma(const PairArgs& a, uint32_t base, uint3
 // parity instead lets, with an odd count, one warpgroup run two phases ahead
 // of the other on a stage, and the barrier's phase parity aliases: seen as a
 // few stale lines per launch on the Llama-3-8B int4 shapes.)
-template <bool B_MN>
+template <bool B_MN, int QF>
 __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, const SmemCtl& c, int group, int t) {
     const PairProb& P = a.prob;
     const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
     const int lane = threadIdx.x & 31;
-    constexpr uint32_t kSB = pair_stage_bytes<true>();
+    constexpr uint32_t kSB = pair_stage_bytes<QF>();
+    constexpr uint32_t kCode = q_code_bytes<QF>();
+    constexpr uint32_t kLineBytes = QF == QF_FP8 ? 64u : 32u;  // code bytes of one 64-element line
     const int lrow = B_MN ? (t & 63) : t;  // tile row: N row (K-major) or K row (MN-major)
     const int lj = B_MN ? (t >> 6) : 0;    // 64-column chunk (MN-major)
-    const uint32_t raw_off = kPairStageBytes + static_cast<uint32_t>(lj) * (kQ4CodeBytes / 2) +
-                             static_cast<uint32_t>(lrow) * 32u;
+    const uint32_t raw_off = kPairStageBytes + static_cast<uint32_t>(lj) * (kCode / 2) +
+                             static_cast<uint32_t>(lrow) * kLineBytes;
     // the scales: one 128-entry run (K-major), or one 64-entry run per chunk
-    const uint32_t sc_off = kPairStageBytes + kQ4CodeBytes + static_cast<uint32_t>(t) * 2u;
+    const uint32_t sc_off = kPairStageBytes + kCode + static_cast<uint32_t>(t) * (QF == QF_FP8 ? 4u : 2u);
     const uint32_t out_off = kATileBytes + static_cast<uint32_t>(lj) * 8192u + static_cast<uint32_t>(lrow) * 128u;
     const uint32_t swz = static_cast<uint32_t>(lrow & 7);
     // read order of the two 16-byte halves: alternating every four rows puts
@@ -437,11 +460,22 @@ __device__ __forceinline__ void pair_dequant(const PairArgs& a, uint32_t base, c
                 if (!wait_or_abort(c.rawf + 8u * stage, phase, c)) return;
                 if (P.seg[seg].q4) {
                     const uint32_t sb = base + static_cast<uint32_t>(stage) * kSB;
-                    const uint4 x0 = lds128(sb + raw_off + h0);
-                    const uint4 x1 = lds128(sb + raw_off + (h0 ^ 16u));
-                    const float sc = __half2float(__ushort_as_half(lds16(sb + sc_off)));
                     uint4 o[8];
-                    int4_line(h0 ? x1 : x0, h0 ? x0 : x1, sc, o);
+                    if constexpr (QF == QF_FP8) {
+                        // 64-byte code rows land in TMA's 64-byte swizzle: 16-byte
+                        // piece q of row R at piece q ^ ((R / 2) mod 4), so the
+                        // eight rows of a quarter-warp hit distinct bank groups
+                        const uint32_t sw = static_cast<uint32_t>((lrow >> 1) & 3);
+                        uint4 x[4];
+#pragma unroll
+                        for (uint32_t q = 0; q < 4; ++q) x[q] = lds128(sb + raw_off + ((q ^ sw) << 4));
+                        fp8_line(x, __uint_as_float(lds32(sb + sc_off)), o);
+                    } else {
+                        const uint4 x0 = lds128(sb + raw_off + h0);
+                        const uint4 x1 = lds128(sb + raw_off + (h0 ^ 16u));
+                        const float sc = __half2float(__ushort_as_half(lds16(sb + sc_off)));
+                        int4_line(h0 ? x1 : x0, h0 ? x0 : x1, sc, o);
+                    }
 #pragma unroll
                     for (uint32_t w = 0; w < 8; ++w) sts128(sb + out_off + ((w ^ swz) << 4), o[w]);
                     fence_proxy_async_smem();
@@ -714,13 +748,14 @@ __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-template <bool B_MN, int EPI, bool Q4 = false>
-__global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
+template <bool B_MN, int EPI, int QF = QF_NONE>
+__global__ void __launch_bounds__(pair_threads<EPI, QF != QF_NONE>(), 1)
     umma2_gemm_kernel(const __grid_constant__ PairArgs args) {
+    constexpr bool Q4 = QF != QF_NONE;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t ctl = base + args.stages * pair_stage_bytes<Q4>();
+    const uint32_t ctl = base + args.stages * pair_stage_bytes<QF>();
     uint8_t* ctl_ptr = smem_raw + (ctl - raw);
 
     const SmemCtl c = make_ctl(ctl, ctl_ptr, args.wait_limit);
@@ -772,7 +807,7 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
             // The leader waits for both CTAs' loads (they count on its full
             // barriers); the other CTA cannot leave before it, since the
             // cluster barrier below holds it until the leader arrives.
-            const long long issued = pair_producer<B_MN, Q4>(args, base, rank, leader, c);
+            const long long issued = pair_producer<B_MN, QF>(args, base, rank, leader, c);
             if (leader) drain_loads(c.full, args.stages, issued, c.wait_limit);
             if (Q4) drain_loads(c.rawf, args.stages, issued, c.wait_limit);  // this CTA's code loads
         }
@@ -780,7 +815,7 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
     };
     auto mma_role = [&]() {
         if (lane == 0 && leader) {
-            pair_mma<B_MN, Q4>(args, base, tmem_base, c);
+            pair_mma<B_MN, QF>(args, base, tmem_base, c);
             umma_commit_pair(c.drain, 1);
             const long long t0 = clock64();
             while (!mbar_try_wait(c.drain, 0)) {
@@ -803,7 +838,7 @@ __global__ void __launch_bounds__(pair_threads<EPI, Q4>(), 1)
         } else {
             regs_dec<kQ4RegsDq>();
             const int dq = static_cast<int>(threadIdx.x) - 8 * 32;  // 0 .. 255
-            pair_dequant<B_MN>(args, base, c, dq >> 7, dq & 127);
+            pair_dequant<B_MN, QF>(args, base, c, dq >> 7, dq & 127);
         }
     } else {
         if (warp == 0) producer_role();

@@ -77,7 +77,8 @@ def test_sampled_rows_and_features(cfg):
     assert not bad, f"{cfg.name}: {bad} (all {errs})"
 
 
-@pytest.mark.parametrize("cfg", [synth.BY_NAME["llama3_8b_mlp"], synth.BY_NAME["llama3_8b_mlp_int4"]],
+@pytest.mark.parametrize("cfg", [synth.BY_NAME["llama3_8b_mlp"], synth.BY_NAME["llama3_8b_mlp_int4"],
+                                 synth.BY_NAME["llama3_8b_mlp_fp8"]],
                          ids=lambda c: c.name)
 def test_every_output_against_full_oracle(cfg):
     inp, got = gpu_run(cfg)
@@ -119,20 +120,26 @@ def test_every_adapter_gradient_against_token_block_sums(cfg):
     assert not bad, f"{cfg.name}: {bad} (all {errs})"
 
 
-def test_int4_full_size_is_bitwise_the_bf16_path_every_run():
-    """The int4 kernels dequantise in-kernel through rings of shared-memory
-    slots shared by several warp roles; a wrong hand-off shows as a few stale
-    lines in a stage, differing from run to run.  At full size (where the
-    rings wrap thousands of times), five forward + backward passes must each
-    give exactly the bits of the bf16 path on the dequantised weights."""
-    cfg = synth.BY_NAME["llama3_8b_mlp_int4"]
+@pytest.mark.parametrize("name", ["llama3_8b_mlp_int4", "llama3_8b_mlp_fp8"])
+def test_quantised_full_size_is_bitwise_the_bf16_path_every_run(name):
+    """The int4 and FP8 kernels dequantise in-kernel through rings of
+    shared-memory slots shared by several warp roles; a wrong hand-off shows
+    as a few stale lines in a stage, differing from run to run.  At full size
+    (where the rings wrap thousands of times), five forward + backward passes
+    must each give exactly the bits of the bf16 path on the dequantised
+    weights."""
+    cfg = synth.BY_NAME[name]
     _cache.clear()
     torch.cuda.empty_cache()
     inp = synth.make_inputs(cfg)
     deq = dict(inp)
     for k in ("Wg", "Wu", "Wd"):
-        deq[k] = oracle.dequant_int4(inp[k + "_q"], inp[k + "_scale"])
-        del deq[k + "_q"], deq[k + "_scale"]
+        if k + "_q" in inp:
+            deq[k] = oracle.dequant_int4(inp[k + "_q"], inp[k + "_scale"])
+            del deq[k + "_q"], deq[k + "_scale"]
+        else:
+            deq[k] = oracle.dequant_fp8(inp[k + "_f8"], inp[k + "_f8scale"])
+            del deq[k + "_f8"], deq[k + "_f8scale"]
     dev = torch.device("cuda:0")
     w4 = api.weights_from_host(inp, cfg.alpha, dev)
     w16 = api.weights_from_host(deq, cfg.alpha, dev)

@@ -26,9 +26,9 @@ def cuda_ready():
     torch.cuda.set_device(0)
 
 
-def cfg_of(N, d_in, d_out, r, alpha, idx, int4=False):
+def cfg_of(N, d_in, d_out, r, alpha, idx, int4=False, fp8=False):
     return synth.LinearConfig(f"lin_{N}_{d_in}_{d_out}_{r}", N, d_in, d_out, r, float(alpha), int4=int4,
-                              index=idx)
+                              index=idx, fp8=fp8)
 
 
 def run_gpu(inp, alpha, w=None, X_override=None):
@@ -140,3 +140,18 @@ def test_linear_full_size_every_output(name):
     got = run_gpu(inp, cfg.alpha)
     torch.cuda.empty_cache()
     assert_parity(got, olin.forward_backward(inp, cfg.alpha))
+
+
+@pytest.mark.parametrize("N,d_in,d_out", [(640, 512, 384), (300, 192, 328)])   # the second: d_out % 64 != 0
+def test_linear_fp8_matches_dequantised_bf16_bitwise_and_oracle(N, d_in, d_out):
+    cfg = cfg_of(N, d_in, d_out, 16, 16.0, 68, fp8=True)
+    inp = synth.make_linear_inputs(cfg)
+    dev = torch.device("cuda:0")
+    w8 = api.linear_weights_from_host(inp, cfg.alpha, dev)
+    Wbf = api.dequant_fp8(w8.W, w8.S)
+    wbf = api.LinearWeights(W=Wbf, A=w8.A, B=w8.B, alpha=cfg.alpha)
+    g8 = run_gpu(inp, cfg.alpha, w=w8)
+    gbf = run_gpu(inp, cfg.alpha, w=wbf)
+    for k in KEYS:
+        assert np.array_equal(g8[k], gbf[k]), k
+    assert_parity(g8, olin.forward_backward(inp, cfg.alpha))

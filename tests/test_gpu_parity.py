@@ -1,8 +1,8 @@
 """GPU parity: the sm_100a path through the C ABI against the fp64 CPU oracle.
 
 Tolerance: per tensor, max|gpu - oracle| / max|oracle| <= 2e-2 for the bf16
-outputs and gradients (fp32 accumulation).  Integer work (the int4
-dequantisation) is compared bit for bit."""
+outputs and gradients (fp32 accumulation).  The dequantisation of int4 and
+FP8 frozen weights is compared bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -157,6 +157,67 @@ def test_int4_path_matches_dequantised_bf16_path_bitwise_and_oracle():
     for k in got4:
         assert np.array_equal(got4[k], got16[k]), k
     assert_parity(got4, oracle.forward_backward(inp, cfg.alpha))
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3, fp32 scale per 64)
+
+
+def same_bits_or_both_nan(got_bits, ref_bits):
+    """bf16 bits equal, except that a NaN may carry any payload and sign."""
+    f = lambda b: (np.asarray(b).astype(np.uint32) << 16).view(np.float32)  # noqa: E731
+    g, r = f(got_bits), f(ref_bits)
+    nan = np.isnan(r)
+    return np.array_equal(nan, np.isnan(g)) and np.array_equal(np.asarray(got_bits)[~nan], np.asarray(ref_bits)[~nan])
+
+
+def test_fp8_dequant_bits_every_code_for_many_scales():
+    """All 256 codes against fp32 scales of every kind: random over 82 decades,
+    negative, +-0, subnormal, the largest finite, infinite and NaN."""
+    rng = np.random.default_rng(37)
+    sc = list(rng.uniform(-3, 3, 100).astype(np.float32)) + list((10.0 ** rng.uniform(-44, 38, 100)).astype(np.float32))
+    sc += [0.0, -0.0, 1e-45, -1e-45, 1e-40, 2.0 ** -126, 3.4e38, -3.4e38, np.inf, -np.inf, np.nan, 1.0 / 448]
+    sc = np.array(sc, dtype=np.float32)
+    rows = len(sc)
+    codes = np.tile(np.arange(256, dtype=np.uint8), (rows, 1))
+    scales = np.repeat(sc[:, None], 4, axis=1)
+    dev = torch.device("cuda:0")
+    got = api.dequant_fp8(torch.from_numpy(codes).to(dev), torch.from_numpy(scales).to(dev))
+    torch.cuda.synchronize()
+    got_bits = got.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert same_bits_or_both_nan(got_bits, oracle.dequant_fp8(codes, scales))
+
+
+def test_fp8_quantised_weight_dequantises_like_the_oracle():
+    rng = np.random.default_rng(38)
+    w = (rng.standard_normal((96, 448)) * 0.05).astype(np.float32)
+    w[5, 128:192] = 0.0
+    codes, scales = synth.quantize_fp8(w)
+    dev = torch.device("cuda:0")
+    got = api.dequant_fp8(torch.from_numpy(codes).view(torch.float8_e4m3fn).to(dev), torch.from_numpy(scales).to(dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), oracle.dequant_fp8(codes, scales))
+
+
+def dequantised_bf16_inputs(inp):
+    deq = dict(inp)
+    for k in ("Wg", "Wu", "Wd"):
+        if k + "_f8" in inp:
+            deq[k] = oracle.dequant_fp8(inp[k + "_f8"], inp[k + "_f8scale"])
+            del deq[k + "_f8"], deq[k + "_f8scale"]
+    return deq
+
+
+@pytest.mark.parametrize("cfg", [synth.custom(384, 256, 512, 16, 16.0, seed_index=34, fp8=True),
+                                 synth.custom(300, 192, 704, 24, 8.0, seed_index=35, fp8=True),   # ragged
+                                 synth.custom(1000, 512, 1408, 64, 128.0, seed_index=36, fp8=True)],
+                         ids=lambda c: f"N{c.N}_d{c.d}_dff{c.d_ff}_r{c.r}")
+def test_fp8_path_matches_dequantised_bf16_path_bitwise_and_oracle(cfg):
+    inp = synth.make_inputs(cfg)
+    got8 = run_gpu(inp, cfg.alpha)
+    got16 = run_gpu(dequantised_bf16_inputs(inp), cfg.alpha)
+    for k in got8:
+        assert np.array_equal(got8[k], got16[k]), k
+    assert_parity(got8, oracle.forward_backward(inp, cfg.alpha))
 
 
 # ----------------------------------------------------------------------------- autograd wrapper
