@@ -65,6 +65,43 @@ int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights*
                             const void* dOut, void* dX, const lora_mlp_grads* grads, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * The block with the norm fused into the gate/up GEMM (bf16 frozen weights).
+ *
+ * With x_hat = diag(rstd) X diag(gamma), the gate and up projections are
+ * x_hat W^T = diag(rstd) X (W diag(gamma))^T: once gamma is folded into Wg and
+ * Wu (lora_mlp_block_fold_gamma, done once, since W and gamma are frozen), the
+ * gate/up GEMM reads the raw rows X and its epilogue scales each row by rstd,
+ * so the normalised rows are never written.  The rank-r path takes
+ * A diag(gamma) (formed each call, A being trainable) the same way.  The
+ * backward's dX GEMM on the folded weights yields dx_hat * gamma, which the
+ * norm's backward maps to dX; the adapter gradients take the rstd and gamma
+ * factors in their split-K finalisation.  Results match the unfused block up
+ * to the rounding of the folded weights and the order of the products.
+ * Workspace and saved sizes: lora_mlp_block_sizes.
+ */
+
+/* Wg_folded = bf16_rne(Wg * gamma) and Wu_folded = bf16_rne(Wu * gamma), each
+ * column e of Wg, Wu [d_ff, d] times gamma[e].  bf16 weights only
+ * (LORA_MLP_ERR_INVALID_ARG otherwise).  One launch. */
+int lora_mlp_block_fold_gamma(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* gamma,
+                              void* Wg_folded, void* Wu_folded, void* stream);
+
+/* Block forward with the folded weights: w_folded is w with Wg, Wu replaced
+ * by the outputs of lora_mlp_block_fold_gamma (Wd and the adapters
+ * unchanged); gamma, eps, X and the outputs as in lora_mlp_block_forward.
+ * Launches: rstd only, A diag(gamma) for both adapters, then the MLP's. */
+int lora_mlp_block_forward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded,
+                                  const void* gamma, float eps, const void* X, void* out, void* g, void* u,
+                                  void* saved, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block backward with the folded weights; arguments as in
+ * lora_mlp_block_backward, `saved` from lora_mlp_block_forward_folded. */
+int lora_mlp_block_backward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded,
+                                   const void* gamma, const void* X, const void* g, const void* u,
+                                   const void* saved, const void* dOut, void* dX, const lora_mlp_grads* grads,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -55,6 +55,9 @@ SYMBOLS = (
     "lora_mlp_block_sizes",
     "lora_mlp_block_forward",
     "lora_mlp_block_backward",
+    "lora_mlp_block_fold_gamma",
+    "lora_mlp_block_forward_folded",
+    "lora_mlp_block_backward_folded",
     "lora_ce_sizes",
     "lora_ce_forward",
     "lora_ce_backward",
@@ -149,6 +152,9 @@ def lib() -> ctypes.CDLL:
                                                  vp, vp, vp, vp, vp, vp, sz, vp]
             L.lora_mlp_block_backward.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp,
                                                   vp, vp, vp, ctypes.POINTER(Grads), vp, sz, vp]
+            L.lora_mlp_block_fold_gamma.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), vp, vp, vp, vp]
+            L.lora_mlp_block_forward_folded.argtypes = L.lora_mlp_block_forward.argtypes
+            L.lora_mlp_block_backward_folded.argtypes = L.lora_mlp_block_backward.argtypes
             L.lora_ce_sizes.argtypes = [ctypes.POINTER(CEShape), ctypes.POINTER(sz)]
             L.lora_ce_forward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, sz, vp]
             L.lora_ce_backward.argtypes = [ctypes.POINTER(CEShape), vp, vp, vp, vp, vp, vp]
@@ -167,7 +173,9 @@ def lib() -> ctypes.CDLL:
                          "lora_rmsnorm_forward", "lora_rmsnorm_backward", "lora_mlp_block_sizes",
                          "lora_mlp_block_forward", "lora_mlp_block_backward", "lora_ce_sizes",
                          "lora_ce_forward", "lora_ce_backward", "lora_ce_device_status",
-                         "lora_ce_forward_reduced", "lora_ce_backward_reduced", "lora_mlp_workspace_size"):
+                         "lora_ce_forward_reduced", "lora_ce_backward_reduced", "lora_mlp_workspace_size",
+                         "lora_mlp_block_fold_gamma", "lora_mlp_block_forward_folded",
+                         "lora_mlp_block_backward_folded"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -298,6 +306,23 @@ def block_backward(shape: Shape, weights: Weights, gamma, X, g, u, saved, dOut, 
                    workspace_bytes, stream) -> int:
     return lib().lora_mlp_block_backward(ctypes.byref(shape), ctypes.byref(weights), gamma, X, g, u, saved, dOut,
                                          dX, ctypes.byref(grads), workspace, workspace_bytes, stream)
+
+
+def block_fold_gamma(shape: Shape, weights: Weights, gamma, Wg_folded, Wu_folded, stream) -> int:
+    return lib().lora_mlp_block_fold_gamma(ctypes.byref(shape), ctypes.byref(weights), gamma, Wg_folded, Wu_folded,
+                                           stream)
+
+
+def block_forward_folded(shape: Shape, weights: Weights, gamma, eps, X, out, g, u, saved, workspace,
+                         workspace_bytes, stream) -> int:
+    return lib().lora_mlp_block_forward_folded(ctypes.byref(shape), ctypes.byref(weights), gamma, float(eps), X, out,
+                                               g, u, saved, workspace, workspace_bytes, stream)
+
+
+def block_backward_folded(shape: Shape, weights: Weights, gamma, X, g, u, saved, dOut, dX, grads: Grads, workspace,
+                          workspace_bytes, stream) -> int:
+    return lib().lora_mlp_block_backward_folded(ctypes.byref(shape), ctypes.byref(weights), gamma, X, g, u, saved,
+                                                dOut, dX, ctypes.byref(grads), workspace, workspace_bytes, stream)
 
 
 def rmsnorm_forward(N, d, eps, x, gamma, y, rstd, stream) -> int:

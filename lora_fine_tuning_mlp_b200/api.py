@@ -532,10 +532,26 @@ class RMSNormFunction(torch.autograd.Function):
         return rmsnorm_backward(x, gamma, rstd, dy.contiguous()), None, None
 
 
+def fold_gamma(w: MLPWeights, gamma: torch.Tensor, stream=None) -> MLPWeights:
+    """The weights of the fused-norm block: Wg, Wu with gamma folded into
+    their columns (bf16_rne(W * gamma), by the library's kernel); Wd and the
+    adapters are the same tensors as w's.  bf16 frozen weights only.  Done
+    once: W and gamma are frozen."""
+    if w.int4 or w.fp8:
+        raise ValueError("gamma folds into bf16 frozen weights only")
+    w.validate()
+    _need(gamma, "gamma", BF16, (w.d,))
+    Wg, Wu = torch.empty_like(w.Wg), torch.empty_like(w.Wu)
+    _lib.check(_lib.block_fold_gamma(w.shape(1), w.c_struct(), _p(gamma), _p(Wg), _p(Wu), _stream(stream)),
+               "lora_mlp_block_fold_gamma")
+    return MLPWeights(Wg=Wg, Wu=Wu, Wd=w.Wd, Ag=w.Ag, Bg=w.Bg, Au=w.Au, Bu=w.Bu, Ad=w.Ad, Bd=w.Bd, alpha=w.alpha)
+
+
 def block_forward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, eps: float, *, out=None,
-                  workspace: Workspace | None = None, stream=None):
+                  workspace: Workspace | None = None, stream=None, folded: bool = False):
     """out = MLP(RMSNorm(X) * gamma).  Returns (out, Saved); Saved.lowrank
-    also holds the per-row rstd."""
+    also holds the per-row rstd.  folded=True: w comes from fold_gamma and
+    the norm runs fused into the gate/up GEMM (lora_mlp_block_forward_folded)."""
     N, d = X.shape
     _need(X, "X", BF16, (N, w.d))
     _need(gamma, "gamma", BF16, (w.d,))
@@ -548,14 +564,16 @@ def block_forward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, eps: floa
     u = torch.empty((N, w.d_ff), dtype=BF16, device=dev)
     saved = torch.empty(max(svs, 256), dtype=torch.uint8, device=dev)
     ws = (workspace or Workspace()).get(fws, dev)
-    _lib.check(_lib.block_forward(shape, w.c_struct(), _p(gamma), eps, _p(X), _p(out), _p(g), _p(u), _p(saved),
-                                  _p(ws), ws.numel(), _stream(stream)), "lora_mlp_block_forward")
+    fn = _lib.block_forward_folded if folded else _lib.block_forward
+    _lib.check(fn(shape, w.c_struct(), _p(gamma), eps, _p(X), _p(out), _p(g), _p(u), _p(saved), _p(ws), ws.numel(),
+                  _stream(stream)), "lora_mlp_block_forward" + ("_folded" if folded else ""))
     return out, Saved(g, u, saved)
 
 
 def block_backward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, saved: Saved, dOut: torch.Tensor, *,
-                   dX=None, grads=None, workspace: Workspace | None = None, stream=None):
-    """Returns (dX, {dAg, dBg, dAu, dBu, dAd, dBd}) for the block input X."""
+                   dX=None, grads=None, workspace: Workspace | None = None, stream=None, folded: bool = False):
+    """Returns (dX, {dAg, dBg, dAu, dBu, dAd, dBd}) for the block input X.
+    folded as in block_forward (and the same as the forward's)."""
     N, d = X.shape
     _need(X, "X", BF16, (N, w.d))
     _need(gamma, "gamma", BF16, (w.d,))
@@ -569,9 +587,10 @@ def block_backward(X: torch.Tensor, w: MLPWeights, gamma: torch.Tensor, saved: S
         grads = {("d" + k): torch.empty_like(getattr(w, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
     gs = _lib.Grads(*[grads[k].data_ptr() for k in _lib.GRAD_FIELDS])
     ws = (workspace or Workspace()).get(bws, dev)
-    _lib.check(_lib.block_backward(shape, w.c_struct(), _p(gamma), _p(X), _p(saved.g), _p(saved.u),
-                                   _p(saved.lowrank), _p(dOut), _p(dX), gs, _p(ws), ws.numel(), _stream(stream)),
-               "lora_mlp_block_backward")
+    fn = _lib.block_backward_folded if folded else _lib.block_backward
+    _lib.check(fn(shape, w.c_struct(), _p(gamma), _p(X), _p(saved.g), _p(saved.u), _p(saved.lowrank), _p(dOut),
+                  _p(dX), gs, _p(ws), ws.numel(), _stream(stream)),
+               "lora_mlp_block_backward" + ("_folded" if folded else ""))
     return dX, grads
 
 

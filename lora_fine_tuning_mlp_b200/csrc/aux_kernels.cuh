@@ -195,8 +195,9 @@ __global__ void __launch_bounds__(kDqThreads) dequant_fp8_kernel(const uint4* __
 // Block scales [rows, nb] (nb = cols / 64) -> their transpose [nb, rows], so
 // that the scales of one 64-column block of consecutive rows are contiguous
 // and a GEMM stage can fetch them with one TMA box.  Up to three matrices per
-// launch (blockIdx.z), 32 x 32 tiles through shared memory.
-// T: unsigned short (int4's fp16 scales) or unsigned int (FP8's fp32 scales).
+// launch (blockIdx.y); a CTA takes a strip of 32 rows and walks its 32 x 32
+// tiles through shared memory (reads along a row, writes along a column of
+// the transpose, both coalesced).
 template <class T>
 struct ScaleT {
     const T* src[3];
@@ -207,19 +208,22 @@ struct ScaleT {
 template <class T>
 __global__ void __launch_bounds__(256) scale_transpose_kernel(const ScaleT<T> a) {
     __shared__ T tile[32][33];
-    const int z = blockIdx.z;
+    const int z = blockIdx.y;
     const int rows = a.rows[z], nb = a.nb[z];
-    const int r0 = blockIdx.x * 32, b0 = blockIdx.y * 32;
-    if (r0 >= rows || b0 >= nb) return;
+    const int r0 = blockIdx.x * 32;
+    if (r0 >= rows) return;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
-    for (int i = ty; i < 32; i += 8) {
-        const int r = r0 + i, b = b0 + tx;
-        if (r < rows && b < nb) tile[i][tx] = a.src[z][static_cast<long long>(r) * nb + b];
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int b = b0 + i, r = r0 + tx;
-        if (r < rows && b < nb) a.dst[z][static_cast<long long>(b) * rows + r] = tile[tx][i];
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+        for (int i = ty; i < 32; i += 8) {
+            const int r = r0 + i, b = b0 + tx;
+            if (r < rows && b < nb) tile[i][tx] = a.src[z][static_cast<long long>(r) * nb + b];
+        }
+        __syncthreads();
+        for (int i = ty; i < 32; i += 8) {
+            const int b = b0 + i, r = r0 + tx;
+            if (r < rows && b < nb) a.dst[z][static_cast<long long>(b) * rows + r] = tile[tx][i];
+        }
+        __syncthreads();
     }
 }
 

@@ -34,6 +34,10 @@ struct EpiOut {
     long long ld;         // row stride (elements) of every out/in
     long long split_off;  // EPI_F32: element offset of this split's partial
     int M, N;             // valid rows / columns
+    // EPI_SWIGLU_FWD: optional factor of each row applied to both
+    // accumulators before they are rounded (the RMSNorm row scale of the
+    // pre-norm block with gamma folded into the gate/up weights)
+    const float* row_scale;
 };
 
 #ifndef LMLP_FAST_SIGMOID
@@ -383,6 +387,14 @@ __device__ __forceinline__ void epilogue_tile(const EpiOut& o, int row, int col_
             } else {  // EPI_SWIGLU_FWD
                 uint32_t vg[32], vu[32];
                 src.load2(ch * 32, vg, acc_stride + ch * 32, vu);
+                if (o.row_scale != nullptr) {
+                    const float rs = row_ok ? o.row_scale[row] : 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        vg[k] = __float_as_uint(__uint_as_float(vg[k]) * rs);
+                        vu[k] = __float_as_uint(__uint_as_float(vu[k]) * rs);
+                    }
+                }
                 uint4 gq[4], uq[4], hq[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {

@@ -613,18 +613,17 @@ template <class T>
 int launch_scale_t_typed(int n, const void* const* src, void* const* dst, const int64_t* rows,
                          const int64_t* cols, cudaStream_t st) {
     ScaleT<T> a{};
-    unsigned gx = 1, gy = 1;
+    unsigned gx = 1;
     for (int i = 0; i < n; ++i) {
         a.src[i] = static_cast<const T*>(src[i]);
         a.dst[i] = static_cast<T*>(dst[i]);
         a.rows[i] = static_cast<int>(rows[i]);
         a.nb[i] = static_cast<int>(cols[i] / 64);
         gx = std::max(gx, static_cast<unsigned>((rows[i] + 31) / 32));
-        gy = std::max(gy, static_cast<unsigned>((cols[i] / 64 + 31) / 32));
     }
     {
         LaunchScope scope("scales_t", st);
-        scale_transpose_kernel<T><<<dim3(gx, gy, n), 256, 0, st>>>(a);
+        scale_transpose_kernel<T><<<dim3(gx, n), 256, 0, st>>>(a);
     }
     return last_launch_error();
 }
@@ -886,6 +885,19 @@ int mlp_scales_t(const Plan& pl, const lora_mlp_weights* w, uint8_t* ws, const s
     return launch_scale_t(pl.qf, 3, src, dst, rows, cols, st);
 }
 
+// The pre-norm block with gamma folded into the gate/up weights runs the
+// MLP on the raw rows X with these hooks (X_hat = diag(rstd) X diag(gamma)):
+// F0 uses A diag(gamma) and writes the saved rank-r copy scaled by rstd; the
+// gate/up epilogue scales its accumulators by rstd; B-mid scales the copy of
+// T that B5 reads by rstd; B4 uses A diag(gamma), so dX comes out as
+// dX_hat * gamma; B5 scales dA by gamma.
+struct Fold {
+    const float* rstd;         // [N]
+    const void* Ag;            // Ag diag(gamma), bf16 [r, d]
+    const void* Au;            // Au diag(gamma)
+    const void* gamma;         // bf16 [d]
+};
+
 }  // namespace
 
 // ============================================================================= C ABI
@@ -906,8 +918,9 @@ int lora_mlp_workspace_size(const lora_mlp_shape* shape, size_t* fwd_bytes, size
     return lora_mlp_sizes(shape, fwd_bytes, bwd_bytes, nullptr);
 }
 
-int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out, void* g,
-                     void* u, void* saved, void* workspace, size_t workspace_bytes, void* stream) {
+static int mlp_forward_impl(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out,
+                            void* g, void* u, void* saved, void* workspace, size_t workspace_bytes, void* stream,
+                            const Fold* fold) {
     LMLP_TRY(validate_shape(shape));
     LMLP_TRY(check_weights(shape, w));
     LMLP_TRY(check_ptrs({X, out, g, u, saved, workspace}));
@@ -932,8 +945,8 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     {  // F0: [S_g | S_u] = s X [Ag; Au]^T  -> Sgu [N, 2r] and saved [S_g^T; S_u^T] [2r, ldN]
         GemmBuilder b(pl.bn_r);
         const int ax = b.a_k(X, N, d, d);
-        const int bg = b.b_k(w->Ag, r, d, d);
-        const int bu = b.b_k(w->Au, r, d, d);
+        const int bg = b.b_k(fold != nullptr ? fold->Ag : w->Ag, r, d, d);
+        const int bu = b.b_k(fold != nullptr ? fold->Au : w->Au, r, d, d);
         Prob* p = b.prob(N, r, pl.splits[SK_F0][0]);
         b.seg(p, ax, bg, bu, d);
         p->out0 = part;
@@ -941,6 +954,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         p->ld = 2 * r;
         p->split_stride = N * 2 * r;
         b.fin(p, pl.s, static_cast<int>(2 * r), Sgu, 2 * r, sv + pl.s_sgT, nullptr, pl.ldN, static_cast<int>(2 * r));
+        if (fold != nullptr) p->tr_row_scale = fold->rstd;
         LMLP_TRY((launch_gemm<2, EPI_F32>(b, di.sms, st, "F0_lowrank_in", ctr)));
     }
     {  // F1: G = X Wg^T + S_g Bg^T, U = X Wu^T + S_u Bu^T; g, u, h  (CTA pairs: half 0 = gate, half 1 = up)
@@ -957,6 +971,7 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
         b.a.prob.out1 = u;
         b.a.prob.out2 = h;
         b.a.prob.ld = dff;
+        if (fold != nullptr) b.a.prob.row_scale = fold->rstd;
         if (pl.qf) {
             const int sg = b.s_map(ws + pl.f_st[0], dff, d, false, pl.qf);
             const int su = b.s_map(ws + pl.f_st[1], dff, d, false, pl.qf);
@@ -995,9 +1010,10 @@ int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, con
     return LORA_MLP_OK;
 }
 
-int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, const void* g,
-                      const void* u, const void* saved, const void* dOut, void* dX, const lora_mlp_grads* grads,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+static int mlp_backward_impl(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, const void* g,
+                             const void* u, const void* saved, const void* dOut, void* dX,
+                             const lora_mlp_grads* grads, void* workspace, size_t workspace_bytes, void* stream,
+                             const Fold* fold) {
     LMLP_TRY(validate_shape(shape));
     LMLP_TRY(check_weights(shape, w));
     if (grads == nullptr) return LORA_MLP_ERR_INVALID_ARG;
@@ -1093,12 +1109,14 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         tg->ld = r;
         tg->split_stride = N * r;
         b.fin(tg, pl.s, static_cast<int>(r), Tgu, 2 * r, TguT, nullptr, ldN, static_cast<int>(r));
+        if (fold != nullptr) tg->tr_row_scale = fold->rstd;
         Prob* tu = b.prob(N, r, sp[1], false, true);
         b.seg(tu, adu_k, bbu, -1, dff);
         tu->out0 = part + po[1];
         tu->ld = r;
         tu->split_stride = N * r;
         b.fin(tu, pl.s, static_cast<int>(r), Tgu + r, 2 * r, TguT + r * ldN, nullptr, ldN, static_cast<int>(r));
+        if (fold != nullptr) tu->tr_row_scale = fold->rstd;
         Prob* pad = b.prob(dff, r, sp[2], true, false);
         b.seg(pad, ah, btd, -1, N);
         pad->out0 = part + po[2];
@@ -1136,8 +1154,8 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         const int atu = b.a_k(Tgu + r, N, r, 2 * r);
         const int bwg = pl.qf ? b.q_map(w->Wg, dff, d, true, pl.qf) : b.b_mn(w->Wg, dff, d, d);
         const int bwu = pl.qf ? b.q_map(w->Wu, dff, d, true, pl.qf) : b.b_mn(w->Wu, dff, d, d);
-        const int bag = b.b_mn(w->Ag, r, d, d);
-        const int bau = b.b_mn(w->Au, r, d, d);
+        const int bag = b.b_mn(fold != nullptr ? fold->Ag : w->Ag, r, d, d);
+        const int bau = b.b_mn(fold != nullptr ? fold->Au : w->Au, r, d, d);
         b.seg(adg, bwg, bwg, 0, kPairHalfN, 0, 0, dff);
         b.seg(adu, bwu, bwu, 0, kPairHalfN, 0, 0, dff);
         b.seg(atg, bag, bag, 0, kPairHalfN, 0, 0, r);
@@ -1162,9 +1180,22 @@ int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, co
         p->ld = 2 * r;
         p->split_stride = d * 2 * r;
         b.fin(p, 1.0f, static_cast<int>(2 * r), nullptr, 0, grads->dAg, grads->dAu, d, static_cast<int>(r));
+        if (fold != nullptr) p->tr_row_scale_bf16 = static_cast<const __nv_bfloat16*>(fold->gamma);
         LMLP_TRY((launch_gemm<1, EPI_F32>(b, di.sms, st, "B5_dA_in", ctr)));
     }
     return LORA_MLP_OK;
+}
+
+int lora_mlp_forward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, void* out, void* g,
+                     void* u, void* saved, void* workspace, size_t workspace_bytes, void* stream) {
+    return mlp_forward_impl(shape, w, X, out, g, u, saved, workspace, workspace_bytes, stream, nullptr);
+}
+
+int lora_mlp_backward(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* X, const void* g,
+                      const void* u, const void* saved, const void* dOut, void* dX, const lora_mlp_grads* grads,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    return mlp_backward_impl(shape, w, X, g, u, saved, dOut, dX, grads, workspace, workspace_bytes, stream,
+                             nullptr);
 }
 
 int lora_mlp_dequant_int4(const void* packed, const void* scales, int64_t rows, int64_t cols, void* w_bf16,
@@ -1594,9 +1625,30 @@ int validate_norm(int64_t N, int64_t d) {
     return LORA_MLP_OK;
 }
 
+// out = bf16_rne(in * gamma) over the columns of up to two bf16 [rows, cols]
+// matrices, one launch.
+int launch_scale_cols(const void* in0, const void* in1, void* out0, void* out1, int64_t rows, int64_t cols,
+                      const void* gamma, int sms, cudaStream_t st) {
+    ScaleCols a{};
+    a.in[0] = static_cast<const __nv_bfloat16*>(in0);
+    a.in[1] = static_cast<const __nv_bfloat16*>(in1);
+    a.out[0] = static_cast<__nv_bfloat16*>(out0);
+    a.out[1] = static_cast<__nv_bfloat16*>(out1);
+    a.rows[0] = a.rows[1] = rows;
+    long long blocks = (rows * (cols / 8) + 255) / 256;
+    if (blocks > static_cast<long long>(sms) * 8) blocks = static_cast<long long>(sms) * 8;
+    if (blocks < 1) blocks = 1;
+    {
+        LaunchScope scope("scale_cols", st);
+        scale_cols_kernel<<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, st>>>(
+            a, static_cast<const __nv_bfloat16*>(gamma), static_cast<int>(cols));
+    }
+    return last_launch_error();
+}
+
 // Workspace / saved layout of the block (offsets in bytes).
 struct BlockPlan {
-    size_t xn, dxn, mlp_f, mlp_b, f_total, b_total;
+    size_t xn, dxn, af, mlp_f, mlp_b, f_total, b_total;  // af: Ag, Au scaled by gamma (folded block)
     size_t s_mlp, s_rstd, s_total;
 };
 
@@ -1604,12 +1656,15 @@ BlockPlan make_block_plan(const lora_mlp_shape& sh) {
     const Plan pl = make_plan(sh);
     BlockPlan b{};
     const size_t xbytes = static_cast<size_t>(sh.N) * static_cast<size_t>(sh.d) * 2;
+    const size_t abytes = 2 * ((static_cast<size_t>(sh.r) * static_cast<size_t>(sh.d) * 2 + kAlign - 1) / kAlign * kAlign);
     Carver f;
     b.xn = f.take(xbytes);
+    b.af = f.take(abytes);
     b.mlp_f = f.take(pl.f_total);
     b.f_total = f.off;
     Carver k;
-    k.take(xbytes);  // xn at offset 0 in both workspaces
+    k.take(xbytes);  // xn and af at the same offsets in both workspaces
+    k.take(abytes);
     b.dxn = k.take(xbytes);
     b.mlp_b = k.take(pl.b_total);
     b.b_total = k.off;
@@ -1699,6 +1754,77 @@ int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights*
     LMLP_TRY(lora_mlp_backward(shape, w, ws + b.xn, g, u, sv + b.s_mlp, dOut, ws + b.dxn, grads, ws + b.mlp_b,
                                b.b_total - b.mlp_b, stream));
     return launch_rmsnorm_bwd(shape->N, shape->d, X, gamma, rstd, ws + b.dxn, dX, di.sms, st);
+}
+
+int lora_mlp_block_fold_gamma(const lora_mlp_shape* shape, const lora_mlp_weights* w, const void* gamma,
+                              void* Wg_folded, void* Wu_folded, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    if (shape->weight_format != LORA_MLP_WEIGHTS_BF16) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_weights(shape, w));
+    LMLP_TRY(check_ptrs({gamma, Wg_folded, Wu_folded}));
+    LMLP_TRY(check_weight_memory(shape, w));
+    LMLP_TRY(check_memory({gamma, Wg_folded, Wu_folded}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    return launch_scale_cols(w->Wg, w->Wu, Wg_folded, Wu_folded, shape->d_ff, shape->d, gamma, di.sms,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int lora_mlp_block_forward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded, const void* gamma,
+                                  float eps, const void* X, void* out, void* g, void* u, void* saved,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    if (shape->weight_format != LORA_MLP_WEIGHTS_BF16) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_weights(shape, w_folded));
+    if (!std::isfinite(eps) || eps < 0.0f) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_ptrs({gamma, X, out, g, u, saved, workspace}));
+    const BlockPlan b = make_block_plan(*shape);
+    if (workspace_bytes < b.f_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w_folded));
+    LMLP_TRY(check_memory({gamma, X, out, g, u, saved, workspace}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* sv = static_cast<uint8_t*>(saved);
+    float* rstd = reinterpret_cast<float*>(sv + b.s_rstd);
+    const size_t ab = (b.mlp_f - b.af) / 2;
+    // rstd only (no normalised rows), then A diag(gamma) for both adapters
+    LMLP_TRY(launch_rmsnorm_fwd(shape->N, shape->d, eps, X, nullptr, nullptr, rstd, nullptr, di.sms, st));
+    LMLP_TRY(launch_scale_cols(w_folded->Ag, w_folded->Au, ws + b.af, ws + b.af + ab, shape->r, shape->d, gamma,
+                               di.sms, st));
+    const Fold f{rstd, ws + b.af, ws + b.af + ab, gamma};
+    return mlp_forward_impl(shape, w_folded, X, out, g, u, sv + b.s_mlp, ws + b.mlp_f, b.f_total - b.mlp_f, stream,
+                            &f);
+}
+
+int lora_mlp_block_backward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded, const void* gamma,
+                                   const void* X, const void* g, const void* u, const void* saved, const void* dOut,
+                                   void* dX, const lora_mlp_grads* grads, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    LMLP_TRY(validate_shape(shape));
+    if (shape->weight_format != LORA_MLP_WEIGHTS_BF16) return LORA_MLP_ERR_INVALID_ARG;
+    LMLP_TRY(check_weights(shape, w_folded));
+    LMLP_TRY(check_ptrs({gamma, X, g, u, saved, dOut, dX, workspace}));
+    const BlockPlan b = make_block_plan(*shape);
+    if (workspace_bytes < b.b_total) return LORA_MLP_ERR_WORKSPACE_TOO_SMALL;
+    LMLP_TRY(check_weight_memory(shape, w_folded));
+    LMLP_TRY(check_memory({gamma, X, g, u, saved, dOut, dX, workspace}));
+    DevInfo di;
+    LMLP_TRY(device_info(&di));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    const float* rstd = reinterpret_cast<const float*>(sv + b.s_rstd);
+    const size_t ab = (b.dxn - b.af) / 2;
+    LMLP_TRY(launch_scale_cols(w_folded->Ag, w_folded->Au, ws + b.af, ws + b.af + ab, shape->r, shape->d, gamma,
+                               di.sms, st));
+    const Fold f{rstd, ws + b.af, ws + b.af + ab, gamma};
+    // the dX GEMM on the folded weights gives dX_hat * gamma; the norm's
+    // backward with gamma = 1 maps it to dX
+    LMLP_TRY(mlp_backward_impl(shape, w_folded, X, g, u, sv + b.s_mlp, dOut, ws + b.dxn, grads, ws + b.mlp_b,
+                               b.b_total - b.mlp_b, stream, &f));
+    return launch_rmsnorm_bwd(shape->N, shape->d, X, nullptr, rstd, ws + b.dxn, dX, di.sms, st);
 }
 
 }  // extern "C"

@@ -8,6 +8,11 @@
 // squares ("Unsloth支持哪些模型？主流LLM兼容性一览", section 4.2).  Sums run in a
 // fixed per-lane order followed by a fixed butterfly across the warp, so the
 // results are deterministic.
+//
+// For the block with gamma folded into the gate/up weights: with y ==
+// nullptr the forward only computes rstd, and with gamma == nullptr both
+// passes take gamma = 1 (the backward then maps dy*gamma, computed by the dX
+// GEMM on the folded weights, to dx).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -15,6 +20,7 @@
 namespace lmlp {
 
 constexpr int kRmsWarps = 8;
+constexpr uint32_t kBf16One2 = 0x3F803F80u;  // two bf16 ones
 
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -71,11 +77,12 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_fwd_kernel(const __nv_
             r = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
             if (lane == 0 && rstd_out != nullptr) rstd_out[row] = r;
         }
+        if (y == nullptr) continue;
         uint4* y4 = reinterpret_cast<uint4*>(y + row * d);
         for (int c = lane; c < nc; c += 32) {
             float f[8], g[8];
             unpack8(__ldg(x4 + c), f);
-            unpack8(__ldg(g4 + c), g);
+            unpack8(gamma != nullptr ? __ldg(g4 + c) : make_uint4(kBf16One2, kBf16One2, kBf16One2, kBf16One2), g);
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] = f[i] * r * g[i];
             y4[c] = pack8(f);
@@ -99,10 +106,11 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_bwd_kernel(const __nv_
         const uint4* d4 = reinterpret_cast<const uint4*>(dy + row * d);
         const float r = rstd[row];
         float dot = 0.0f;
+        const uint4 ones = make_uint4(kBf16One2, kBf16One2, kBf16One2, kBf16One2);
         for (int c = lane; c < nc; c += 32) {
             float f[8], g[8], e[8];
             unpack8(__ldg(x4 + c), f);
-            unpack8(__ldg(g4 + c), g);
+            unpack8(gamma != nullptr ? __ldg(g4 + c) : ones, g);
             unpack8(__ldg(d4 + c), e);
 #pragma unroll
             for (int i = 0; i < 8; ++i) dot = fmaf(e[i] * g[i], f[i] * r, dot);
@@ -112,7 +120,7 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_bwd_kernel(const __nv_
         for (int c = lane; c < nc; c += 32) {
             float f[8], g[8], e[8];
             unpack8(__ldg(x4 + c), f);
-            unpack8(__ldg(g4 + c), g);
+            unpack8(gamma != nullptr ? __ldg(g4 + c) : ones, g);
             unpack8(__ldg(d4 + c), e);
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] = r * (e[i] * g[i] - f[i] * r * m);
@@ -155,7 +163,9 @@ __global__ void __launch_bounds__(kRowThreads) rmsnorm_fwd_row_kernel(const __nv
         for (int i = 0; i < NCH; ++i) {
             const int c = threadIdx.x + kRowThreads * i;
             v[i] = c < nc ? __ldg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
-            gv[i] = c < nc ? __ldg(g4 + c) : make_uint4(0u, 0u, 0u, 0u);
+            gv[i] = c < nc && y != nullptr
+                        ? (gamma != nullptr ? __ldg(g4 + c) : make_uint4(kBf16One2, kBf16One2, kBf16One2, kBf16One2))
+                        : make_uint4(0u, 0u, 0u, 0u);
         }
         float r;
         if (rstd_in != nullptr) {
@@ -173,6 +183,7 @@ __global__ void __launch_bounds__(kRowThreads) rmsnorm_fwd_row_kernel(const __nv
             r = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
             if (threadIdx.x == 0 && rstd_out != nullptr) rstd_out[row] = r;
         }
+        if (y == nullptr) continue;
         uint4* y4 = reinterpret_cast<uint4*>(y + row * d);
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
@@ -209,7 +220,8 @@ __global__ void __launch_bounds__(kRowThreads) rmsnorm_bwd_row_kernel(const __nv
             const int c = threadIdx.x + kRowThreads * i;
             xv[i] = c < nc ? __ldg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
             dv[i] = c < nc ? __ldg(d4 + c) : make_uint4(0u, 0u, 0u, 0u);
-            gv[i] = c < nc ? __ldg(g4 + c) : make_uint4(0u, 0u, 0u, 0u);
+            gv[i] = c < nc ? (gamma != nullptr ? __ldg(g4 + c) : make_uint4(kBf16One2, kBf16One2, kBf16One2, kBf16One2))
+                           : make_uint4(0u, 0u, 0u, 0u);
         }
         const float r = rstd[row];
         float dot = 0.0f;
@@ -237,6 +249,34 @@ __global__ void __launch_bounds__(kRowThreads) rmsnorm_bwd_row_kernel(const __nv
                 o4[c] = pack8(f);
             }
         }
+    }
+}
+
+// out[i, j] = bf16_rne(in[i, j] * gamma[j]) for a bf16 [rows, cols] matrix
+// (cols a multiple of 8), up to two matrices per launch (blockIdx.y): gamma
+// folded into a weight or adapter that multiplies the normalised rows.
+struct ScaleCols {
+    const __nv_bfloat16* in[2];
+    __nv_bfloat16* out[2];
+    long long rows[2];
+};
+
+__global__ void __launch_bounds__(256) scale_cols_kernel(const ScaleCols a, const __nv_bfloat16* __restrict__ gamma,
+                                                         int cols) {
+    const int z = blockIdx.y;
+    const long long n8 = a.rows[z] * (cols >> 3);
+    const uint4* in4 = reinterpret_cast<const uint4*>(a.in[z]);
+    uint4* out4 = reinterpret_cast<uint4*>(a.out[z]);
+    const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
+    const int gc = cols >> 3;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        float f[8], g[8];
+        unpack8(__ldg(in4 + i), f);
+        unpack8(__ldg(g4 + i % gc), g);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) f[k] *= g[k];
+        out4[i] = pack8(f);
     }
 }
 

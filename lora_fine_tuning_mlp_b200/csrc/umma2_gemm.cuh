@@ -205,6 +205,7 @@ struct PairProb {
     const void* in1;
     long long ld;
     int omap[3];  // tensor maps of out0..out2 for TMA stores (when the kind uses them)
+    const float* row_scale;  // EPI_SWIGLU_FWD: optional factor of each output row (see EpiOut)
 };
 
 // Tail split (stream-K for the last partial wave): the first `full_units`
@@ -652,6 +653,7 @@ __device__ __forceinline__ void pair_epilogue(const PairArgs& a, uint32_t tmem_b
     o.split_off = 0;
     o.M = P.M;
     o.N = P.N;
+    o.row_scale = P.row_scale;
     const int bn = 256 / NACC;               // columns of each accumulator
     const int gcols = bn / kGroups;          // of which this warp's group takes
     const int gcol0 = group * gcols;

@@ -78,6 +78,11 @@ struct Prob {
     void* tr0;
     void* tr1;
     long long ld_tr;
+    // Optional factor of each accumulator row m for the transposed outputs
+    // only (fp32, or bf16), applied after `scale`: the RMSNorm row scale of
+    // the pre-norm block with gamma folded into the weights.
+    const float* tr_row_scale;
+    const __nv_bfloat16* tr_row_scale_bf16;
 };
 
 struct alignas(64) GemmArgs {
@@ -406,6 +411,12 @@ __device__ __forceinline__ void splitk_finalize(const Prob& P, const Unit& t, in
 #pragma unroll
         for (int e = 0; e < 4; ++e) w[e] = pack_bf16(acc[2 * e] * P.scale, acc[2 * e + 1] * P.scale);
         if (rm != nullptr) *reinterpret_cast<uint4*>(rm + row * P.ld_rm + j) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (tr0 != nullptr && (P.tr_row_scale != nullptr || P.tr_row_scale_bf16 != nullptr)) {
+            const float rs = P.tr_row_scale != nullptr ? P.tr_row_scale[row] : __bfloat162float(P.tr_row_scale_bf16[row]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w[e] = pack_bf16(acc[2 * e] * P.scale * rs, acc[2 * e + 1] * P.scale * rs);
+        }
         if (tr0 != nullptr) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -445,6 +456,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmArgs& a, uint32_t tmem_b
         o.split_off = t.ks * P.split_stride;
         o.M = P.M;
         o.N = P.N;
+        o.row_scale = nullptr;
         const int row = t.mb * kBM + quarter * 32 + lane;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * acc_cols;
         epilogue_tile<NACC, EPI>(o, row, t.nb * a.bn, a.bn, TmemSrc{tacc});

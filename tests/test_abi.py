@@ -241,6 +241,37 @@ def test_norm_and_block_argument_errors(L):
         == _lib.ERR_INVALID_ARG
 
 
+def test_folded_block_argument_errors(L):
+    """The gamma-folded block takes bf16 frozen weights only, and the same
+    workspace and saved sizes as the unfused block."""
+    sh = shape()
+    bf, bb, _ = _lib.block_sizes(sh)
+    f, b, _ = _lib.sizes(sh)
+    assert bf >= f + 512 * 256 * 2 + 2 * 8 * 256 * 2     # normalised rows and the two A diag(gamma)
+    assert bb >= b + 2 * 512 * 256 * 2 + 2 * 8 * 256 * 2
+    assert _lib.block_fold_gamma(sh, weights(), None, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.block_fold_gamma(sh, weights(), FAKE, FAKE + 8, FAKE, None) == _lib.ERR_MISALIGNED
+    q = shape(d_ff=768, fmt=1)
+    wq = weights(Sg=FAKE, Su=FAKE, Sd=FAKE)
+    assert _lib.block_fold_gamma(q, wq, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert _lib.block_forward_folded(sh, weights(), FAKE, 1e-5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bf - 1, None) \
+        == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.block_forward_folded(sh, weights(), None, 1e-5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bf, None) \
+        == _lib.ERR_INVALID_ARG
+    assert _lib.block_forward_folded(sh, weights(), FAKE, -1.0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, bf, None) \
+        == _lib.ERR_INVALID_ARG
+    qf, qb, _ = _lib.block_sizes(q)
+    assert _lib.block_forward_folded(q, wq, FAKE, 1e-5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, qf, None) \
+        == _lib.ERR_INVALID_ARG
+    g = _lib.Grads(*([FAKE] * 6))
+    assert _lib.block_backward_folded(sh, weights(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, g, FAKE, bb - 1,
+                                      None) == _lib.ERR_WORKSPACE_TOO_SMALL
+    assert _lib.block_backward_folded(sh, weights(), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, g, FAKE, bb, None) \
+        == _lib.ERR_INVALID_ARG
+    assert _lib.block_backward_folded(q, wq, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, g, FAKE, qb, None) \
+        == _lib.ERR_INVALID_ARG
+
+
 # ----------------------------------------------------------------------------- cross-entropy
 
 

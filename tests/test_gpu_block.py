@@ -37,14 +37,16 @@ def np64(t):
     return t.float().double().cpu().numpy()
 
 
-def run_block(inp, alpha):
+def run_block(inp, alpha, folded=False):
     dev = torch.device("cuda:0")
     w = api.weights_from_host(inp, alpha, dev)
     X = api.to_device_bf16(inp["X"], dev)
     gamma = api.to_device_bf16(inp["gamma"], dev)
     dOut = api.to_device_bf16(inp["dOut"], dev)
-    out, saved = api.block_forward(X, w, gamma, EPS)
-    dX, grads = api.block_backward(X, w, gamma, saved, dOut)
+    if folded:
+        w = api.fold_gamma(w, gamma)
+    out, saved = api.block_forward(X, w, gamma, EPS, folded=folded)
+    dX, grads = api.block_backward(X, w, gamma, saved, dOut, folded=folded)
     torch.cuda.synchronize()
     assert _lib.device_status(None) == 0
     res = {"out": out, "g": saved.g, "u": saved.u, "dX": dX}
@@ -80,11 +82,12 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("folded", [False, True], ids=["norm_kernel", "gamma_folded"])
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"N{c.N}_d{c.d}_dff{c.d_ff}_r{c.r}")
-def test_block_parity_small(cfg):
+def test_block_parity_small(cfg, folded):
     inp = synth.make_block_inputs(cfg)
     ref = orn.block_forward_backward(inp, cfg.alpha, EPS)
-    got = run_block(inp, cfg.alpha)
+    got = run_block(inp, cfg.alpha, folded)
     errs = {k: relerr(got[k], ref[k]) for k in ("out", "dX") + GRADS}
     errs["g"] = relerr(got["g"], ref["G"])
     errs["u"] = relerr(got["u"], ref["U"])
@@ -114,6 +117,34 @@ def test_block_equals_its_parts_bitwise():
     assert torch.equal(dX, dX2)
     for k in GRADS:
         assert torch.equal(grads[k], grads2[k]), k
+
+
+def test_fold_gamma_is_the_rounded_column_product():
+    """fold_gamma writes bf16_rne(W[j, c] * gamma[c]) (one fp32 product,
+    exact for two bf16 factors, then one rounding) and shares the rest."""
+    cfg = synth.custom(64, 192, 320, 8, 16.0, seed_index=86)
+    inp = synth.make_block_inputs(cfg)
+    dev = torch.device("cuda:0")
+    w = api.weights_from_host(inp, cfg.alpha, dev)
+    gamma = api.to_device_bf16(inp["gamma"], dev)
+    wf = api.fold_gamma(w, gamma)
+    torch.cuda.synchronize()
+    for k in ("Wg", "Wu"):
+        exact = om.bf16_to_f64(inp[k]) * om.bf16_to_f64(inp["gamma"])[None, :]
+        want = om.f32_to_bf16_rne(exact.astype(np.float32))
+        assert np.array_equal(getattr(wf, k).view(torch.int16).cpu().numpy().view(np.uint16), want), k
+    assert wf.Wd is w.Wd and wf.Ag is w.Ag and wf.Bd is w.Bd
+
+
+def test_folded_block_is_deterministic_and_near_the_unfused_block():
+    cfg = synth.custom(1000, 512, 1408, 64, 128.0, seed_index=87)
+    inp = synth.make_block_inputs(cfg)
+    a = run_block(inp, cfg.alpha, folded=True)
+    b = run_block(inp, cfg.alpha, folded=True)
+    c = run_block(inp, cfg.alpha, folded=False)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+        assert relerr(a[k], c[k]) <= TOL, k
 
 
 def test_rmsnorm_autograd_function_matches_oracle():
@@ -157,10 +188,11 @@ def test_block_autograd_function():
 
 
 @pytest.mark.slow
-def test_block_full_size_sampled_rows():
+@pytest.mark.parametrize("folded", [False, True], ids=["norm_kernel", "gamma_folded"])
+def test_block_full_size_sampled_rows(folded):
     cfg = synth.BY_NAME["llama3_8b_mlp"]
     inp = synth.make_block_inputs(cfg)
-    got = run_block(inp, cfg.alpha)
+    got = run_block(inp, cfg.alpha, folded)
     torch.cuda.empty_cache()
     rng = np.random.default_rng(cfg.seed)
     rows = np.unique(np.concatenate([[0, cfg.N - 1], rng.choice(cfg.N, 30, replace=False)]))
