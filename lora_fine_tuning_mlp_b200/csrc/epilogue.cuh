@@ -228,27 +228,29 @@ __device__ __forceinline__ void emit_chunk(__nv_bfloat16* base, long long ld, in
     }
 }
 
-// TMA stores of 32 x 32 bf16 output blocks.  Each epilogue warp owns
-// kTmaBufs 2 KB shared-memory buffers (512-byte aligned; rows of 64 bytes in the
+// TMA stores of 32 x 32 bf16 output blocks.  Each epilogue warp owns NB
+// 2 KB shared-memory buffers (512-byte aligned; rows of 64 bytes in the
 // 64-byte swizzle: 16-byte piece q of row r sits at piece q ^ ((r / 2) % 4),
 // so the 32 lanes' row writes hit every bank once per quarter-warp) used in
-// turn; a buffer is rewritten only once the store issued from it kTmaBufs
-// stores earlier has read it.  The tensor map clips rows and columns outside
-// the output.  Warp-uniform state.
+// turn; a buffer is rewritten only once the store issued from it NB stores
+// earlier has read it.  The tensor map clips rows and columns outside the
+// output.  Warp-uniform state.
 constexpr int kTmaBufs = 3;
 constexpr uint32_t kTmaBlockBytes = 32 * 64;
 constexpr uint32_t kTmaWarpBytes = kTmaBufs * kTmaBlockBytes;
-struct TmaStore {
+template <int NB>
+struct TmaStoreN {
+    static_assert(NB >= 1 && NB <= 4, "1 to 4 store buffers a warp");
     const CUtensorMap* map[3];  // out0, out1, out2
-    uint32_t buf;               // this warp's three buffers
+    uint32_t buf;               // this warp's NB buffers
     int next;                   // buffer of the next store
     // Warp-collective: output `which`, the warp's 32 rows starting at row y
     // (lane = row; v = its 32 values), columns x .. x + 31.
     __device__ __forceinline__ void emit(int which, int x, int y, const uint4 (&v)[4]) {
         const int lane = threadIdx.x & 31;
         const uint32_t b = buf + static_cast<uint32_t>(next) * kTmaBlockBytes;
-        if (++next == kTmaBufs) next = 0;
-        if (lane == 0) bulk_wait_read<kTmaBufs - 1>();  // this buffer's last store has read it
+        if (++next == NB) next = 0;
+        if (lane == 0) bulk_wait_read<NB - 1>();  // this buffer's last store has read it
         __syncwarp();
         const uint32_t rowb = b + static_cast<uint32_t>(lane) * 64u;
         const uint32_t sw = static_cast<uint32_t>(lane >> 1) & 3u;
@@ -267,6 +269,7 @@ struct TmaStore {
         __syncwarp();
     }
 };
+using TmaStore = TmaStoreN<kTmaBufs>;
 
 // One output tile row per thread: `row` (may be >= M: stores are skipped),
 // columns [col_base, col_base + bn); accumulator a's column c is read from

@@ -133,11 +133,31 @@ __host__ __device__ constexpr int pair_epi_first() {
 #endif
 constexpr int kGuRing = LMLP_BWD_GU_RING;
 static_assert(kGuRing == 0 || kGuRing >= 2, "a ring holds at least two chunks");
-constexpr uint32_t kGuSlotBytes = 2 * kStageWarpBytes;  // g then u of one 32 x 32 chunk, 80-byte rows
+// Ring slot layout: 1 = 64-byte rows in the 64-byte swizzle (16-byte piece q
+// of row R at piece q ^ ((R / 2) mod 4)), so that both the coalesced
+// cp.async writes (two rows per quarter-warp) and the per-row reads (eight
+// rows per quarter-warp) touch every bank once; 0 = 80-byte padded rows,
+// whose cp.async writes conflict.  Measured interleaved (medians, identical
+// bits): Llama-3-8B 456 -> 453 us, TinyLlama-1.1B 802 -> 796 us, Qwen2-7B
+// 1009 -> 985 us.  A three-deep ring with two TMA-store buffers a warp (same
+// shared memory, five stages) measured within noise of it; every layout
+// that left four operand stages was 3-8 % slower.
+#ifndef LMLP_BWD_GU_SWZ
+#define LMLP_BWD_GU_SWZ 1
+#endif
+constexpr bool kGuSwz = LMLP_BWD_GU_SWZ != 0;
+constexpr uint32_t kGuHalfBytes = kGuSwz ? 32u * 64u : kStageWarpBytes;  // g (then u) of one 32 x 32 chunk
+constexpr uint32_t kGuSlotBytes = 2 * kGuHalfBytes;
 template <int EPI>
 __host__ __device__ constexpr uint32_t pair_ring_bytes() {
     return (EPI == EPI_SWIGLU_BWD && kGuRing > 0) ? pair_epi_warps<EPI>() * kGuRing * kGuSlotBytes : 0u;
 }
+// TMA-store buffers a warp of the dH epilogue cycles through (the others use
+// kTmaBufs).
+#ifndef LMLP_BWD_TMA_BUFS
+#define LMLP_BWD_TMA_BUFS 3
+#endif
+constexpr int kBwdTmaBufs = LMLP_BWD_TMA_BUFS;
 // bf16 outputs leave through TMA stores (32 x 32 blocks staged in shared
 // memory) instead of per-lane stores, by epilogue kind.  Measured
 // interleaved against the transposing per-lane stores: the SwiGLU epilogues
@@ -162,7 +182,9 @@ __host__ __device__ constexpr bool pair_tma_store() {
 // (transposes or TMA-store buffers; none for direct bf16 stores).
 template <int EPI>
 __host__ __device__ constexpr uint32_t pair_stage_warp_bytes() {
-    return pair_tma_store<EPI>() ? kTmaWarpBytes : (EPI == EPI_BF16 ? 0u : kStageWarpBytes);
+    return pair_tma_store<EPI>()
+               ? (EPI == EPI_SWIGLU_BWD && kGuRing > 0 ? kBwdTmaBufs * kTmaBlockBytes : kTmaWarpBytes)
+               : (EPI == EPI_BF16 ? 0u : kStageWarpBytes);
 }
 // Start of the epilogue's shared memory: 512-byte aligned, as the TMA-store
 // buffers' swizzle requires.
@@ -515,7 +537,7 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
     const uint32_t stg = area + static_cast<uint32_t>(warp - kFirst) * pair_stage_warp_bytes<EPI>();
     const uint32_t ring = area + pair_epi_warps<EPI>() * pair_stage_warp_bytes<EPI>() +
                           static_cast<uint32_t>(warp - kFirst) * (kGuRing * kGuSlotBytes);
-    TmaStore ts;
+    TmaStoreN<kBwdTmaBufs> ts;
     ts.map[0] = &a.maps[P.omap[0]];
     ts.map[1] = &a.maps[P.omap[1]];
     ts.map[2] = &a.maps[P.omap[2]];
@@ -538,9 +560,13 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
         }
     };
     // 16-byte piece (row 8q + lane/4, columns 8 (lane%4) ..) of a chunk, as in
-    // a coalesced load: four lanes cover one row's 64 bytes.
+    // a coalesced load: four lanes cover one row's 64 bytes.  With the
+    // swizzled slots, rows 8q + lane/4 have (row / 2) mod 4 = (lane / 8) mod 4.
     const int prow = lane >> 2, pcol = 8 * (lane & 3);
-    const uint32_t poff = static_cast<uint32_t>(prow) * kStageRowBytes + static_cast<uint32_t>(lane & 3) * 16u;
+    constexpr uint32_t kRowB = kGuSwz ? 64u : kStageRowBytes;
+    const uint32_t ppiece = kGuSwz ? ((static_cast<uint32_t>(lane & 3) ^ (static_cast<uint32_t>(lane >> 3) & 3u)) << 4)
+                                   : static_cast<uint32_t>(lane & 3) * 16u;
+    const uint32_t poff = static_cast<uint32_t>(prow) * kRowB + ppiece;
     auto issue = [&]() {
         if (iu < a.total_units) {
             const uint32_t sb = ring + islot * kGuSlotBytes + poff;
@@ -550,8 +576,8 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
                 const int r = irow0 + 8 * q + prow;
                 const bool ok = r < P.M && cc < P.N;
                 const long long off = ok ? static_cast<long long>(r) * P.ld + cc : 0;
-                cp_async16(sb + q * 8 * kStageRowBytes, gbase + off, ok ? 16u : 0u);
-                cp_async16(sb + kStageWarpBytes + q * 8 * kStageRowBytes, ubase + off, ok ? 16u : 0u);
+                cp_async16(sb + q * 8 * kRowB, gbase + off, ok ? 16u : 0u);
+                cp_async16(sb + kGuHalfBytes + q * 8 * kRowB, ubase + off, ok ? 16u : 0u);
             }
             if (++ich == nch) {
                 ich = 0;
@@ -588,12 +614,14 @@ __device__ __forceinline__ void pair_epilogue_bwd_ring(const PairArgs& a, uint32
             if (col0 < P.N) {  // warp-uniform
                 uint32_t v[32];
                 tmem_ld32(tacc + ch * 32, v);
-                const uint32_t rb = ring + cslot * kGuSlotBytes + static_cast<uint32_t>(lane) * kStageRowBytes;
+                const uint32_t rb = ring + cslot * kGuSlotBytes + static_cast<uint32_t>(lane) * kRowB;
+                const uint32_t rsw = kGuSwz ? (static_cast<uint32_t>(lane >> 1) & 3u) : 0u;
                 uint4 gv[4], uv[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    gv[q] = lds128(rb + q * 16);
-                    uv[q] = lds128(rb + kStageWarpBytes + q * 16);
+                    const uint32_t pq = (static_cast<uint32_t>(q) ^ rsw) << 4;
+                    gv[q] = lds128(rb + pq);
+                    uv[q] = lds128(rb + kGuHalfBytes + pq);
                 }
                 tmem_ld_wait();
                 uint4 dgq[4], duq[4], hq[4];
