@@ -39,6 +39,7 @@
 #include "ptx.cuh"
 #include "umma_gemm.cuh"
 #include "umma2_gemm.cuh"
+#include "lowrank_dual.cuh"
 
 using namespace lmlp;
 
@@ -633,6 +634,23 @@ int launch_scale_t(int qf, int n, const void* const* src, void* const* dst, cons
                         : launch_scale_t_typed<unsigned short>(n, src, dst, rows, cols, st);
 }
 
+// Bg, Bu [dff, r] -> Bg^T, Bu^T [r, dff] (the K-major B operands of the
+// single-pass adapter-gradient launch), one launch.
+int launch_adapter_t(const void* Bg, const void* Bu, void* BgT, void* BuT, int64_t dff, int64_t r, cudaStream_t st) {
+    ScaleT<unsigned short> a{};
+    a.src[0] = static_cast<const unsigned short*>(Bg);
+    a.src[1] = static_cast<const unsigned short*>(Bu);
+    a.dst[0] = static_cast<unsigned short*>(BgT);
+    a.dst[1] = static_cast<unsigned short*>(BuT);
+    a.rows[0] = a.rows[1] = static_cast<int>(dff);
+    a.nb[0] = a.nb[1] = static_cast<int>(r);
+    {
+        LaunchScope scope("B_mid_adapter_t", st);
+        scale_transpose_kernel<unsigned short><<<dim3(static_cast<unsigned>((dff + 31) / 32), 2), 256, 0, st>>>(a);
+    }
+    return last_launch_error();
+}
+
 // ----------------------------------------------------------------------------- layout
 // Split-K factors for the skinny problems of one launch.  All problems of a
 // launch are cut into units of about T K blocks (problem p gets
@@ -705,6 +723,11 @@ struct Plan {
     size_t f_h, f_sgu, f_sd, f_part, f_ctr, f_tail, f_st[3], f_total;  // f_st: block scales, transposed
     // backward workspace
     size_t b_dg, b_du, b_h, b_td, b_tdT, b_tgu, b_tguT, b_part, b_ctr, b_tail, b_st[3], b_total;
+    // single-pass adapter-gradient launch (ranks <= 32): its partition and
+    // buffers (Bg^T | Bu^T, the dB and T partial sums)
+    bool dual;
+    int dual_ntb, dual_ntr, dual_fchunks;
+    size_t b_bT, b_pdb, b_pt;
     size_t ctr_bytes;  // per-tile split-K counters (zeroed at the start of each call)
     // saved
     size_t s_sgT, s_suT, s_sdT, s_total;
@@ -718,6 +741,41 @@ struct Carver {
         return o;
     }
 };
+
+// Partition of the single-pass adapter-gradient launch (lowrank_dual.cuh):
+// n_tb token blocks per token range (at most kDualMaxTb, for TMEM), as many
+// feature ranges per token range as fill 148 SMs.  Chosen by an estimate of
+// its time: the busiest CTA's bytes at one SM's share of HBM, or all of them
+// at HBM's rate, whichever is longer, plus the partial sums written and read
+// back.  Depends only on the shape.
+#ifndef LMLP_DUAL
+#define LMLP_DUAL 1  // 0: the adapter-gradient launch as five split-K problems (two reads of dg, du)
+#endif
+void dual_plan(Plan& p) {
+    p.dual = false;
+    if (!LMLP_DUAL || p.r > kDualBN) return;
+    const int64_t tiles_t = ceil_div(p.N, 128), tiles_f = ceil_div(p.d_ff, 128);
+    const double kSmRate = 45e9, kHbmRate = 6.5e12;
+    const double tile_bytes = 3.0 * kDualA + 2.0 * kDualBT + 3.0 * kDualBD;  // one (token, feature) block, 3 matrices
+    double best = 1e300;
+    for (int ntb = 1; ntb <= kDualMaxTb; ++ntb) {
+        const int64_t ntr = ceil_div(tiles_t, ntb);
+        if (ntr > kTargetCtas) continue;
+        const int64_t fch = std::min<int64_t>(tiles_f, kTargetCtas / ntr);
+        if (fch < 1) continue;
+        const int64_t per_cta = std::min<int64_t>(ntb, tiles_t) * ceil_div(tiles_f, fch);
+        const double stream = std::max(per_cta * tile_bytes / kSmRate, tiles_t * tiles_f * tile_bytes / kHbmRate);
+        const double partial = 4.0 * (ntr * 3.0 * p.d_ff * p.r + fch * 2.0 * p.N * p.r);
+        const double est = stream + 2.0 * partial / kHbmRate;
+        if (est < best) {
+            best = est;
+            p.dual = true;
+            p.dual_ntb = ntb;
+            p.dual_ntr = static_cast<int>(ntr);
+            p.dual_fchunks = static_cast<int>(fch);
+        }
+    }
+}
 
 Plan make_plan(const lora_mlp_shape& sh) {
     Plan p{};
@@ -791,6 +849,12 @@ Plan make_plan(const lora_mlp_shape& sh) {
     p.b_ctr = b.take(p.ctr_bytes);
     p.b_tail = b.take(kTailPartFloats * f32);
     for (int i = 0; i < 3; ++i) p.b_st[i] = p.qf ? b.take(stsz) : 0;
+    dual_plan(p);
+    if (p.dual) {
+        p.b_bT = kDualBtMn ? 0 : b.take(2 * rz * fz * bf);
+        p.b_pdb = b.take(static_cast<size_t>(p.dual_ntr) * 3 * fz * rz * f32);
+        p.b_pt = b.take(static_cast<size_t>(p.dual_fchunks) * Nz * 2 * rz * f32);
+    }
     p.b_total = b.off;
 
     Carver sv;
@@ -804,6 +868,95 @@ Plan make_plan(const lora_mlp_shape& sh) {
 
 // ----------------------------------------------------------------------------- validation
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The single-pass adapter-gradient launch and the launch that sums its
+// partials (lowrank_dual.cuh).  row_scale: optional factor per token of the
+// transposed T outputs.
+int launch_dual(const Plan& pl, const void* dg, const void* du, const void* h, const void* BgT, const void* BuT,
+                const void* SgT, const void* SuT, const void* TdT, uint8_t* ws, const lora_mlp_grads* grads,
+                void* Tgu, void* TguT, const float* row_scale, cudaStream_t st) {
+    DualArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int64_t N = pl.N, dff = pl.d_ff, r = pl.r, ldN = pl.ldN;
+    bool ok = true;
+    const void* mats[3] = {dg, du, h};
+    for (int m = 0; m < 3; ++m) ok = ok && encode_map(&a.maps[m], mats[m], dff, N, dff, 64, 128);
+    if (kDualBtMn) {
+        ok = ok && encode_map(&a.maps[3], BgT, r, dff, r, 64, 64);
+        ok = ok && encode_map(&a.maps[4], BuT, r, dff, r, 64, 64);
+    } else {
+        ok = ok && encode_map(&a.maps[3], BgT, dff, r, dff, 64, kDualBN);
+        ok = ok && encode_map(&a.maps[4], BuT, dff, r, dff, 64, kDualBN);
+    }
+    const void* bd[3] = {SgT, SuT, TdT};
+    for (int m = 0; m < 3; ++m) ok = ok && encode_map(&a.maps[5 + m], bd[m], N, r, ldN, 64, kDualBN);
+    if (!ok) return LORA_MLP_ERR_CUDA;
+    a.nmaps = 8;
+    a.N = static_cast<int>(N);
+    a.dff = static_cast<int>(dff);
+    a.r = static_cast<int>(r);
+    a.n_tb = pl.dual_ntb;
+    a.n_tr = pl.dual_ntr;
+    a.fchunks = pl.dual_fchunks;
+    a.tiles_t = ceil_div(N, 128);
+    a.tiles_f = ceil_div(dff, 128);
+    a.part_db = reinterpret_cast<float*>(ws + pl.b_pdb);
+    a.part_t = reinterpret_cast<float*>(ws + pl.b_pt);
+    a.wait_limit = g_wait_limit.load();
+    a.force_timeout = g_force_timeout.load();
+    const size_t smem = 1024 + static_cast<size_t>(kDualStages) * kDualStage + gemm_ctl_bytes();
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(dual_lowrank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+            cudaSuccess)
+            return LORA_MLP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.n_tr * a.fchunks), 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = LMLP_PDL ? 1 : 0;
+    cudaError_t err;
+    {
+        LaunchScope scope("B_mid_lowrank_grads", st);
+        err = cudaLaunchKernelEx(&cfg, dual_lowrank_kernel, a);
+    }
+    if (err != cudaSuccess || last_launch_error() != LORA_MLP_OK) return LORA_MLP_ERR_CUDA;
+    DualFin f{};
+    f.part_db = a.part_db;
+    f.part_t = a.part_t;
+    f.dBg = static_cast<__nv_bfloat16*>(grads->dBg);
+    f.dBu = static_cast<__nv_bfloat16*>(grads->dBu);
+    f.dAd = static_cast<__nv_bfloat16*>(grads->dAd);
+    f.Tgu = static_cast<__nv_bfloat16*>(Tgu);
+    f.TguT = static_cast<__nv_bfloat16*>(TguT);
+    f.row_scale = row_scale;
+    f.ldN = ldN;
+    f.N = a.N;
+    f.dff = a.dff;
+    f.r = a.r;
+    f.n_tr = a.n_tr;
+    f.fchunks = a.fchunks;
+    f.s = pl.s;
+    f.db_blocks = ceil_div(3 * dff * (r / 4), kDualFinThreads);
+    cfg.gridDim = dim3(static_cast<unsigned>(f.db_blocks + ceil_div(N * (r / 2), kDualFinThreads)), 1, 1);
+    cfg.blockDim = dim3(kDualFinThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    {
+        LaunchScope scope("B_mid_finalize", st);
+        err = cudaLaunchKernelEx(&cfg, dual_finalize_kernel, f);
+    }
+    if (err != cudaSuccess) return LORA_MLP_ERR_CUDA;
+    return last_launch_error();
+}
 
 int validate_shape(const lora_mlp_shape* sh) {
     if (sh == nullptr) return LORA_MLP_ERR_INVALID_ARG;
@@ -1045,6 +1198,13 @@ static int mlp_backward_impl(const lora_mlp_shape* shape, const lora_mlp_weights
     const void* SgT = sv + pl.s_sgT;
     const void* SuT = sv + pl.s_suT;
     const void* SdT = sv + pl.s_sdT;
+    if (pl.dual && !kDualBtMn) {
+        // Bg^T, Bu^T for the single-pass adapter-gradient launch: they depend
+        // on the weights only, so this runs first, off the chain of launches
+        // that depend on each other's outputs
+        __nv_bfloat16* BgT = reinterpret_cast<__nv_bfloat16*>(ws + pl.b_bT);
+        LMLP_TRY(launch_adapter_t(w->Bg, w->Bu, BgT, BgT + r * dff, dff, r, st));
+    }
     // adapter B matrices as K-major operands of the rank-r projections
     {  // B0: T_d = s dOut Bd -> Td [N, r], Td^T [r, ldN];  dBd = dOut^T S_d
         const int* sp = pl.splits[SK_B0];
@@ -1088,7 +1248,11 @@ static int mlp_backward_impl(const lora_mlp_shape* shape, const lora_mlp_weights
         }
         LMLP_TRY((launch_pair_q<true, EPI_SWIGLU_BWD>(b, pl.qf, di.sms, st, "B1_dh_swiglu_bwd", tailp, ctr)));
     }
-    {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
+    if (pl.dual) {  // B-mid in one pass over dg, du and h (ranks <= 32)
+        const __nv_bfloat16* BgT = reinterpret_cast<const __nv_bfloat16*>(ws + pl.b_bT);
+        LMLP_TRY(launch_dual(pl, dg, du, hb, kDualBtMn ? w->Bg : BgT, kDualBtMn ? w->Bu : BgT + r * dff, SgT, SuT,
+                             TdT, ws, grads, Tgu, TguT, fold != nullptr ? fold->rstd : nullptr, st));
+    } else {  // B-mid: T_g = s dg Bg, T_u = s du Bu -> Tgu [N, 2r], Tgu^T [2r, ldN];
        //        dAd = T_d^T h (written transposed);  dBg = dg^T S_g, dBu = du^T S_u
         const int* sp = pl.splits[SK_BMID];
         const size_t* po = pl.part_off[SK_BMID];
