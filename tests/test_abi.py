@@ -55,6 +55,19 @@ def test_sizes_are_positive_and_grow_with_N(L):
     assert b1 >= 3 * 512 * 704 * 2
 
 
+def test_one_pass_adapter_gradient_buffers_only_for_ranks_up_to_32(L):
+    """Ranks <= 32 run the adapter-gradient reductions in one pass and keep
+    their fp32 partial sums in the backward workspace: at least one token
+    range's dB part (3 x d_ff x r) and one feature range's T part (N x 2r);
+    rank 40 (> 32) keeps the split-K form, whose workspace is smaller than
+    rank 32's although its rank is larger."""
+    N, d, dff = 4096, 4096, 14336
+    bw = {r: _lib.sizes(shape(N=N, d=d, d_ff=dff, r=r))[1] for r in (16, 32, 40)}
+    for r in (16, 32):
+        assert bw[r] >= 3 * N * dff * 2 + 4 * (3 * dff * r + N * 2 * r)
+    assert bw[40] < bw[32]
+
+
 def test_int4_workspace_holds_no_dequantised_weight(L):
     with pytest.raises(_lib.LoraMLPError) as e:
         _lib.sizes(shape(d=256, d_ff=712, fmt=1))   # 712 is not a multiple of 64
