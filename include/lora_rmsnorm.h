@@ -76,7 +76,7 @@ int lora_mlp_block_backward(const lora_mlp_shape* shape, const lora_mlp_weights*
  * A diag(gamma) (formed each call, A being trainable) the same way.  The
  * backward's dX GEMM on the folded weights yields dx_hat * gamma, which the
  * norm's backward maps to dX; the adapter gradients take the rstd and gamma
- * factors in their split-K finalisation.  Results match the unfused block up
+ * factors where their partial sums are finalised.  Results match the unfused block up
  * to the rounding of the folded weights and the order of the products.
  * Workspace and saved sizes: lora_mlp_block_sizes.
  */
@@ -90,13 +90,16 @@ int lora_mlp_block_fold_gamma(const lora_mlp_shape* shape, const lora_mlp_weight
 /* Block forward with the folded weights: w_folded is w with Wg, Wu replaced
  * by the outputs of lora_mlp_block_fold_gamma (Wd and the adapters
  * unchanged); gamma, eps, X and the outputs as in lora_mlp_block_forward.
+ * bf16 frozen weights only (LORA_MLP_ERR_INVALID_ARG otherwise).
  * Launches: rstd only, A diag(gamma) for both adapters, then the MLP's. */
 int lora_mlp_block_forward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded,
                                   const void* gamma, float eps, const void* X, void* out, void* g, void* u,
                                   void* saved, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Block backward with the folded weights; arguments as in
- * lora_mlp_block_backward, `saved` from lora_mlp_block_forward_folded. */
+ * lora_mlp_block_backward, `saved` from lora_mlp_block_forward_folded; bf16
+ * frozen weights only.  Launches: A diag(gamma) for both adapters, the
+ * MLP's backward, then the norm's backward with gamma = 1. */
 int lora_mlp_block_backward_folded(const lora_mlp_shape* shape, const lora_mlp_weights* w_folded,
                                    const void* gamma, const void* X, const void* g, const void* u,
                                    const void* saved, const void* dOut, void* dX, const lora_mlp_grads* grads,
