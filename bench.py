@@ -60,7 +60,9 @@ def load_peaks():
 def csrc_sha256() -> str:
     """Hash of the translation unit the GEMM kernels are built from (lora_mlp.cu
     and every local file it includes, transitively), to tell whether a stored
-    ncu figure still applies to the kernels this build runs."""
+    ncu figure still applies to the kernels this build runs.  Comments and
+    blank space are left out, so that an edit to documentation alone keeps
+    the figure."""
     import hashlib
     import re as _re
     csrc = os.path.join(ROOT, "lora_fine_tuning_mlp_b200", "csrc")
@@ -82,7 +84,8 @@ def csrc_sha256() -> str:
         path = next(os.path.join(dd, f) for dd in (csrc, inc) if os.path.exists(os.path.join(dd, f)))
         h.update(f.encode())
         with open(path, "rb") as fh:
-            h.update(fh.read())
+            code = _re.sub(rb"/\*.*?\*/|//[^\n]*", b" ", fh.read(), flags=_re.S)
+        h.update(b" ".join(code.split()))
     return h.hexdigest()
 
 
