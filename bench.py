@@ -60,9 +60,9 @@ def load_peaks():
 def csrc_sha256() -> str:
     """Hash of the translation unit the GEMM kernels are built from (lora_mlp.cu
     and every local file it includes, transitively), to tell whether a stored
-    ncu figure still applies to the kernels this build runs.  Comments and
-    blank space are left out, so that an edit to documentation alone keeps
-    the figure."""
+    ncu figure still applies to the kernels the current sources compile to.
+    Comments and blank space are left out, so that an edit to documentation
+    alone keeps the figure."""
     import hashlib
     import re as _re
     csrc = os.path.join(ROOT, "lora_fine_tuning_mlp_b200", "csrc")

@@ -1,8 +1,8 @@
 """bench.py reports a kernel's DRAM traffic from the committed ncu summary
-only while the kernels it was taken from are the ones this build runs.  The
-fingerprint is the GEMM translation unit with comments and blank space left
-out: an edit to comments keeps it, an edit to code changes it.  Host logic
-only (no GPU)."""
+only while the kernels it was taken from are the ones the sources compile
+to.  The fingerprint is the GEMM translation unit with comments and blank
+space left out: an edit to comments keeps it, an edit to code changes it.
+Host logic only (no GPU)."""
 import importlib
 import os
 import shutil
